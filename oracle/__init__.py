@@ -1,0 +1,13 @@
+"""fp64 CPU oracle for the sparse MoE feed-forward layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the CPU-baseline leg
+of the benchmark are the only callers.  The product path never imports this
+package, and this package imports nothing from the product.
+"""
+from .oracle import (  # noqa: F401
+    build,
+    num_threads,
+    route,
+    forward,
+    swiglu,
+)

@@ -1,0 +1,282 @@
+/*
+ * moe_oracle.c -- fp64 CPU oracle for the forward pass of a Mixtral-style
+ * sparse Mixture-of-Experts feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may load this file
+ * or the library built from it: only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark do.  It shares no code, header, table or
+ * helper with the CUDA library; it reads the same bf16 input bits and nothing
+ * else.
+ *
+ * What it computes, per token t (a plain restatement of the method, evaluated
+ * token by token in double precision with no intermediate rounding):
+ *
+ *   l[e]   = sum_i x[t,i] * Wg[e,i]  (+ bias[e] when a bias is given)
+ *       -- the router is a bias-free linear layer d -> E
+ *          ("Mistral 8x7B SMoE ..." (jsqmd.com) sec. 3.2 Gating Network;
+ *           "MoE: ..." (theaiera.top, LLMs-from-scratch ch.10) sec. 10.3)
+ *   sel    = the k experts with the largest l, ordered by (l descending,
+ *            expert index ascending): equal logits go to the lower index
+ *       -- torch.topk in sec. 10.3 / sec. 3.2; the pages fix no tie rule,
+ *          the lower-index rule is the reading this library adopts
+ *   w[j]   = exp(l[sel[j]] - m) / sum_j' exp(l[sel[j']] - m),  m = l[sel[0]]
+ *       -- softmax over the k selected logits only, so the weights sum to 1
+ *          (sec. 10.3; sec. 3.2 step 3)
+ *   h_e[f] = silu(sum_i W1[e,f,i] x[t,i]) * (sum_i W3[e,f,i] x[t,i])
+ *   y_e[o] = sum_f W2[e,o,f] h_e[f]
+ *       -- the SwiGLU expert w2(silu(w1 x) * w3 x)
+ *          ("Mistral 8x7B SMoE ..." sec. 3.1 FeedForward;
+ *           "Mixtral and MoE architecture" (astro-blog) FeedForward listing)
+ *   out[t] = sum_j w[j] * y_{sel[j]}   summed in slot order j = 0..k-1
+ *            (+ the shared expert's SwiGLU output, unweighted, when given)
+ *       -- weighted scatter-add back to token order and the always-on shared
+ *          expert (sec. 10.4 and sec. 10.5 of the theaiera.top chapter)
+ *   silu(z) = z / (1 + exp(-z))
+ *
+ * Sums run in index order with one accumulator; OpenMP only splits the
+ * independent tokens across threads and changes no arithmetic.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Widen raw bf16 bits to double; exact (bf16 is the top half of a float). */
+static double bf16_bits_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* Router for one token: logits, the selected set, the softmax weights over
+ * that set and the gap between the k-th and (k+1)-th largest logits
+ * (+inf when k == E).  The selection is k rounds of "largest remaining
+ * logit"; a strict '>' keeps the lower index on equal values. */
+static void route_one(int d, int E, int k, const double *xt, const uint16_t *Wg,
+                      const double *bias, double *l, int32_t *sel, double *w,
+                      double *gap, unsigned char *taken)
+{
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        const uint16_t *row = Wg + (size_t)e * d;
+        for (int i = 0; i < d; ++i) acc += xt[i] * bf16_bits_to_double(row[i]);
+        if (bias) acc += bias[e];
+        l[e] = acc;
+        taken[e] = 0;
+    }
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e)
+            if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+        sel[j] = best;
+        taken[best] = 1;
+    }
+    if (gap) {
+        if (k < E) {
+            int next = -1;
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && (next < 0 || l[e] > l[next])) next = e;
+            *gap = l[sel[k - 1]] - l[next];
+        } else {
+            *gap = INFINITY;
+        }
+    }
+    double m = l[sel[0]];
+    double s = 0.0;
+    for (int j = 0; j < k; ++j) {
+        w[j] = exp(l[sel[j]] - m);
+        s += w[j];
+    }
+    for (int j = 0; j < k; ++j) w[j] /= s;
+}
+
+/* One SwiGLU expert on one token: y = W2 (silu(W1 x) * (W3 x)).
+ * W1, W3 are [dff, d] and W2 is [d, dff], row-major (nn.Linear's [out, in]). */
+static void swiglu_one(int d, int dff, const uint16_t *W1, const uint16_t *W3,
+                       const uint16_t *W2, const double *xt, double *h, double *y)
+{
+    for (int f = 0; f < dff; ++f) {
+        const uint16_t *r1 = W1 + (size_t)f * d;
+        const uint16_t *r3 = W3 + (size_t)f * d;
+        double a = 0.0, b = 0.0;
+        for (int i = 0; i < d; ++i) a += bf16_bits_to_double(r1[i]) * xt[i];
+        for (int i = 0; i < d; ++i) b += bf16_bits_to_double(r3[i]) * xt[i];
+        h[f] = silu(a) * b;
+    }
+    for (int o = 0; o < d; ++o) {
+        const uint16_t *r2 = W2 + (size_t)o * dff;
+        double acc = 0.0;
+        for (int f = 0; f < dff; ++f) acc += bf16_bits_to_double(r2[f]) * h[f];
+        y[o] = acc;
+    }
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Routing for all T tokens.
+ *   x [T,d], Wg [E,d] : bf16 bits;  bias [E] or NULL (added to the logits
+ *   before both the selection and the softmax)
+ *   idx [T,k] int32, w [T,k], gap [T] (may be NULL), logits [T,E] (may be
+ *   NULL), counts [E] (may be NULL): number of (token, slot) pairs per expert.
+ * Returns 0, or -1 on bad arguments. */
+int oracle_route(int T, int d, int E, int k, const uint16_t *x, const uint16_t *Wg,
+                 const double *bias, int32_t *idx, double *w, double *gap,
+                 double *logits, int64_t *counts)
+{
+    if (T < 0 || d < 1 || E < 1 || k < 1 || k > E || !x || !Wg || !idx || !w) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *l = (double *)malloc(sizeof(double) * (size_t)E);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        if (!xt || !l || !taken) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (int t = 0; t < T; ++t) {
+                for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)t * d + i]);
+                route_one(d, E, k, xt, Wg, bias, l, idx + (size_t)t * k, w + (size_t)t * k,
+                          gap ? gap + t : NULL, taken);
+                if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);
+            }
+        }
+        free(xt);
+        free(l);
+        free(taken);
+    }
+    if (err) return -1;
+    if (counts) {
+        for (int e = 0; e < E; ++e) counts[e] = 0;
+        for (size_t s = 0; s < (size_t)T * k; ++s) counts[idx[s]] += 1;
+    }
+    return 0;
+}
+
+/* Layer output for n selected tokens.
+ *   tokens [n] : token indices into x (NULL means tokens 0..n-1)
+ *   x [T,d], Wg [E,d], W1/W3 [E,dff,d], W2 [E,d,dff] : bf16 bits
+ *   bias [E] or NULL
+ *   dffs > 0 with Ws1/Ws3 [dffs,d], Ws2 [d,dffs]: shared expert, added with
+ *   weight 1; dffs == 0 means no shared expert
+ *   forced [n,k] or NULL: when given, token r uses experts forced[r,*] in that
+ *   order instead of its own top-k; the weights are still the softmax over
+ *   those experts' logits.  This re-evaluates a token with another set
+ *   (used where the k-th and (k+1)-th logits nearly tie).
+ *   out [n,d] double.
+ * Returns 0, or -1 on bad arguments. */
+int oracle_forward(int n, const int32_t *tokens, int T, int d, int E, int dff, int k,
+                   const uint16_t *x, const uint16_t *Wg, const double *bias,
+                   const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
+                   int dffs, const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
+                   const int32_t *forced, double *out)
+{
+    if (n < 0 || T < 1 || d < 1 || E < 1 || dff < 1 || k < 1 || k > E) return -1;
+    if (!x || !Wg || !W1 || !W3 || !W2 || !out) return -1;
+    if (dffs < 0 || (dffs > 0 && (!Ws1 || !Ws3 || !Ws2))) return -1;
+    for (int r = 0; r < n; ++r) {
+        int t = tokens ? tokens[r] : r;
+        if (t < 0 || t >= T) return -1;
+        if (forced)
+            for (int j = 0; j < k; ++j)
+                if (forced[(size_t)r * k + j] < 0 || forced[(size_t)r * k + j] >= E) return -1;
+    }
+    int hmax = dff > dffs ? dff : dffs;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *l = (double *)malloc(sizeof(double) * (size_t)E);
+        double *h = (double *)malloc(sizeof(double) * (size_t)hmax);
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
+        double *w = (double *)malloc(sizeof(double) * (size_t)k);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        if (!xt || !l || !h || !y || !w || !sel || !taken) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r) {
+                int t = tokens ? tokens[r] : r;
+                for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)t * d + i]);
+                route_one(d, E, k, xt, Wg, bias, l, sel, w, NULL, taken);
+                if (forced) {
+                    /* softmax over the forced experts' logits, in forced order */
+                    double m = -INFINITY, s = 0.0;
+                    for (int j = 0; j < k; ++j) {
+                        sel[j] = forced[(size_t)r * k + j];
+                        if (l[sel[j]] > m) m = l[sel[j]];
+                    }
+                    for (int j = 0; j < k; ++j) {
+                        w[j] = exp(l[sel[j]] - m);
+                        s += w[j];
+                    }
+                    for (int j = 0; j < k; ++j) w[j] /= s;
+                }
+                double *o = out + (size_t)r * d;
+                for (int i = 0; i < d; ++i) o[i] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    int e = sel[j];
+                    swiglu_one(d, dff, W1 + (size_t)e * dff * d, W3 + (size_t)e * dff * d,
+                               W2 + (size_t)e * d * dff, xt, h, y);
+                    for (int i = 0; i < d; ++i) o[i] += w[j] * y[i];
+                }
+                if (dffs > 0) {
+                    swiglu_one(d, dffs, Ws1, Ws3, Ws2, xt, h, y);
+                    for (int i = 0; i < d; ++i) o[i] += y[i];
+                }
+            }
+        }
+        free(xt);
+        free(l);
+        free(h);
+        free(y);
+        free(w);
+        free(sel);
+        free(taken);
+    }
+    return err ? -1 : 0;
+}
+
+/* One SwiGLU expert applied to n rows (no routing): out[r] = W2(silu(W1 x_r) * W3 x_r).
+ * Used to check the expert FFN by itself. */
+int oracle_swiglu(int n, int d, int dff, const uint16_t *x, const uint16_t *W1,
+                  const uint16_t *W3, const uint16_t *W2, double *out)
+{
+    if (n < 0 || d < 1 || dff < 1 || !x || !W1 || !W3 || !W2 || !out) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *h = (double *)malloc(sizeof(double) * (size_t)dff);
+        if (!xt || !h) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r) {
+                for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)r * d + i]);
+                swiglu_one(d, dff, W1, W3, W2, xt, h, out + (size_t)r * d);
+            }
+        }
+        free(xt);
+        free(h);
+    }
+    return err ? -1 : 0;
+}

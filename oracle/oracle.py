@@ -1,0 +1,137 @@
+"""ctypes front end of the fp64 C oracle (``moe_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY -- see ``moe_oracle.c`` for what is computed and
+which passages of the pages each step follows.  Inputs are numpy ``uint16``
+arrays holding raw bf16 bits (the exact bits the GPU library receives);
+outputs are float64 / int32 numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def build(force: bool = False) -> str:
+    """Compile ``moe_oracle.c`` with gcc (OpenMP across tokens, no fast-math,
+    no FMA contraction) into ``libmoe_oracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+             "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"],
+            check=True,
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        # MOE_ORACLE_LIB points the tests' mutation check at a deliberately
+        # broken copy of the oracle; normally the library is built from source.
+        path = os.environ.get("MOE_ORACLE_LIB") or build()
+        lib = ctypes.CDLL(path)
+        lib.oracle_num_threads.restype = _I
+        lib.oracle_route.restype = _I
+        lib.oracle_route.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]
+        lib.oracle_forward.restype = _I
+        lib.oracle_forward.argtypes = [_I, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                       _I, _P, _P, _P, _P, _P]
+        lib.oracle_swiglu.restype = _I
+        lib.oracle_swiglu.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P]
+        _lib = lib
+    return _lib
+
+
+def _bits(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are raw bf16 bits (numpy uint16)")
+    return a
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_P)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def route(x, Wg, k: int, bias=None):
+    """Router of every token.  Returns dict with ``idx`` [T,k] int32, ``w``
+    [T,k] f64, ``gap`` [T] f64 (k-th minus (k+1)-th logit, inf if k == E),
+    ``logits`` [T,E] f64 and ``counts`` [E] int64."""
+    x, Wg = _bits(x), _bits(Wg)
+    T, d = x.shape
+    E = Wg.shape[0]
+    assert Wg.shape[1] == d
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    gap = np.empty((T,), np.float64)
+    logits = np.empty((T, E), np.float64)
+    counts = np.empty((E,), np.int64)
+    rc = _load().oracle_route(T, d, E, k, _ptr(x), _ptr(Wg), _ptr(b), _ptr(idx), _ptr(w),
+                              _ptr(gap), _ptr(logits), _ptr(counts))
+    if rc != 0:
+        raise ValueError("oracle_route rejected its arguments")
+    return {"idx": idx, "w": w, "gap": gap, "logits": logits, "counts": counts}
+
+
+def forward(x, Wg, W1, W3, W2, k: int, bias=None, tokens=None, shared=None, forced=None):
+    """Layer output (f64) for ``tokens`` (default: all).  ``shared`` is an
+    optional (Ws1, Ws3, Ws2) triple of the always-on expert; ``forced`` an
+    optional [n,k] int array of experts to use instead of the token's top-k."""
+    x, Wg, W1, W3, W2 = (_bits(a) for a in (x, Wg, W1, W3, W2))
+    T, d = x.shape
+    E, dff = W1.shape[0], W1.shape[1]
+    assert Wg.shape == (E, d) and W1.shape == (E, dff, d) and W3.shape == (E, dff, d)
+    assert W2.shape == (E, d, dff)
+    tok = None
+    if tokens is not None:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = tok.shape[0]
+    else:
+        n = T
+    dffs, Ws1, Ws3, Ws2 = 0, None, None, None
+    if shared is not None:
+        Ws1, Ws3, Ws2 = (_bits(a) for a in shared)
+        dffs = Ws1.shape[0]
+        assert Ws1.shape == (dffs, d) and Ws3.shape == (dffs, d) and Ws2.shape == (d, dffs)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+    f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
+    if f is not None:
+        assert f.shape == (n, k)
+    out = np.empty((n, d), np.float64)
+    rc = _load().oracle_forward(n, _ptr(tok), T, d, E, dff, k, _ptr(x), _ptr(Wg), _ptr(b),
+                                _ptr(W1), _ptr(W3), _ptr(W2), dffs, _ptr(Ws1), _ptr(Ws3),
+                                _ptr(Ws2), _ptr(f), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_forward rejected its arguments")
+    return out
+
+
+def swiglu(x, W1, W3, W2):
+    """One SwiGLU expert applied to every row of x (f64 result)."""
+    x, W1, W3, W2 = (_bits(a) for a in (x, W1, W3, W2))
+    n, d = x.shape
+    dff = W1.shape[0]
+    assert W1.shape == (dff, d) and W3.shape == (dff, d) and W2.shape == (d, dff)
+    out = np.empty((n, d), np.float64)
+    rc = _load().oracle_swiglu(n, d, dff, _ptr(x), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_swiglu rejected its arguments")
+    return out

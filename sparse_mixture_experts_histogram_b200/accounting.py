@@ -1,0 +1,92 @@
+"""Parameter, FLOP and byte accounting of the sparse MoE layer.
+
+Closed forms, stated on the pages and used to turn measured times into
+throughput and roofline fractions:
+
+* a SwiGLU feed-forward of width d_hidden holds 3 * d * d_hidden parameters
+  (2 matrices for GELU): "MoE: ..." (theaiera.top) sec. 10.6 estimator;
+* the router holds d * E parameters (same section);
+* one MoE layer holds 3 * d * E * d_ff expert parameters and its activation
+  ratio is k / E: "万亿 MoE 只激活 4.9%" (m.xxqk.cn), parameter-count paragraph;
+* parameters active per token = router + k * (one expert) (sec. 10.6);
+* "match dense" shrinks each expert's hidden width so that the MoE holds as
+  many parameters as the dense layer (sec. 10.6; its worked example gives
+  1792 for d_hidden = 14336, E = 8).
+
+FLOPs count one multiply-add as 2.  The bytes are the algorithmic minimum of
+one layer call: bf16 weights of the experts the batch actually hits, the
+router matrix, the bf16 input and the fp32 output.
+"""
+from __future__ import annotations
+
+
+def ffn_params(d: int, d_hidden: int, matrices: int = 3) -> int:
+    """Dense feed-forward parameters: matrices * d * d_hidden (3 for SwiGLU)."""
+    return matrices * d * d_hidden
+
+
+def router_params(d: int, E: int) -> int:
+    return d * E
+
+
+def expert_params(d: int, d_ff: int) -> int:
+    """One SwiGLU expert: W1, W3 [d_ff, d] and W2 [d, d_ff]."""
+    return 3 * d * d_ff
+
+
+def moe_expert_params(d: int, E: int, d_ff: int) -> int:
+    """All experts of one layer: 3 * d * E * d_ff."""
+    return E * expert_params(d, d_ff)
+
+
+def active_params_per_token(d: int, E: int, d_ff: int, k: int) -> int:
+    return router_params(d, E) + k * expert_params(d, d_ff)
+
+
+def match_dense_hidden(d: int, d_hidden: int, E: int) -> int:
+    """Per-expert hidden width that makes E experts plus the router hold as
+    many parameters as the dense SwiGLU layer, rounded to the nearest integer
+    (the reading that reproduces the worked example's 1792)."""
+    return round((ffn_params(d, d_hidden) - router_params(d, E)) / (E * expert_params(d, 1)))
+
+
+def active_flops(T: int, d: int, E: int, d_ff: int, k: int, d_ff_shared: int = 0) -> int:
+    """2*3*d*d_ff*k*T expert FLOPs + 2*T*d*E router FLOPs (+ the shared expert)."""
+    return 2 * 3 * d * d_ff * k * T + 2 * T * d * E + 2 * 3 * d * d_ff_shared * T
+
+
+def algorithmic_bytes(T: int, d: int, E: int, d_ff: int, k: int, experts_hit: int,
+                      d_ff_shared: int = 0) -> int:
+    """Minimum HBM bytes of one layer call: hit experts' bf16 weights, bf16 Wg,
+    bf16 x read, fp32 out written (+ the shared expert's bf16 weights)."""
+    return (2 * experts_hit * expert_params(d, d_ff) + 2 * d * E + 2 * T * d + 4 * T * d
+            + 2 * expert_params(d, d_ff_shared))
+
+
+def gemm_bytes(kind: str, T: int, d: int, d_ff: int, k: int, experts_hit: int,
+               d_ff_shared: int = 0) -> int:
+    """Algorithmic bytes of one grouped-GEMM launch.
+
+    kind "up":   bf16 W1 and W3 of the hit experts + the permuted bf16 rows
+                 read (S = T*k rows of d) + bf16 H written (S rows of d_ff).
+    kind "down": bf16 W2 of the hit experts + bf16 H read + fp32 Y written
+                 (S rows of d).
+    A shared expert adds one more segment of T rows with its own weights.
+    """
+    S = T * k
+    if kind == "up":
+        return (2 * 2 * experts_hit * d * d_ff + 2 * S * d + 2 * S * d_ff
+                + (2 * 2 * d * d_ff_shared + 2 * T * d + 2 * T * d_ff_shared if d_ff_shared else 0))
+    if kind == "down":
+        return (2 * experts_hit * d * d_ff + 2 * S * d_ff + 4 * S * d
+                + (2 * d * d_ff_shared + 2 * T * d_ff_shared + 4 * T * d if d_ff_shared else 0))
+    raise ValueError(kind)
+
+
+def gemm_flops(kind: str, T: int, d: int, d_ff: int, k: int, d_ff_shared: int = 0) -> int:
+    S = T * k
+    if kind == "up":
+        return 2 * 2 * S * d * d_ff + 2 * 2 * T * d * d_ff_shared
+    if kind == "down":
+        return 2 * S * d * d_ff + 2 * T * d * d_ff_shared
+    raise ValueError(kind)

@@ -1,0 +1,50 @@
+"""The oracle's pins must catch plausible slips.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU,
+in a temporary directory), builds it, and runs the pin suite against the
+broken copy: the suite has to fail.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
+
+MUTANTS = {
+    "ties_to_higher_index": ("if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;",
+                             "if (!taken[e] && (best < 0 || l[e] >= l[best])) best = e;"),
+    "selects_smallest": ("if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;",
+                         "if (!taken[e] && (best < 0 || l[e] < l[best])) best = e;"),
+    "silu_on_w3_branch": ("h[f] = silu(a) * b;", "h[f] = a * silu(b);"),
+    "dropped_w3_term": ("h[f] = silu(a) * b;", "h[f] = silu(a);"),
+    "w2_transposed": ("acc += bf16_bits_to_double(r2[f]) * h[f];",
+                      "acc += bf16_bits_to_double(W2[(size_t)f * d + o]) * h[f];"),
+    "softmax_sign": ("        w[j] = exp(l[sel[j]] - m);\n        s += w[j];\n    }\n    for (int j = 0; j < k; ++j) w[j] /= s;\n}",
+                     "        w[j] = exp(m - l[sel[j]]);\n        s += w[j];\n    }\n    for (int j = 0; j < k; ++j) w[j] /= s;\n}"),
+    "bias_ignored": ("if (bias) acc += bias[e];", "if (bias) acc += 0.0 * bias[e];"),
+    "shared_expert_dropped": ("for (int i = 0; i < d; ++i) o[i] += y[i];",
+                              "for (int i = 0; i < d; ++i) o[i] += 0.0 * y[i];"),
+    "unnormalised_weights": ("for (int j = 0; j < k; ++j) w[j] /= s;\n}",
+                             "for (int j = 0; j < k; ++j) w[j] /= 1.0;\n}"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new, 1)
+    c = tmp_path / "mutant.c"
+    so = tmp_path / "libmutant.so"
+    c.write_text(mutated)
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fopenmp", "-shared", "-fPIC", "-o", str(so),
+                    str(c), "-lm"], check=True)
+    env = dict(os.environ, MOE_ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"planted mistake '{name}' passed every pin:\n{r.stdout[-2000:]}"

@@ -1,0 +1,283 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test names the passage it follows.  A plausible slip in the oracle (a
+dropped term, SiLU on the wrong branch, a transposed W2, a softmax over the
+wrong set or with the wrong sign, the opposite tie rule, a bias applied to
+only one of the two steps, a lost shared expert) fails at least one of them.
+The second formulations written here (torch/numpy fp64 matmuls, exhaustive
+subset search, softmax-all-then-renormalise, dense-all-experts-then-mask)
+share nothing with the oracle's C code.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from sparse_mixture_experts_histogram_b200 import synth
+from sparse_mixture_experts_histogram_b200.synth import Workload, bits
+
+
+def _inputs(T, d, E, dff, k, seed=42, dffs=0, skew=False):
+    wl = Workload("t", T, d, E, dff, k, d_ff_shared=dffs, skew=skew)
+    return wl, synth.make_inputs(wl, seed=seed)
+
+
+def _f64(t):
+    return t.to(torch.float64)
+
+
+def _swiglu_torch(x, W1, W3, W2):
+    """Library formulation: W2 (silu(W1 x) * W3 x) with torch fp64 matmuls."""
+    x, W1, W3, W2 = map(_f64, (x, W1, W3, W2))
+    return (F.silu(x @ W1.T) * (x @ W3.T)) @ W2.T
+
+
+def _rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300))
+
+
+def test_single_expert_top1_is_dense_swiglu():
+    # E = 1, k = 1 is the dense SwiGLU FFN ("万亿 MoE" sweep's dense row;
+    # FeedForward w2(silu(w1 x) * w3 x), jsqmd.com sec. 3.1).  d != d_ff so a
+    # transposed W2 cannot pass.
+    wl, inp = _inputs(T=7, d=24, E=1, dff=40, k=1)
+    out = oracle.forward(*(bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")), k=1)
+    ref = _swiglu_torch(inp["x"], inp["W1"][0], inp["W3"][0], inp["W2"][0]).numpy()
+    assert _rel(out, ref) < 1e-12
+    out2 = oracle.swiglu(bits(inp["x"]), bits(inp["W1"][0]), bits(inp["W3"][0]), bits(inp["W2"][0]))
+    assert _rel(out2, ref) < 1e-12
+
+
+def test_silu_branch_is_w1_not_w3():
+    # Swapping W1 and W3 must change the result (silu(a)*b != silu(b)*a).
+    wl, inp = _inputs(T=5, d=16, E=1, dff=24, k=1)
+    args = [bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")]
+    out = oracle.forward(*args, k=1)
+    swapped = oracle.forward(args[0], args[1], args[3], args[2], args[4], k=1)
+    assert _rel(out, swapped) > 1e-3
+
+
+def test_equal_logits_k_equals_E_gives_mean_of_experts():
+    # All router logits equal and k = E: every expert gets weight 1/E, the
+    # output is the plain mean of the experts.
+    wl, inp = _inputs(T=6, d=16, E=4, dff=24, k=4)
+    Wg0 = torch.zeros_like(inp["Wg"])
+    out = oracle.forward(bits(inp["x"]), bits(Wg0), bits(inp["W1"]), bits(inp["W3"]),
+                         bits(inp["W2"]), k=4)
+    ref = sum(_swiglu_torch(inp["x"], inp["W1"][e], inp["W3"][e], inp["W2"][e])
+              for e in range(4)) / 4
+    assert _rel(out, ref.numpy()) < 1e-12
+
+
+def test_equal_logits_ties_go_to_lower_index():
+    # Tie rule: equal logits select the lower expert index.
+    wl, inp = _inputs(T=9, d=16, E=6, dff=8, k=3)
+    r = oracle.route(bits(inp["x"]), bits(torch.zeros_like(inp["Wg"])), k=3)
+    assert (r["idx"] == np.array([0, 1, 2], np.int32)).all()
+    assert np.allclose(r["w"], 1.0 / 3.0, rtol=0, atol=1e-15)
+    assert (r["gap"] == 0).all()
+
+
+def test_duplicate_router_rows_tie_to_lower_index():
+    # Two experts with identical router rows have bit-identical logits; the
+    # lower index must come first whenever the pair is selected or split.
+    wl, inp = _inputs(T=64, d=32, E=6, dff=8, k=2)
+    Wg = inp["Wg"].clone()
+    Wg[4] = Wg[1]
+    r = oracle.route(bits(inp["x"]), bits(Wg), k=2)
+    for t in range(64):
+        s = list(r["idx"][t])
+        assert not (4 in s and 1 not in s), "expert 4 chosen over its twin 1"
+        if 1 in s and 4 in s:
+            assert s.index(1) < s.index(4)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(6, 8, 5, 2), (5, 8, 5, 3), (4, 6, 4, 4), (6, 8, 5, 1)])
+def test_top_k_set_is_best_subset(T, d, E, k):
+    # Brute force: the selected set maximises the sum of logits over all
+    # C(E,k) subsets; among equal sums the lexicographically smallest index
+    # set wins (the lower-index tie rule).  Logits from a torch fp64 matmul.
+    wl, inp = _inputs(T=T, d=d, E=E, dff=8, k=k)
+    Wg = inp["Wg"].clone()
+    Wg[E - 1] = Wg[0]  # force exact ties in some tokens
+    r = oracle.route(bits(inp["x"]), bits(Wg), k=k)
+    L = (_f64(inp["x"]) @ _f64(Wg).T).numpy()
+    for t in range(T):
+        best = None
+        for sub in itertools.combinations(range(E), k):  # lexicographic order
+            s = sum(L[t, e] for e in sub)
+            if best is None or s > best[0] + 1e-12:
+                best = (s, sub)
+        assert sorted(r["idx"][t]) == list(best[1])
+        # slot order: logits non-increasing
+        lv = L[t, r["idx"][t]]
+        assert (np.diff(lv) <= 1e-12).all()
+
+
+def test_weights_sum_to_one_and_follow_logits():
+    # Softmax over the k selected logits: weights sum to 1 ("MoE: ..." sec.
+    # 10.3), and a larger logit gets a larger weight.
+    wl, inp = _inputs(T=200, d=64, E=16, dff=8, k=4)
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=4)
+    assert np.allclose(r["w"].sum(1), 1.0, rtol=0, atol=1e-14)
+    assert (np.diff(r["w"], axis=1) <= 1e-15).all()
+    assert (r["w"] > 0).all()
+
+
+def test_top2_weight_closed_form():
+    # k = 2: w0 = 1 / (1 + exp(l1 - l0)), the logistic of the logit gap.
+    wl, inp = _inputs(T=50, d=32, E=8, dff=8, k=2)
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=2)
+    L = (_f64(inp["x"]) @ _f64(inp["Wg"]).T).numpy()
+    l0 = L[np.arange(50), r["idx"][:, 0]]
+    l1 = L[np.arange(50), r["idx"][:, 1]]
+    assert np.allclose(r["w"][:, 0], 1.0 / (1.0 + np.exp(l1 - l0)), rtol=1e-13, atol=0)
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_softmax_all_then_renormalise_matches(with_bias):
+    # Second formulation ("Mixtral and MoE architecture" MixtralMoE listing):
+    # softmax over all E logits, top-k of the probabilities, renormalise.  It
+    # must equal the softmax over the k selected logits, bias included in
+    # both the selection and the weights.
+    wl, inp = _inputs(T=100, d=48, E=12, dff=8, k=3)
+    bias = np.linspace(-0.7, 0.9, 12) if with_bias else None
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=3, bias=bias)
+    L = (_f64(inp["x"]) @ _f64(inp["Wg"]).T).numpy()
+    if with_bias:
+        L = L + bias[None, :]
+    P = np.exp(L - L.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    for t in range(100):
+        order = sorted(range(12), key=lambda e: (-P[t, e], e))[:3]
+        assert list(r["idx"][t]) == order
+        ww = P[t, order] / P[t, order].sum()
+        assert np.allclose(r["w"][t], ww, rtol=1e-12, atol=0)
+
+
+def test_per_token_logit_shift_changes_nothing():
+    # Mean-centring the logits before top-k ("Mistral 8x7B SMoE" sec. 3.2,
+    # logits calibration) -- in general any per-token shift -- changes
+    # neither the selection nor the weights.  The shift is built by an extra
+    # input column c_t whose router weight is 1 for every expert.
+    wl, inp = _inputs(T=40, d=32, E=8, dff=8, k=2)
+    c = torch.randn(40, 1, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16) * 4
+    x2 = torch.cat([inp["x"], c], 1)
+    Wg2 = torch.cat([inp["Wg"], torch.ones(8, 1, dtype=torch.bfloat16)], 1)
+    r1 = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=2)
+    r2 = oracle.route(bits(x2), bits(Wg2), k=2)
+    ok = r1["gap"] > 1e-9
+    assert (r1["idx"][ok] == r2["idx"][ok]).all()
+    assert np.allclose(r1["w"][ok], r2["w"][ok], rtol=1e-10, atol=0)
+
+
+def test_token_permutation_equivariance():
+    # Tokens are independent: permuting them permutes the outputs, exactly.
+    wl, inp = _inputs(T=12, d=16, E=5, dff=16, k=2)
+    perm = torch.randperm(12, generator=torch.Generator().manual_seed(1))
+    names = ("Wg", "W1", "W3", "W2")
+    out = oracle.forward(bits(inp["x"]), *(bits(inp[n]) for n in names), k=2)
+    outp = oracle.forward(bits(inp["x"][perm]), *(bits(inp[n]) for n in names), k=2)
+    assert np.array_equal(outp, out[perm.numpy()])
+    sub = oracle.forward(bits(inp["x"]), *(bits(inp[n]) for n in names), k=2,
+                         tokens=perm.numpy()[:5])
+    assert np.array_equal(sub, out[perm.numpy()[:5]])
+
+
+@pytest.mark.parametrize("T,d,E,dff,k", [(6, 8, 5, 12, 2), (5, 16, 4, 8, 3), (4, 8, 3, 8, 3)])
+def test_dense_all_experts_then_mask(T, d, E, dff, k):
+    # Second formulation of the whole layer: run every expert on every token
+    # (numpy fp64), then keep each token's k experts with their weights via a
+    # [T, E] mask ("Mixtral and MoE architecture" MixtralMoE listing: mask per
+    # expert; "MoE: ..." sec. 10.4: weighted index_add).
+    wl, inp = _inputs(T=T, d=d, E=E, dff=dff, k=k, seed=7)
+    x, Wg, W1, W3, W2 = (_f64(inp[n]).numpy() for n in ("x", "Wg", "W1", "W3", "W2"))
+    out = oracle.forward(*(bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")), k=k)
+    L = x @ Wg.T
+    M = np.zeros((T, E))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -L[t]))[:k]
+        z = np.exp(L[t, order] - L[t, order].max())
+        M[t, order] = z / z.sum()
+    Y = np.zeros((T, d))
+    for e in range(E):
+        a, b = x @ W1[e].T, x @ W3[e].T
+        Y += M[:, e:e + 1] * (((a / (1 + np.exp(-a))) * b) @ W2[e].T)
+    assert _rel(out, Y) < 1e-12
+
+
+def test_linear_in_w2_and_w3_zero_w3():
+    # out is linear in W2 and in W3: doubling either (exact in bf16) doubles
+    # the output exactly; W3 = 0 gives 0.
+    wl, inp = _inputs(T=6, d=16, E=4, dff=16, k=2)
+    args = {n: inp[n] for n in ("x", "Wg", "W1", "W3", "W2")}
+    base = oracle.forward(*(bits(args[n]) for n in ("x", "Wg", "W1", "W3", "W2")), k=2)
+    for n in ("W2", "W3"):
+        a2 = dict(args)
+        a2[n] = args[n] * 2
+        o = oracle.forward(*(bits(a2[m]) for m in ("x", "Wg", "W1", "W3", "W2")), k=2)
+        assert np.array_equal(o, 2 * base)
+    a0 = dict(args)
+    a0["W3"] = torch.zeros_like(args["W3"])
+    o = oracle.forward(*(bits(a0[m]) for m in ("x", "Wg", "W1", "W3", "W2")), k=2)
+    assert not np.any(o)
+
+
+def test_shared_expert_is_added_unweighted():
+    # The shared expert runs on every token and is added with weight 1
+    # ("MoE: ..." sec. 10.5).
+    wl, inp = _inputs(T=8, d=16, E=6, dff=8, k=2, dffs=24)
+    names = ("x", "Wg", "W1", "W3", "W2")
+    a = oracle.forward(*(bits(inp[n]) for n in names), k=2,
+                       shared=(bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"])))
+    b = oracle.forward(*(bits(inp[n]) for n in names), k=2)
+    ref = _swiglu_torch(inp["x"], inp["Ws1"], inp["Ws3"], inp["Ws2"]).numpy()
+    assert np.max(np.abs((a - b) - ref)) < 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_forced_set_equal_to_own_set_is_identity_and_other_set_renormalises():
+    wl, inp = _inputs(T=10, d=16, E=6, dff=8, k=2)
+    names = ("x", "Wg", "W1", "W3", "W2")
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=2)
+    a = oracle.forward(*(bits(inp[n]) for n in names), k=2)
+    b = oracle.forward(*(bits(inp[n]) for n in names), k=2, forced=r["idx"])
+    assert np.array_equal(a, b)
+    # a forced set is weighted by the softmax over its own logits
+    forced = np.tile(np.array([[5, 0]], np.int32), (10, 1))
+    c = oracle.forward(*(bits(inp[n]) for n in names), k=2, forced=forced)
+    L = (_f64(inp["x"]) @ _f64(inp["Wg"]).T).numpy()
+    y = [_swiglu_torch(inp["x"], inp["W1"][e], inp["W3"][e], inp["W2"][e]).numpy() for e in (5, 0)]
+    z = np.exp(L[:, [5, 0]] - L[:, [5, 0]].max(1, keepdims=True))
+    z /= z.sum(1, keepdims=True)
+    ref = z[:, :1] * y[0] + z[:, 1:] * y[1]
+    assert _rel(c, ref) < 1e-12
+
+
+def test_counts_histogram_and_gap():
+    wl, inp = _inputs(T=300, d=32, E=10, dff=8, k=3)
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=3)
+    assert r["counts"].sum() == 300 * 3
+    assert np.array_equal(r["counts"], np.bincount(r["idx"].ravel(), minlength=10))
+    assert all(len(set(row)) == 3 for row in r["idx"])
+    assert (r["gap"] >= 0).all()
+    rk = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=10)
+    assert np.isinf(rk["gap"]).all()
+
+
+def test_expert_call_statistics_plausible():
+    # "万亿 MoE 只激活 4.9%": 512 tokens, 128 experts, top-8 -> 4096 expert
+    # calls, 128/128 experts hit, 17..46 tokens per expert.  The call count is
+    # exact; the spread is only a plausibility check (the page's weights were
+    # not published, so the per-expert counts are parity unpinned).
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_numbers.json")))
+    p = g["expert_calls"]
+    wl, inp = _inputs(T=p["T"], d=512, E=p["E"], dff=8, k=p["k"])
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=p["k"])
+    assert int(r["counts"].sum()) == p["calls"]
+    assert int((r["counts"] > 0).sum()) >= p["experts_hit"] - 4
+    assert r["counts"].min() >= 5 and r["counts"].max() <= 80
