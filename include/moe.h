@@ -1,0 +1,181 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts
+ * feed-forward layer (forward pass).
+ *
+ * The layer (Mixtral-style SMoE with SwiGLU experts):
+ *   logits = x Wg^T                       router, a bias-free linear layer
+ *   idx    = top-k experts per token      largest logits, equal logits go to
+ *                                         the lower expert index
+ *   w      = softmax over the k selected logits (weights sum to 1)
+ *   y_e    = W2_e (silu(W1_e x) * (W3_e x))   one SwiGLU expert
+ *   out    = sum_j w_j * y_{idx_j}        gate-weighted sum in token order
+ *            (+ an always-on shared expert, weight 1, in moe_forward_ex)
+ * Sources: "Mistral 8x7B SMoE architecture" (jsqmd.com) sec. 3.1
+ * FeedForward and sec. 3.2 Gating Network; "MoE" chapter 10 of
+ * LLMs-from-scratch (theaiera.top) sec. 10.3 router/top-k, sec. 10.4
+ * sparse dispatch and weighted index_add, sec. 10.5 shared expert;
+ * "Mixtral and MoE architecture" (astro-blog) MixtralMoE and FeedForward
+ * listings.  Dispatch is dropless: every (token, slot) pair is computed.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Shapes: T tokens, d model width, E experts, d_ff expert hidden width,
+ *   k experts per token, S = T*k routed rows.  All matrices are row-major
+ *   with nn.Linear's [out, in] layout:
+ *     x [T,d] bf16, Wg [E,d] bf16, W1 and W3 [E,d_ff,d] bf16,
+ *     W2 [E,d,d_ff] bf16, out [T,d] fp32; shared expert Ws1 and Ws3
+ *     [d_ffs,d] bf16, Ws2 [d,d_ffs] bf16.
+ *   bf16 values are passed as raw 16-bit patterns (moe_bf16).
+ * Supported sizes: 1 <= T <= 2^24; 1 <= k <= min(E, 8); 1 <= E <= 256;
+ *   d and d_ff (and d_ffs) multiples of 128 with d <= 16384 and
+ *   d_ff <= 65536; S*max(d, d_ff) < 2^31.  Other sizes return
+ *   MOE_ERR_UNSUPPORTED; nothing falls back to another code path.
+ * Pointers: every array argument is a DEVICE pointer on the current CUDA
+ *   device, 16-byte aligned (MOE_ERR_INVALID_ARG otherwise); optional
+ *   arguments may be NULL where stated.
+ * Ownership: the caller allocates and frees every buffer, including the
+ *   workspace `ws` (at least moe_workspace_size() bytes, 256-byte aligned).
+ *   The library allocates no memory in any call and keeps no pointer after
+ *   it returns.
+ * Asynchrony: work is enqueued on `stream` and the call returns without
+ *   waiting for it; no call synchronises the host except
+ *   moe_get_device_error.  Buffers must stay valid until the stream has
+ *   finished the work.  Calls sharing a workspace must be ordered on one
+ *   stream.
+ * Errors: arguments are checked on the host before anything is launched;
+ *   the first failed check is returned and nothing is enqueued.  A failed
+ *   launch returns MOE_ERR_CUDA.  Problems only the GPU can see (an
+ *   inconsistent offsets array, a bounded wait that ran out) set an error
+ *   word inside the workspace, readable with moe_get_device_error; each
+ *   entry point that takes a workspace clears that word when it starts.
+ *   No C++ exception crosses this interface.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+typedef uint16_t moe_bf16;                /* raw bfloat16 bits */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null or misaligned pointer, negative size, k > E, ... */
+    MOE_ERR_UNSUPPORTED = 2, /* valid but outside the supported sizes above */
+    MOE_ERR_WORKSPACE = 3,   /* ws_bytes smaller than moe_workspace_size() */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime/driver call or a launch failed */
+    MOE_ERR_DEVICE = 5,      /* the device error word is set (moe_get_device_error) */
+    MOE_ERR_TIMEOUT = 6      /* a device-side bounded wait ran out */
+} moe_status;
+
+/* Device error word bits (moe_get_device_error's *code). */
+#define MOE_DEVERR_TIMEOUT_TMA 0x1u  /* a pipeline wait for a tensor-memory copy ran out */
+#define MOE_DEVERR_TIMEOUT_MMA 0x2u  /* a wait for tensor-core work ran out */
+#define MOE_DEVERR_TIMEOUT_EPI 0x4u  /* a wait for the epilogue ran out */
+#define MOE_DEVERR_OFFSETS 0x8u      /* offsets[] not non-decreasing within [0, S] */
+#define MOE_DEVERR_INDEX 0x10u       /* an expert index or row index out of range */
+
+/* Bytes of workspace every entry point below needs for these shapes
+ * (the largest need over all of them).  0 if the shapes are unsupported. */
+MOE_API size_t moe_workspace_size(int T, int d, int E, int d_ff, int k);
+
+/* Same, with a shared expert of hidden width d_ff_shared (0 = none). */
+MOE_API size_t moe_workspace_size_ex(int T, int d, int E, int d_ff, int k, int d_ff_shared);
+
+/* Router: logits = x Wg^T (+ router_bias), per-token top-k (ties to the
+ * lower expert index), softmax over the k selected logits, and the
+ * per-expert histogram.
+ *   router_bias [E] fp32 or NULL: added to every token's logits before both
+ *     the selection and the softmax (no bias on the pages' routers; used to
+ *     build skewed loads)
+ *   idx [T,k] int32 out: experts of each token, by logit descending
+ *   w [T,k] fp32 out: their softmax weights (sum to 1 per token)
+ *   counts [E] int32 out: number of (token, slot) pairs routed to each expert
+ * Passages: jsqmd.com sec. 3.2 (gate -> topk -> softmax over the selected
+ * values); theaiera.top sec. 10.3 (weights sum to 1); torch.unique / per
+ * expert token lists of sec. 10.4 become the histogram. */
+MOE_API moe_status moe_route(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
+                     const float *router_bias, int32_t *idx, float *w, int32_t *counts,
+                     void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Dispatch: group the S = T*k (token, slot) pairs by expert.
+ *   idx [T,k] int32 in: experts per token (values in [0,E), distinct per token)
+ *   offsets [E+1] int32 out: exclusive prefix sum of the per-expert counts;
+ *     expert e owns rows offsets[e] .. offsets[e+1]-1 of x_perm
+ *   row_of_slot [T,k] int32 out: the x_perm row that holds (token t, slot j)
+ *   x_perm [S,d] bf16 out: x_perm[row_of_slot[t,j]] = x[t]
+ * Within an expert's rows the order is by token index (stable), so the
+ * result is deterministic.  An index outside [0,E) sets MOE_DEVERR_INDEX
+ * and that pair is skipped.  Passage: theaiera.top sec. 10.4 (mask,
+ * nonzero and index_select per expert). */
+MOE_API moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int32_t *idx,
+                       int32_t *offsets, int32_t *row_of_slot, moe_bf16 *x_perm, void *ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* Experts: for every expert e and row r in [offsets[e], offsets[e+1]):
+ *   y_perm[r] = W2_e (silu(W1_e x_perm[r]) * (W3_e x_perm[r]))
+ *   S: rows of x_perm and y_perm; offsets [E+1] int32 (device) as returned
+ *   by moe_permute; y_perm [S,d] fp32 out.  H = silu(.)*(.) is rounded to
+ *   bf16 between the two products.
+ * An offsets array that is not non-decreasing within [0,S] sets
+ * MOE_DEVERR_OFFSETS and no row is computed.  Passages: jsqmd.com sec. 3.1
+ * FeedForward; theaiera.top sec. 10.4 (fc1/fc2/fc3 of the selected rows). */
+MOE_API moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
+                          const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
+                          const moe_bf16 *W2, float *y_perm, void *ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* Combine: out[t] = sum_{j<k} w[t,j] * y_perm[row_of_slot[t,j]]
+ * (+ shared_y[t]), summed in slot order j = 0..k-1.
+ *   y_perm [T*k, d] fp32, row_of_slot [T,k] int32, w [T,k] fp32,
+ *   shared_y [T,d] fp32 or NULL, out [T,d] fp32 out (overwritten).
+ * Passages: theaiera.top sec. 10.4 (weighted index_add back to token order)
+ * and sec. 10.5 (shared expert added). */
+MOE_API moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *row_of_slot,
+                       const float *w, const float *shared_y, float *out, moe_stream_t stream);
+
+/* The whole layer: route, dispatch, experts and combine in one call.
+ * out [T,d] fp32 out.  Equivalent to moe_route + moe_permute +
+ * moe_expert_ffn + moe_combine, without leaving the GPU and without any
+ * host synchronisation (the call can be captured in a CUDA graph). */
+MOE_API moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                       const moe_bf16 *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
+                       const moe_bf16 *W2, float *out, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* moe_forward with an optional router bias (see moe_route) and an optional
+ * shared expert of hidden width d_ff_shared (0 = none; Ws1/Ws3/Ws2 may then
+ * be NULL), whose output is added to every token with weight 1
+ * (theaiera.top sec. 10.5).  The workspace must hold
+ * moe_workspace_size_ex(..., d_ff_shared) bytes. */
+MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                          const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
+                          const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
+                          const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
+                          float *out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Waits for `stream`, then reads the device error word of workspace `ws`
+ * into *code (may be NULL).  Returns MOE_OK if it is zero, MOE_ERR_TIMEOUT
+ * if a timeout bit is set, MOE_ERR_DEVICE for any other bit, MOE_ERR_CUDA if
+ * the wait or the read failed. */
+MOE_API moe_status moe_get_device_error(const void *ws, uint32_t *code, moe_stream_t stream);
+
+/* Static description of a status code; never NULL. */
+MOE_API const char *moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,22 @@
+"""B200 (sm_100a) sparse Mixture-of-Experts feed-forward layer, forward pass.
+
+The compute lives in the CUDA library ``libmoe_b200.so`` behind the C ABI of
+``include/moe.h``; ``binding`` exposes the same entry points to Python.
+``synth`` draws the seeded synthetic inputs and ``accounting`` holds the
+FLOP/byte/parameter closed forms used for throughput and roofline numbers.
+"""
+from .binding import (  # noqa: F401
+    ABI_FUNCTIONS,
+    MoEError,
+    load_library,
+    moe_combine,
+    moe_expert_ffn,
+    moe_forward,
+    moe_forward_ex,
+    moe_get_device_error,
+    moe_permute,
+    moe_route,
+    moe_status_string,
+    moe_workspace_size,
+    moe_workspace_size_ex,
+)

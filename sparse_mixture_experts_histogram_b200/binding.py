@@ -1,0 +1,163 @@
+"""Python binding of the C ABI in ``include/moe.h`` (ctypes).
+
+Argument marshalling only: every function has the same name and argument
+order as its C counterpart, takes torch tensors (or raw device addresses as
+ints) and turns a non-zero status into ``MoEError``.  All work runs in the
+CUDA library ``libmoe_b200.so``; there is no other implementation to fall
+back to, so a missing library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+    4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE", 6: "MOE_ERR_TIMEOUT",
+}
+DEVERR_BITS = {0x1: "TIMEOUT_TMA", 0x2: "TIMEOUT_MMA", 0x4: "TIMEOUT_EPI", 0x8: "OFFSETS",
+               0x10: "INDEX"}
+
+#: Every symbol the C header declares (checked against ``include/moe.h`` by the tests).
+ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "moe_permute",
+                 "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_ex",
+                 "moe_get_device_error", "moe_status_string")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+_I, _P, _SZ = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load ``libmoe_b200.so`` (built in-tree by ``build.py``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(
+                f"{p} is missing: build it with `python -m sparse_mixture_experts_histogram_b200"
+                ".build` (the layer has no implementation other than this CUDA library)")
+        lib = ctypes.CDLL(p)
+        sig = {
+            "moe_workspace_size": (_SZ, [_I] * 5),
+            "moe_workspace_size_ex": (_SZ, [_I] * 6),
+            "moe_route": (_I, [_I] * 4 + [_P] * 6 + [_P, _SZ, _P]),
+            "moe_permute": (_I, [_I] * 4 + [_P] * 6 + [_SZ, _P]),
+            "moe_expert_ffn": (_I, [_I] * 4 + [_P] * 7 + [_SZ, _P]),
+            "moe_combine": (_I, [_I] * 3 + [_P] * 5 + [_P]),
+            "moe_forward": (_I, [_I] * 5 + [_P] * 7 + [_SZ, _P]),
+            "moe_forward_ex": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P]),
+            "moe_get_device_error": (_I, [_P, _P, _P]),
+            "moe_status_string": (ctypes.c_char_p, [_I]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().moe_status_string(status).decode()
+    except RuntimeError:
+        return STATUS_NAMES.get(status, f"status {status}")
+
+
+moe_status_string = status_string
+
+
+def moe_workspace_size(T, d, E, d_ff, k) -> int:
+    return int(load_library().moe_workspace_size(T, d, E, d_ff, k))
+
+
+def moe_workspace_size_ex(T, d, E, d_ff, k, d_ff_shared) -> int:
+    return int(load_library().moe_workspace_size_ex(T, d, E, d_ff, k, d_ff_shared))
+
+
+def _ws_bytes(ws) -> int:
+    if isinstance(ws, int):
+        raise TypeError("pass the workspace as a tensor so its size is known")
+    return ws.numel() * ws.element_size()
+
+
+def moe_route(T, d, E, k, x, Wg, router_bias, idx, w, counts, ws, stream=None):
+    _check(load_library().moe_route(T, d, E, k, _ptr(x), _ptr(Wg), _ptr(router_bias), _ptr(idx),
+                                    _ptr(w), _ptr(counts), _ptr(ws), _ws_bytes(ws),
+                                    _stream(stream)), "moe_route")
+
+
+def moe_permute(T, d, E, k, x, idx, offsets, row_of_slot, x_perm, ws, stream=None):
+    _check(load_library().moe_permute(T, d, E, k, _ptr(x), _ptr(idx), _ptr(offsets),
+                                      _ptr(row_of_slot), _ptr(x_perm), _ptr(ws), _ws_bytes(ws),
+                                      _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(S, d, E, d_ff, x_perm, offsets, W1, W3, W2, y_perm, ws, stream=None):
+    _check(load_library().moe_expert_ffn(S, d, E, d_ff, _ptr(x_perm), _ptr(offsets), _ptr(W1),
+                                         _ptr(W3), _ptr(W2), _ptr(y_perm), _ptr(ws),
+                                         _ws_bytes(ws), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(T, d, k, y_perm, row_of_slot, w, shared_y, out, stream=None):
+    _check(load_library().moe_combine(T, d, k, _ptr(y_perm), _ptr(row_of_slot), _ptr(w),
+                                      _ptr(shared_y), _ptr(out), _stream(stream)), "moe_combine")
+
+
+def moe_forward(T, d, E, d_ff, k, x, Wg, W1, W3, W2, out, ws, stream=None):
+    _check(load_library().moe_forward(T, d, E, d_ff, k, _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3),
+                                      _ptr(W2), _ptr(out), _ptr(ws), _ws_bytes(ws),
+                                      _stream(stream)), "moe_forward")
+
+
+def moe_forward_ex(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3, Ws2,
+                   out, ws, stream=None):
+    _check(load_library().moe_forward_ex(T, d, E, d_ff, k, _ptr(x), _ptr(Wg), _ptr(router_bias),
+                                         _ptr(W1), _ptr(W3), _ptr(W2), d_ff_shared, _ptr(Ws1),
+                                         _ptr(Ws3), _ptr(Ws2), _ptr(out), _ptr(ws),
+                                         _ws_bytes(ws), _stream(stream)), "moe_forward_ex")
+
+
+def moe_get_device_error(ws, stream=None) -> tuple[int, int]:
+    """(status, error word) of the last call that used workspace ``ws``."""
+    code = ctypes.c_uint32(0)
+    st = load_library().moe_get_device_error(_ptr(ws), ctypes.byref(code), _stream(stream))
+    return int(st), int(code.value)

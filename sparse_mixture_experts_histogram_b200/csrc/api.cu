@@ -1,0 +1,415 @@
+// api.cu -- the C ABI declared in include/moe.h: argument checks, workspace
+// layout, tensor-map encoding and the launch sequence of each entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, ranks counter @8
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+    size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, xperm, H, Y, Hs, Ys, total;
+};
+
+// Workspace of moe_forward_ex (a superset of every other entry point's need).
+Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
+{
+    Layout L{};
+    size_t o = kHeaderBytes;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o += align_up(bytes);
+        return r;
+    };
+    const size_t ntiles = (static_cast<size_t>(T) + 127) / 128;
+    const size_t S = static_cast<size_t>(T) * k;
+    L.tilecnt = take(ntiles * E * 4);
+    L.tilebase = take(ntiles * E * 4);
+    L.rank = take(S * 4);
+    L.offsets = take((static_cast<size_t>(E) + 1) * 4);
+    L.counts = take(static_cast<size_t>(E) * 4);
+    L.idx = take(S * 4);
+    L.w = take(S * 4);
+    L.row = take(S * 4);
+    L.xperm = take(S * d * 2);
+    L.H = take(S * d_ff * 2);
+    L.Y = take(S * d * 4);
+    if (d_ffs > 0) {
+        L.Hs = take(static_cast<size_t>(T) * d_ffs * 2);
+        L.Ys = take(static_cast<size_t>(T) * d * 4);
+    } else {
+        L.Hs = L.Ys = 0;
+    }
+    L.total = o;
+    return L;
+}
+
+moe_status check_shapes(int T, int d, int E, int d_ff, int k, int d_ffs)
+{
+    if (T < 1 || d < 1 || E < 1 || d_ff < 1 || k < 1 || d_ffs < 0) return MOE_ERR_INVALID_ARG;
+    if (k > E) return MOE_ERR_INVALID_ARG;
+    if (k > 8 || E > 256 || T > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+    if (d % 128 || d_ff % 128 || d_ffs % 128) return MOE_ERR_UNSUPPORTED;
+    if (d > 16384 || d_ff > 65536 || d_ffs > 65536) return MOE_ERR_UNSUPPORTED;
+    const long long S = static_cast<long long>(T) * k;
+    const long long w = std::max({d, d_ff, d_ffs});
+    if (S * w >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ---------------------------------------------------------------- driver bits
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encode()
+{
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+}  // namespace
+
+cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows)
+{
+    std::call_once(g_encode_once, load_encode);
+    if (g_encode == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int device_sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    int n = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        n = 148;
+    g_sm_count[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size_ex(int T, int d, int E, int d_ff, int k, int d_ff_shared)
+{
+    if (check_shapes(T, d, E, d_ff, k, d_ff_shared) != MOE_OK) return 0;
+    return forward_layout(T, d, E, d_ff, k, d_ff_shared).total;
+}
+
+size_t moe_workspace_size(int T, int d, int E, int d_ff, int k)
+{
+    return moe_workspace_size_ex(T, d, E, d_ff, k, 0);
+}
+
+const char *moe_status_string(moe_status s)
+{
+    switch (s) {
+    case MOE_OK: return "MOE_OK: success";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument (null or misaligned pointer, bad size, k > E)";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: sizes outside the supported range";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace smaller than moe_workspace_size()";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE: the device error word is set";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a device-side bounded wait ran out";
+    }
+    return "unknown moe_status";
+}
+
+static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
+                             const float *bias, int32_t *idx, float *w, int32_t *counts,
+                             int32_t *offsets, uint8_t *ws, const Layout &L, cudaStream_t s)
+{
+    RouteLaunch a;
+    a.T = T;
+    a.d = d;
+    a.E = E;
+    a.k = k;
+    a.x = x;
+    a.Wg = Wg;
+    a.bias = bias;
+    a.idx = idx;
+    a.w = w;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.tilecnt = reinterpret_cast<int32_t *>(ws + L.tilecnt);
+    a.tilebase = reinterpret_cast<int32_t *>(ws + L.tilebase);
+    a.rank = reinterpret_cast<int32_t *>(ws + L.rank);
+    a.done = reinterpret_cast<uint32_t *>(ws + 4);
+    a.err = reinterpret_cast<uint32_t *>(ws);
+    return from_cuda(launch_route(a, s));
+}
+
+moe_status moe_route(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
+                     const float *router_bias, int32_t *idx, float *w, int32_t *counts, void *ws,
+                     size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = check_shapes(T, d, E, 128, k, 0);
+    if (st != MOE_OK) return st;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(idx) || !ok_ptr(w) || !ok_ptr(counts) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (router_bias != nullptr && !aligned16(router_bias)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_workspace_size(T, d, E, 128, k)) return MOE_ERR_WORKSPACE;
+    const Layout L = forward_layout(T, d, E, 128, k, 0);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    if (st != MOE_OK) return st;
+    return route_impl(T, d, E, k, x, Wg, router_bias, idx, w, counts,
+                      reinterpret_cast<int32_t *>(wsb + L.offsets), wsb, L, s);
+}
+
+moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int32_t *idx,
+                       int32_t *offsets, int32_t *row_of_slot, moe_bf16 *x_perm, void *ws,
+                       size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = check_shapes(T, d, E, 128, k, 0);
+    if (st != MOE_OK) return st;
+    if (!ok_ptr(x) || !ok_ptr(idx) || !ok_ptr(offsets) || !ok_ptr(row_of_slot) ||
+        !ok_ptr(x_perm) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_workspace_size(T, d, E, 128, k)) return MOE_ERR_WORKSPACE;
+    const Layout L = forward_layout(T, d, E, 128, k, 0);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    if (st != MOE_OK) return st;
+    RanksLaunch r;
+    r.T = T;
+    r.E = E;
+    r.k = k;
+    r.idx = idx;
+    r.offsets = offsets;
+    r.tilecnt = reinterpret_cast<int32_t *>(wsb + L.tilecnt);
+    r.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
+    r.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
+    r.done = reinterpret_cast<uint32_t *>(wsb + 8);
+    r.err = reinterpret_cast<uint32_t *>(wsb);
+    st = from_cuda(launch_ranks(r, s));
+    if (st != MOE_OK) return st;
+    ScatterLaunch c;
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.k = k;
+    c.x = x;
+    c.idx = idx;
+    c.rank = r.rank;
+    c.tilebase = r.tilebase;
+    c.x_perm = x_perm;
+    c.row_of_slot = row_of_slot;
+    c.err = r.err;
+    return from_cuda(launch_scatter(c, s));
+}
+
+static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const moe_bf16 *x_perm,
+                           const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
+                           const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *err,
+                           cudaStream_t s)
+{
+    GemmLaunch g;
+    g.up = 1;
+    g.E = E;
+    g.M_rows = d_ff;
+    g.K = d;
+    g.S = S;
+    g.max_rows = max_rows;
+    g.offsets = offsets;
+    g.A0 = W1;
+    g.A1 = W3;
+    g.B = x_perm;
+    g.out = H;
+    g.err = err;
+    moe_status st = from_cuda(launch_gemm(g, s));
+    if (st != MOE_OK) return st;
+    g.up = 0;
+    g.M_rows = d;
+    g.K = d_ff;
+    g.A0 = W2;
+    g.A1 = nullptr;
+    g.B = H;
+    g.out = y;
+    return from_cuda(launch_gemm(g, s));
+}
+
+moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
+                          const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
+                          const moe_bf16 *W2, float *y_perm, void *ws, size_t ws_bytes,
+                          moe_stream_t stream)
+{
+    moe_status st = check_shapes(S, d, E, d_ff, 1, 0);
+    if (st != MOE_OK) return st;
+    if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(y_perm) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = kHeaderBytes + align_up(static_cast<size_t>(S) * d_ff * 2);
+    if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    if (st != MOE_OK) return st;
+    return ffn_impl(S, d, E, d_ff, S, x_perm, offsets, W1, W3, W2,
+                    reinterpret_cast<moe_bf16 *>(wsb + kHeaderBytes), y_perm,
+                    reinterpret_cast<uint32_t *>(wsb), s);
+}
+
+moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *row_of_slot,
+                       const float *w, const float *shared_y, float *out, moe_stream_t stream)
+{
+    if (T < 1 || d < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+    if (k > 8 || T > (1 << 24) || d % 128 || d > 16384) return MOE_ERR_UNSUPPORTED;
+    if (!ok_ptr(y_perm) || !ok_ptr(row_of_slot) || !ok_ptr(w) || !ok_ptr(out))
+        return MOE_ERR_INVALID_ARG;
+    if (shared_y != nullptr && !aligned16(shared_y)) return MOE_ERR_INVALID_ARG;
+    CombineLaunch c;
+    c.T = T;
+    c.d = d;
+    c.k = k;
+    c.y = y_perm;
+    c.row_of_slot = row_of_slot;
+    c.w = w;
+    c.shared_y = shared_y;
+    c.out = out;
+    return from_cuda(launch_combine(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                          const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
+                          const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
+                          const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
+                          float *out, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = check_shapes(T, d, E, d_ff, k, d_ff_shared);
+    if (st != MOE_OK) return st;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) || !ok_ptr(out) ||
+        !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (router_bias != nullptr && !aligned16(router_bias)) return MOE_ERR_INVALID_ARG;
+    if (d_ff_shared > 0 && (!ok_ptr(Ws1) || !ok_ptr(Ws3) || !ok_ptr(Ws2)))
+        return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_INVALID_ARG;
+    const Layout L = forward_layout(T, d, E, d_ff, k, d_ff_shared);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    uint32_t *err = reinterpret_cast<uint32_t *>(wsb);
+    const int S = T * k;
+    int32_t *idx = reinterpret_cast<int32_t *>(wsb + L.idx);
+    float *w = reinterpret_cast<float *>(wsb + L.w);
+    int32_t *offsets = reinterpret_cast<int32_t *>(wsb + L.offsets);
+    int32_t *row = reinterpret_cast<int32_t *>(wsb + L.row);
+    moe_bf16 *xperm = reinterpret_cast<moe_bf16 *>(wsb + L.xperm);
+    moe_bf16 *H = reinterpret_cast<moe_bf16 *>(wsb + L.H);
+    float *Y = reinterpret_cast<float *>(wsb + L.Y);
+
+    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    if (st != MOE_OK) return st;
+    st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
+                    reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s);
+    if (st != MOE_OK) return st;
+
+    ScatterLaunch c;
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.k = k;
+    c.x = x;
+    c.idx = idx;
+    c.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
+    c.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
+    c.x_perm = xperm;
+    c.row_of_slot = row;
+    c.err = err;
+    st = from_cuda(launch_scatter(c, s));
+    if (st != MOE_OK) return st;
+
+    // A token never picks one expert twice, so no segment exceeds T rows.
+    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y, err, s);
+    if (st != MOE_OK) return st;
+
+    const float *shared_y = nullptr;
+    if (d_ff_shared > 0) {
+        moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
+        float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
+        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys, err, s);
+        if (st != MOE_OK) return st;
+        shared_y = Ys;
+    }
+
+    CombineLaunch cb;
+    cb.T = T;
+    cb.d = d;
+    cb.k = k;
+    cb.y = Y;
+    cb.row_of_slot = row;
+    cb.w = w;
+    cb.shared_y = shared_y;
+    cb.out = out;
+    return from_cuda(launch_combine(cb, s));
+}
+
+moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                       const moe_bf16 *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
+                       const moe_bf16 *W2, float *out, void *ws, size_t ws_bytes,
+                       moe_stream_t stream)
+{
+    return moe_forward_ex(T, d, E, d_ff, k, x, Wg, nullptr, W1, W3, W2, 0, nullptr, nullptr,
+                          nullptr, out, ws, ws_bytes, stream);
+}
+
+moe_status moe_get_device_error(const void *ws, uint32_t *code, moe_stream_t stream)
+{
+    if (ws == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (code) *code = word;
+    if (word == 0) return MOE_OK;
+    if (word & (MOE_DEVERR_TIMEOUT_TMA | MOE_DEVERR_TIMEOUT_MMA | MOE_DEVERR_TIMEOUT_EPI))
+        return MOE_ERR_TIMEOUT;
+    return MOE_ERR_DEVICE;
+}
+
+}  // extern "C"

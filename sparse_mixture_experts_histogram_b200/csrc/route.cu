@@ -1,0 +1,298 @@
+// route.cu -- router kernel: logits = x Wg^T on the tensor cores (tcgen05,
+// accumulators in tensor memory, operands brought in by TMA), then in the
+// epilogue the per-token top-k (ties to the lower expert index), the softmax
+// over the k selected logits, the per-tile expert histogram with stable
+// ranks, and -- in the last tile to finish -- the expert offsets.
+//
+// One CTA routes 128 tokens (the MMA's M).  Warp 0 issues TMA loads, warp 1
+// issues the MMAs, warps 2..5 are the epilogue (thread = token row).
+//
+// Method: "Mistral 8x7B SMoE architecture" (jsqmd.com) sec. 3.2, the gate
+// linear followed by torch.topk and a softmax over the selected values;
+// "MoE" (theaiera.top, LLMs-from-scratch ch.10) sec. 10.3 (weights sum to
+// 1) and sec. 10.4 (per-expert token lists, here the histogram).
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteMaxStages = 8;
+constexpr int kRouteThreads = 192;
+constexpr uint32_t kRouteABytes = 128 * 128;   // 128 token rows x 64 bf16
+
+struct RouteParams {
+    int T, d, E, Npad, stages, ntiles;
+    uint32_t tmem_cols;
+    const float *bias;
+    int32_t *idx;
+    float *w;
+    uint32_t *err;
+    DispatchOut dout;
+};
+
+__host__ __device__ constexpr uint32_t route_stage_bytes(int Npad)
+{
+    return kRouteABytes + static_cast<uint32_t>(Npad) * 128u;
+}
+
+constexpr size_t kRouteFixedSmem = 1024 /* alignment slack */ + 2 * kRouteMaxStages * 8 + 8 + 16 +
+                                   kMaxE * sizeof(float) + sizeof(DispatchSmem) + 64;
+
+template <int K>
+__device__ __forceinline__ void topk_insert(float (&tv)[K], int (&ti)[K], float v, int e)
+{
+    if (v > tv[K - 1]) {
+#pragma unroll
+        for (int j = K - 1; j > 0; --j) {
+            if (v > tv[j]) {
+                if (v > tv[j - 1]) {
+                    tv[j] = tv[j - 1];
+                    ti[j] = ti[j - 1];
+                } else {
+                    tv[j] = v;
+                    ti[j] = e;
+                }
+            }
+        }
+        if (v > tv[0]) {
+            tv[0] = v;
+            ti[0] = e;
+        }
+    }
+}
+
+// Waits for the copies the producer issued into each stage to land, so that
+// no copy is still writing shared memory when the CTA exits after an abort.
+__device__ __forceinline__ void drain_stages(uint64_t *full, const uint32_t *last_parity,
+                                             uint32_t issued_mask, int stages)
+{
+    for (int s = 0; s < stages; ++s) {
+        if (!(issued_mask & (1u << s))) continue;
+        const uint64_t t0 = ptx::globaltimer();
+        while (!ptx::mbar_try_wait(&full[s], last_parity[s])) {
+            if (ptx::globaltimer() - t0 > 100000000ull) break;  // 100 ms
+        }
+    }
+}
+
+template <int K>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+    route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWg,
+                 const RouteParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t stage_bytes = route_stage_bytes(p.Npad);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.stages * stage_bytes);
+    uint64_t *empty = full + kRouteMaxStages;
+    uint64_t *tfull = empty + kRouteMaxStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tfull + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    uint32_t *epi_fail = tmem_slot + 2;
+    float *bias_s = reinterpret_cast<float *>(tmem_slot + 4);
+    DispatchSmem &ds = *reinterpret_cast<DispatchSmem *>(bias_s + kMaxE);
+
+    const int tile = blockIdx.x;
+    const int ksteps = p.d / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        ptx::mbar_init(tfull, 1);
+        *abort_flag = 0u;
+        *epi_fail = 0u;
+        ptx::fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        ptx::prefetch_tensormap(&tmX);
+        ptx::prefetch_tensormap(&tmWg);
+    }
+    for (int e = threadIdx.x; e < kMaxE; e += blockDim.x)
+        bias_s[e] = (p.bias != nullptr && e < p.E) ? p.bias[e] : 0.0f;
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, p.tmem_cols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, issued = 0;
+            uint32_t last_parity[kRouteMaxStages];
+            for (int s = 0; s < kRouteMaxStages; ++s) last_parity[s] = 0;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                if (!bounded_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrTimeoutMma))
+                    break;
+                uint8_t *sa = smem + stage * stage_bytes;
+                ptx::mbar_arrive_expect_tx(&full[stage], stage_bytes);
+                ptx::tma_load_2d(sa, &tmX, &full[stage], ks * 64, tile * kTileTokens);
+                ptx::tma_load_2d(sa + kRouteABytes, &tmWg, &full[stage], ks * 64, 0);
+                issued |= 1u << stage;
+                last_parity[stage] = phase;
+                if (++stage == static_cast<uint32_t>(p.stages)) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            drain_stages(full, last_parity, issued, p.stages);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(128, p.Npad);
+            uint32_t stage = 0, phase = 0;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                if (!bounded_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutTma)) break;
+                ptx::tc_fence_after();
+                const uint32_t sa = ptx::smem_addr(smem + stage * stage_bytes);
+                const uint32_t sb = sa + kRouteABytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    ptx::tc_mma_bf16(tmem, ptx::sw128_kmajor_desc(sa + kk * 32),
+                                     ptx::sw128_kmajor_desc(sb + kk * 32), idesc,
+                                     (ks | kk) ? 1u : 0u);
+                ptx::tc_commit(&empty[stage]);
+                if (++stage == static_cast<uint32_t>(p.stages)) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // Arrives once every MMA issued above has completed (also after
+            // an abort, so the epilogue never reads half-written tensor memory
+            // while MMAs still run).
+            ptx::tc_commit(tfull);
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        const int t = tile * kTileTokens + row;
+        const bool ok_w = bounded_wait_warp(tfull, 0u, abort_flag, p.err, kErrTimeoutMma);
+        if (lane == 0 && !ok_w) atomicOr(epi_fail, 1u);
+        ptx::named_bar(1, 128);
+        const bool ok = (*reinterpret_cast<volatile uint32_t *>(epi_fail) == 0u);
+        ptx::tc_fence_after();
+
+        float tv[K];
+        int ti[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            tv[j] = -CUDART_INF_F;
+            ti[j] = -1;
+        }
+        if (ok) {
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
+            for (int c0 = 0; c0 < p.Npad; c0 += 16) {
+                uint32_t r[16];
+                ptx::tmem_ld16(tbase + static_cast<uint32_t>(c0), r);
+                ptx::tc_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int e = c0 + jj;
+                    if (e < p.E) topk_insert<K>(tv, ti, __uint_as_float(r[jj]) + bias_s[e], e);
+                }
+            }
+        }
+        ptx::tc_fence_before();
+
+        const bool valid = ok && (t < p.T);
+        if (valid) {
+            const float m = tv[0];
+            float ex[K];
+            float s = 0.0f;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                ex[j] = expf(tv[j] - m);
+                s += ex[j];
+            }
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                p.idx[static_cast<size_t>(t) * K + j] = ti[j];
+                p.w[static_cast<size_t>(t) * K + j] = ex[j] / s;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < K; ++j) ds.sel[row][j] = valid ? ti[j] : -1;
+        dispatch_tile(ds, row, tile, p.T, p.E, K, p.dout, 1);
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+template <int K>
+cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
+{
+    const int Npad = ((a.E + 15) / 16) * 16 < 16 ? 16 : ((a.E + 15) / 16) * 16;
+    const uint32_t sb = route_stage_bytes(Npad);
+    int stages = static_cast<int>((227 * 1024 - kRouteFixedSmem) / sb);
+    if (stages > kRouteMaxStages) stages = kRouteMaxStages;
+    const size_t smem = kRouteFixedSmem + static_cast<size_t>(stages) * sb;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(Npad)) cols <<= 1;
+
+    CUtensorMap tmX, tmWg;
+    cudaError_t e = make_tmap_bf16(&tmX, a.x, a.T, a.d, 128);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(&tmWg, a.Wg, a.E, a.d, static_cast<uint32_t>(Npad));
+    if (e != cudaSuccess) return e;
+
+    e = cudaFuncSetAttribute(route_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+
+    RouteParams p;
+    p.T = a.T;
+    p.d = a.d;
+    p.E = a.E;
+    p.Npad = Npad;
+    p.stages = stages;
+    p.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
+    p.tmem_cols = cols;
+    p.bias = a.bias;
+    p.idx = a.idx;
+    p.w = a.w;
+    p.err = a.err;
+    p.dout.tilecnt = a.tilecnt;
+    p.dout.tilebase = a.tilebase;
+    p.dout.rank = a.rank;
+    p.dout.offsets = a.offsets;
+    p.dout.counts = a.counts;
+    p.dout.done = a.done;
+    p.dout.ntiles = p.ntiles;
+    route_kernel<K><<<p.ntiles, kRouteThreads, smem, s>>>(tmX, tmWg, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s)
+{
+    switch (a.k) {
+    case 1: return launch_route_k<1>(a, s);
+    case 2: return launch_route_k<2>(a, s);
+    case 3: return launch_route_k<3>(a, s);
+    case 4: return launch_route_k<4>(a, s);
+    case 5: return launch_route_k<5>(a, s);
+    case 6: return launch_route_k<6>(a, s);
+    case 7: return launch_route_k<7>(a, s);
+    case 8: return launch_route_k<8>(a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,266 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64
+oracle on the same seeded inputs (tolerances in tests/gpu_util.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_mixture_experts_histogram_b200 as moe
+from sparse_mixture_experts_histogram_b200 import synth
+from sparse_mixture_experts_histogram_b200.synth import Workload, bits
+
+from gpu_util import (assert_close, check_forward, check_routing, gpu_forward, sample_tokens,
+                      workspace)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _inputs(wl, seed=42, device=DEV):
+    if device == DEV:
+        # small workloads are drawn on the CPU (same bits as the CPU tests),
+        # large ones on the GPU
+        return {k: (None if v is None else v.to(DEV)) for k, v in
+                synth.make_inputs(wl, seed=seed, device="cpu").items()}
+    return synth.make_inputs(wl, seed=seed, device=device)
+
+
+# ------------------------------------------------------------------ routing
+ROUTE_CASES = [
+    synth.small(),
+    *synth.sweep(),
+    Workload("T1_E8_k2", 1, 512, 8, 128, 2),
+    Workload("T129_E64_k4", 129, 256, 64, 128, 4),
+    Workload("T300_E256_k8", 300, 384, 256, 128, 8),
+    Workload("T257_E5_k5", 257, 128, 5, 128, 5),
+    Workload("T200_E3_k1", 200, 128, 3, 128, 1),
+    Workload("T640_E17_k3", 640, 640, 17, 128, 3),
+]
+
+
+@pytest.mark.parametrize("wl", ROUTE_CASES, ids=lambda w: w.name)
+def test_route_matches_oracle(wl):
+    check_routing(wl, _inputs(wl))
+
+
+def test_route_equal_logits_pick_lowest_indices():
+    wl = Workload("ties", 300, 256, 16, 128, 4)
+    inp = _inputs(wl)
+    inp["Wg"] = torch.zeros_like(inp["Wg"])
+    idx, r, near = check_routing(wl, inp)
+    assert (idx == np.arange(4)).all()
+
+
+def test_route_skewed_bias():
+    wl = synth.mixtral_prefill(2048, skew=True)
+    inp = synth.make_inputs(wl, device=DEV)
+    idx, r, near = check_routing(wl, inp)
+    share = float((idx[:, 0] == synth.SKEW_EXPERT).mean())
+    assert 0.30 < share < 0.55, share
+
+
+# ------------------------------------------------------------------ permute
+def _expected_dispatch(idx, E):
+    T, k = idx.shape
+    counts = np.bincount(idx.ravel(), minlength=E)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    row = np.empty_like(idx)
+    fill = offsets[:-1].copy()
+    for t in range(T):                      # stable: token order within an expert
+        for j in range(k):
+            e = idx[t, j]
+            row[t, j] = fill[e]
+            fill[e] += 1
+    return offsets, row
+
+
+PERMUTE_CASES = [
+    (Workload("T1_E8_k2", 1, 128, 8, 128, 2), "random"),
+    (Workload("T129_E8_k2", 129, 256, 8, 128, 2), "random"),
+    (Workload("T1000_E64_k4", 1000, 128, 64, 128, 4), "random"),
+    (Workload("T700_E256_k8", 700, 256, 256, 128, 8), "random"),
+    (Workload("T513_E8_k1_one_expert", 513, 128, 8, 128, 1), "one"),
+    (Workload("T5_E256_k1_mostly_empty", 5, 128, 256, 128, 1), "random"),
+]
+
+
+@pytest.mark.parametrize("wl,mode", PERMUTE_CASES, ids=lambda c: getattr(c, "name", c))
+def test_permute_matches_stable_grouping(wl, mode):
+    inp = _inputs(wl)
+    g = np.random.default_rng(5)
+    if mode == "one":
+        idx = np.full((wl.T, wl.k), 3, np.int32)
+    else:
+        idx = np.stack([g.choice(wl.E, size=wl.k, replace=False) for _ in range(wl.T)]).astype(np.int32)
+    offsets_ref, row_ref = _expected_dispatch(idx, wl.E)
+    S = wl.T * wl.k
+    d_idx = torch.as_tensor(idx, device=DEV)
+    offsets = torch.empty(wl.E + 1, dtype=torch.int32, device=DEV)
+    row = torch.empty(wl.T, wl.k, dtype=torch.int32, device=DEV)
+    xp = torch.empty(S, wl.d, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(wl)
+    moe.moe_permute(wl.T, wl.d, wl.E, wl.k, inp["x"], d_idx, offsets, row, xp, ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 0, hex(code)
+    assert np.array_equal(offsets.cpu().numpy(), offsets_ref)
+    assert np.array_equal(row.cpu().numpy(), row_ref)
+    xb = bits(inp["x"])
+    xpb = bits(xp)
+    for t in range(wl.T):
+        for j in range(wl.k):
+            assert np.array_equal(xpb[row_ref[t, j]], xb[t])
+
+
+def test_permute_flags_out_of_range_expert():
+    wl = Workload("bad_idx", 64, 128, 8, 128, 2)
+    inp = _inputs(wl)
+    idx = np.tile(np.array([[0, 1]], np.int32), (64, 1))
+    idx[5, 1] = 9  # outside [0, E)
+    d_idx = torch.as_tensor(idx, device=DEV)
+    offsets = torch.empty(9, dtype=torch.int32, device=DEV)
+    row = torch.empty(64, 2, dtype=torch.int32, device=DEV)
+    xp = torch.zeros(128, 128, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(wl)
+    moe.moe_permute(64, 128, 8, 2, inp["x"], d_idx, offsets, row, xp, ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 5 and code & 0x10
+    assert row.cpu().numpy()[5, 1] == -1
+
+
+# ------------------------------------------------------------------ experts
+FFN_SEGMENTS = [
+    ("ragged", 512, 384, [0, 1, 15, 16, 17, 127, 128, 129, 300, 0, 33]),
+    ("one_big", 256, 256, [700]),
+    ("tiny", 128, 128, [1, 2, 3]),
+    ("wide_ff", 384, 1024, [40, 0, 200, 5]),
+]
+
+
+@pytest.mark.parametrize("name,d,d_ff,sizes", FFN_SEGMENTS, ids=lambda c: c if isinstance(c, str) else None)
+def test_expert_ffn_matches_oracle(name, d, d_ff, sizes):
+    E = len(sizes)
+    S = int(sum(sizes))
+    wl = Workload(name, S, d, E, d_ff, 1)
+    inp = _inputs(wl, seed=11)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    y = torch.empty(S, d, dtype=torch.float32, device=DEV)
+    ws = workspace(wl)
+    moe.moe_expert_ffn(S, d, E, d_ff, inp["x"], torch.as_tensor(offsets, device=DEV), inp["W1"],
+                       inp["W3"], inp["W2"], y, ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 0, hex(code)
+    y = y.cpu().numpy()
+    xb = bits(inp["x"])
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        ref = oracle.swiglu(xb[a:b], bits(inp["W1"][e]), bits(inp["W3"][e]), bits(inp["W2"][e]))
+        assert_close(y[a:b], ref, f"{name} expert {e}")
+
+
+def test_expert_ffn_rejects_inconsistent_offsets():
+    wl = Workload("bad_offsets", 64, 128, 4, 128, 1)
+    inp = _inputs(wl)
+    offsets = torch.tensor([0, 40, 20, 64, 64], dtype=torch.int32, device=DEV)  # decreasing
+    y = torch.full((64, 128), 7.0, dtype=torch.float32, device=DEV)
+    ws = workspace(wl)
+    moe.moe_expert_ffn(64, 128, 4, 128, inp["x"], offsets, inp["W1"], inp["W3"], inp["W2"], y, ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 5 and code & 0x8
+    assert (y == 7.0).all()  # nothing computed
+
+
+# ------------------------------------------------------------------ combine
+def test_combine_weighted_sum_in_slot_order():
+    T, d, k = 77, 256, 3
+    g = torch.Generator().manual_seed(3)
+    y = torch.randn(T * k, d, generator=g)
+    perm = torch.randperm(T * k, generator=g).reshape(T, k).to(torch.int32)
+    w = torch.rand(T, k, generator=g)
+    ys = torch.randn(T, d, generator=g)
+    out = torch.empty(T, d, device=DEV)
+    moe.moe_combine(T, d, k, y.to(DEV), perm.to(DEV), w.to(DEV), ys.to(DEV), out)
+    torch.cuda.synchronize()
+    ref = (w.double().unsqueeze(-1) * y.double()[perm.long()]).sum(1) + ys.double()
+    assert_close(out.cpu().numpy(), ref.numpy(), "combine")
+
+
+# ------------------------------------------------------------------ whole layer
+SMALL_FORWARD = [synth.small(), *synth.sweep(),
+                 Workload("dense_E1_k1", 300, 256, 1, 512, 1),
+                 Workload("k_equals_E", 130, 256, 4, 256, 4),
+                 Workload("T1", 1, 512, 8, 1024, 2),
+                 Workload("T129_ragged", 129, 384, 16, 640, 3),
+                 Workload("E256_k8_small", 200, 256, 256, 128, 8),
+                 Workload("shared_small", 150, 256, 32, 256, 4, d_ff_shared=384)]
+
+
+@pytest.mark.parametrize("wl", SMALL_FORWARD, ids=lambda w: w.name)
+def test_forward_matches_oracle_all_tokens(wl):
+    check_forward(wl, _inputs(wl))
+
+
+def test_forward_all_tokens_one_expert():
+    # a bias that sends every token to expert 2 first: one segment of T rows
+    wl = Workload("one_expert", 600, 256, 8, 256, 2)
+    inp = _inputs(wl)
+    inp["bias"] = torch.tensor([0, 0, 50.0, 0, 0, 0, 0, 0], dtype=torch.float32, device=DEV)
+    check_forward(wl, inp)
+
+
+def test_forward_equal_logits_mean_of_first_k():
+    wl = Workload("ties_forward", 64, 256, 8, 256, 3)
+    inp = _inputs(wl)
+    inp["Wg"] = torch.zeros_like(inp["Wg"])
+    check_forward(wl, inp)
+
+
+def test_forward_is_deterministic_and_graph_capturable():
+    wl = synth.small()
+    inp = _inputs(wl)
+    ws = workspace(wl)
+    a = gpu_forward(wl, inp, ws).clone()
+    b = gpu_forward(wl, inp, ws).clone()
+    assert torch.equal(a, b)
+    out = torch.empty_like(a)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        moe.moe_forward(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["W1"],
+                        inp["W3"], inp["W2"], out, ws, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    out.zero_()
+    with torch.cuda.graph(g, stream=s):
+        moe.moe_forward(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["W1"],
+                        inp["W3"], inp["W2"], out, ws, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, a)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 128])
+def test_forward_mixtral_decode(T):
+    wl = synth.mixtral_decode(T)
+    inp = synth.make_inputs(wl, device=DEV)
+    idx, r, near = check_routing(wl, inp)
+    tok = sample_tokens(T, 12, idx, near)
+    check_forward(wl, inp, tokens=tok, r=r)
+
+
+@pytest.mark.parametrize("T,skew", [(2048, False), (2048, True), (8192, False), (8192, True)])
+def test_forward_mixtral_prefill(T, skew):
+    wl = synth.mixtral_prefill(T, skew)
+    inp = synth.make_inputs(wl, device=DEV)
+    idx, r, near = check_routing(wl, inp)
+    tok = sample_tokens(T, 12, idx, near)
+    check_forward(wl, inp, tokens=tok, r=r)
+
+
+def test_forward_fine_grained_shared():
+    wl = synth.fine_grained(8192)
+    inp = synth.make_inputs(wl, device=DEV)
+    idx, r, near = check_routing(wl, inp)
+    tok = sample_tokens(wl.T, 8, None, near)
+    check_forward(wl, inp, tokens=tok, r=r)
