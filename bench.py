@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Throughput of the B200 sparse MoE feed-forward layer (forward pass).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One JSON line on rank 0.  A *step* is one pass of the whole layer (routing,
+dispatch, both expert GEMMs, combine) over one batch of every layer of the
+workload.  The default workload is the fixed-total-parameter granularity
+sweep of the "万亿 MoE 只激活 4.9%" page: T = 512 tokens, d = 512,
+E * d_ff = 32768, (E, d_ff, k) in {(8,4096,1), (8,4096,2), (32,1024,1),
+(32,1024,2), (64,512,4), (128,256,8)} -- six layers, 604 MB of bf16 weights,
+more than the 126 MB L2, so every step streams its weights from HBM.
+
+Metric: MoE-layer tokens/s (tokens x layers per second) and active TFLOP/s.
+Timing: K steps captured in one CUDA graph (with CUDA events recorded at
+every kernel boundary, so each kernel's duration comes from the same timed
+region), bracketed by a barrier and device synchronisation, max over ranks.
+Multi-GPU is weak scaling: every rank runs the same workload on its own seeded
+batch with its own weights (data parallel replicas, no collective on the data
+path).  ``--impl reference`` times the fp64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_histogram_b200 import accounting as acc  # noqa: E402
+from sparse_mixture_experts_histogram_b200 import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s & active TFLOP/s, % of bf16 tensor / HBM roofline"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+# ----------------------------------------------------------------------------- workloads
+def workload(name: str) -> list:
+    if name == "sweep":
+        return synth.sweep()
+    if name == "small":
+        return [synth.small()]
+    if name.startswith("mixtral_prefill_T"):
+        rest = name[len("mixtral_prefill_T"):]
+        skew = rest.endswith("_skewed")
+        return [synth.mixtral_prefill(int(rest.replace("_skewed", "")), skew)]
+    if name.startswith("mixtral_decode_T"):
+        return [synth.mixtral_decode(int(name[len("mixtral_decode_T"):]))]
+    if name.startswith("fine_grained_T"):
+        return [synth.fine_grained(int(name[len("fine_grained_T"):]))]
+    raise SystemExit(f"unknown workload {name}")
+
+
+def describe(wls, name):
+    return {
+        "workload": ("granularity_sweep_T512_d512_Edff32768" if name == "sweep" else name),
+        "layers": [{"T": w.T, "d": w.d, "E": w.E, "d_ff": w.d_ff, "k": w.k,
+                    **({"d_ff_shared": w.d_ff_shared} if w.d_ff_shared else {}),
+                    **({"router_bias": f"+{synth.SKEW_BIAS} on expert {synth.SKEW_EXPERT}"}
+                       if w.skew else {})} for w in wls],
+        "global_batch_tokens": sum(w.T for w in wls),
+    }
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in a thread."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append((time.time(), parts))
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=2)
+        except Exception:
+            self.proc.kill()
+        win = [p for (t, p) in self.samples if t0 - 0.1 <= t <= t1 + 0.1] or \
+            [p for (_, p) in self.samples]
+        mhz = [float(p[0]) for p in win if p[0].replace(".", "").isdigit()]
+        mx = [float(p[1]) for p in win if p[1].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for p in win for i in range(4) if p[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(win)}
+
+
+def clocks_bad(c) -> bool:
+    if any(r in BAD_REASONS for r in c.get("reasons", [])):
+        return True
+    if c.get("sm_mhz") and c.get("sm_max_mhz"):
+        if c["sm_mhz"] < 0.6 * c["sm_max_mhz"] and not c["reasons"]:
+            return True
+    return False
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_init(nccl: bool):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and nccl:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def dist_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_step_fn(wls, seed, tokens_per_layer):
+    """A bounded sample of one step on the host cores: the oracle's forward of
+    ``tokens_per_layer`` seeded tokens of every layer."""
+    import oracle
+    from sparse_mixture_experts_histogram_b200.synth import bits
+    data = []
+    g = np.random.default_rng(seed)
+    for wl in wls:
+        inp = synth.make_inputs(wl, seed=seed, device="cpu")
+        b = None if inp["bias"] is None else inp["bias"].double().numpy()
+        shared = (bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"])) if wl.d_ff_shared else None
+        arrs = [bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")]
+        tok = np.sort(g.choice(wl.T, size=min(tokens_per_layer, wl.T), replace=False))
+        data.append((wl, arrs, b, shared, tok))
+
+    def step():
+        n = 0
+        for wl, arrs, b, shared, tok in data:
+            oracle.forward(*arrs, wl.k, bias=b, tokens=tok, shared=shared)
+            n += len(tok)
+        return n
+    return step
+
+
+def run_oracle(wls, steps, warmup, target_s=2.0, seed=42):
+    """Times the oracle: calibrate a per-layer token sample that takes about
+    ``target_s`` per step, then run ``warmup`` + ``steps`` steps."""
+    import oracle
+    oracle.build()
+    probe = oracle_step_fn(wls, seed, 4)
+    t0 = time.perf_counter()
+    n = probe()
+    dt = max(time.perf_counter() - t0, 1e-6)
+    per_tok = dt / n
+    tpl = int(max(1, min(max(w.T for w in wls), target_s / per_tok / len(wls))))
+    step = oracle_step_fn(wls, seed, tpl)
+    for _ in range(warmup):
+        step()
+    t0 = time.perf_counter()
+    tot = 0
+    for _ in range(steps):
+        tot += step()
+    el = time.perf_counter() - t0
+    return {"value": tot / el, "tokens_per_layer": tpl, "seconds": el, "steps": steps,
+            "cores": oracle.num_threads()}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    wls = workload(args.workload)
+    r = run_oracle(wls, args.steps, args.warmup, target_s=args.oracle_step_s)
+    sample = (f"{r['tokens_per_layer']} seeded tokens of each of the {len(wls)} layer(s) per step "
+              f"(fp64 oracle, all routing and expert work of those tokens)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * r["seconds"] / r["steps"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": describe(wls, args.workload),
+        "cpu_baseline": {"value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": r["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def traffic_record(kernel_key):
+    """DRAM traffic per launch of the dominant kernel from a committed ncu
+    capture, if the kernel sources have not changed since."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    r = rec.get(kernel_key)
+    if not r:
+        return None
+    h = hashlib.sha256()
+    for src in r.get("sources", []):
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != r.get("sources_sha256"):
+        return None
+    return r
+
+
+def gpu_arm(args):
+    import sparse_mixture_experts_histogram_b200 as moe
+    rank, world, local = dist_init(nccl=True)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wls = workload(args.workload)
+    seed = synth.rank_seed(42, rank)
+    moe.load_library()
+
+    # ---- resident inputs and buffers
+    inps, outs = [], []
+    for i, wl in enumerate(wls):
+        inps.append(synth.make_inputs(wl, seed=seed + i, device=dev))
+        outs.append(torch.empty(wl.T, wl.d, dtype=torch.float32, device=dev))
+    ws_bytes = max(moe.moe_workspace_size_ex(w.T, w.d, w.E, w.d_ff, w.k, w.d_ff_shared)
+                   for w in wls)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- routing pre-pass: experts each batch hits (for the algorithmic bytes)
+    hit = []
+    with torch.cuda.stream(stream):
+        for wl, inp in zip(wls, inps):
+            idx = torch.empty(wl.T, wl.k, dtype=torch.int32, device=dev)
+            w = torch.empty(wl.T, wl.k, dtype=torch.float32, device=dev)
+            cnt = torch.empty(wl.E, dtype=torch.int32, device=dev)
+            moe.moe_route(wl.T, wl.d, wl.E, wl.k, inp["x"], inp["Wg"], inp["bias"], idx, w, cnt,
+                          ws, stream=stream)
+            stream.synchronize()
+            hit.append(int((cnt > 0).sum().item()))
+
+    def layer_call(i, events=None):
+        wl, inp = wls[i], inps[i]
+        a = (wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["bias"], inp["W1"],
+             inp["W3"], inp["W2"], wl.d_ff_shared, inp.get("Ws1"), inp.get("Ws3"),
+             inp.get("Ws2"), outs[i], ws)
+        if events is None:
+            moe.moe_forward_ex(*a, stream=stream)
+        else:
+            moe.moe_forward_traced(*a, events, stream=stream)
+
+    def make_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for e in evs:
+                e.record(stream)
+        stream.synchronize()
+        return evs
+
+    # ---- eager warm-up (loads kernels, sets attributes)
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            for i in range(len(wls)):
+                layer_call(i)
+    stream.synchronize()
+    st, code = moe.moe_get_device_error(ws, stream)
+    if st != 0:
+        raise SystemExit(f"device error word {code:#x} after warm-up")
+
+    # ---- graphs: one step (warm-up / soak) and K traced steps (timed)
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        for i in range(len(wls)):
+            layer_call(i)
+    trace = [[make_events(moe.binding.TRACE_EVENTS) for _ in wls] for _ in range(args.steps)]
+    gK = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gK, stream=stream):
+        for s in range(args.steps):
+            for i in range(len(wls)):
+                layer_call(i, trace[s][i])
+    gK_plain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gK_plain, stream=stream):
+        for s in range(args.steps):
+            for i in range(len(wls)):
+                layer_call(i)
+
+    def timed(graph_k, soak_s=1.0):
+        sampler = ClockSampler(local)
+        t_start = time.time()
+        with torch.cuda.stream(stream):
+            n = 0
+            while n < args.warmup or time.time() - t_start < soak_s:
+                g1.replay()
+                n += 1
+                if n % 50 == 0:
+                    stream.synchronize()
+        stream.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        tw0 = time.time()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            graph_k.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        tw1 = time.time()
+        barrier(world)
+        ms = dist_max(e0.elapsed_time(e1), world)
+        return ms, sampler.stop(t_start, tw1)
+
+    ms, clocks = timed(gK)
+    if clocks_bad(clocks):
+        ms, clocks = timed(gK)
+        clocks["remeasured"] = True
+    ms_plain, _ = timed(gK_plain, soak_s=0.2)
+    st, code = moe.moe_get_device_error(ws, stream)
+    if st != 0:
+        raise SystemExit(f"device error word {code:#x} after the timed region")
+
+    # ---- per-kernel durations from the trace events of the timed region
+    stages = moe.binding.TRACE_STAGES
+    dur = {s: [] for s in stages}        # ms per launch
+    per_layer_up = [[] for _ in wls]
+    for s in range(args.steps):
+        for i, wl in enumerate(wls):
+            ev = trace[s][i]
+            for j, name in enumerate(stages):
+                t = ev[j].elapsed_time(ev[j + 1])
+                if name.startswith("shared") and not wl.d_ff_shared:
+                    continue
+                dur[name].append(t)
+                if name == "up_gemm":
+                    per_layer_up[i].append(t)
+    kernel_ms = {k: (sum(v) / len(v) if v else None) for k, v in dur.items()}
+    kernel_share = {k: (sum(v) / max(1e-12, sum(sum(x) for x in dur.values())))
+                    for k, v in dur.items() if v}
+
+    # ---- throughput and roofline
+    tokens_per_step = sum(w.T for w in wls)
+    flops_per_step = sum(acc.active_flops(w.T, w.d, w.E, w.d_ff, w.k, w.d_ff_shared) for w in wls)
+    bytes_per_step = sum(acc.algorithmic_bytes(w.T, w.d, w.E, w.d_ff, w.k, h, w.d_ff_shared)
+                         for w, h in zip(wls, hit))
+    sec = ms / 1e3
+    value = world * tokens_per_step * args.steps / sec
+    pk, pk_src = peaks()
+    # dominant kernel: the up-projection GEMM (W1|W3 + SwiGLU)
+    up_bytes = [acc.gemm_bytes("up", w.T, w.d, w.d_ff, w.k, h, w.d_ff_shared) for w, h in
+                zip(wls, hit)]
+    up_flops = [acc.gemm_flops("up", w.T, w.d, w.d_ff, w.k, w.d_ff_shared) for w in wls]
+    up_time = [sum(t) / len(t) for t in per_layer_up]
+    ai = sum(up_flops) / sum(up_bytes)
+    ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    if ai >= ridge:
+        achieved = sum(up_flops) / sum(up_time) / 1e9  # TFLOP/s (ms -> 1e-3)
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "peak_source": f"bf16_tflops_sustained ({pk_src})"}
+    else:
+        achieved = sum(up_bytes) / sum(up_time) / 1e6  # GB/s
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "peak_source": f"hbm_gbs ({pk_src})"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = traffic_record(f"up_gemm:{args.workload}")
+    roof["traffic"] = None if tr is None else tr["bytes_per_launch"]
+    roof["kernel"] = "gemm_kernel<up> (W1|W3 grouped GEMM + SwiGLU epilogue)"
+    roof["algorithmic_bytes_per_launch"] = sum(up_bytes) / len(up_bytes)
+    roof["launch_ms"] = sum(up_time) / len(up_time)
+    step_roof = max(flops_per_step / (pk["bf16_tflops_sustained"] * 1e12),
+                    bytes_per_step / (pk["hbm_gbs"] * 1e9))
+
+    # ---- end to end through the public API with host buffers
+    xs_host = [inp["x"].cpu().pin_memory() for inp in inps]
+    out_host = [torch.empty(w.T, w.d, dtype=torch.float32).pin_memory() for w in wls]
+    x_dev = [torch.empty_like(inp["x"]) for inp in inps]
+
+    def e2e_step():
+        for i in range(len(wls)):
+            x_dev[i].copy_(xs_host[i], non_blocking=True)
+            wl, inp = wls[i], inps[i]
+            moe.moe_forward_ex(wl.T, wl.d, wl.E, wl.d_ff, wl.k, x_dev[i], inp["Wg"], inp["bias"],
+                               inp["W1"], inp["W3"], inp["W2"], wl.d_ff_shared, inp.get("Ws1"),
+                               inp.get("Ws3"), inp.get("Ws2"), outs[i], ws, stream=stream)
+            out_host[i].copy_(outs[i], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+    stream.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1), world)
+    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+    h2d = sum(w.T * w.d * 2 for w in wls)
+    d2h = sum(w.T * w.d * 4 for w in wls)
+    ok = all(torch.isfinite(o).all().item() for o in outs)
+
+    launches_per_layer = [5 + (2 if w.d_ff_shared else 0) for w in wls]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**describe(wls, args.workload), "parallelism": f"dp{world} (replicas)",
+                   "l2": ("no flush: the step's working set "
+                          f"({bytes_per_step / 1e6:.0f} MB of algorithmic bytes) exceeds the "
+                          "126 MB L2" if bytes_per_step > L2_BYTES else
+                          "working set below L2 size: warm-L2 number")},
+        "active_tflops": world * flops_per_step * args.steps / sec / 1e12,
+        "step_roofline_frac": step_roof * args.steps / sec * 1.0,
+        "roofline": roof,
+        "kernel_ms": kernel_ms,
+        "kernel_share": kernel_share,
+        "ms_per_step_untraced": ms_plain / args.steps,
+        "experts_hit": hit,
+        "gpu_launches": sum(launches_per_layer) * args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
+                "path": "pinned host x -> device copy, moe_forward_ex, device -> pinned host out, "
+                        "eager launches on one stream"},
+        "clocks": clocks,
+        "outputs_finite": ok,
+        "cpu_baseline": None,
+    }
+    del g1, gK, gK_plain
+    if world == 1 and not args.no_cpu_baseline:
+        r = run_oracle(wls, steps=2, warmup=0, target_s=args.oracle_step_s)
+        line["cpu_baseline"] = {
+            "value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+            "sample": (f"{r['tokens_per_layer']} seeded tokens of each of the {len(wls)} layers, "
+                       f"2 steps, {r['seconds']:.1f} s on the host cores (fp64 oracle)")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="sweep")
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--oracle-step-s", type=float, default=5.0,
+                    help="seconds of host work per oracle step (bounded sample)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return reference_arm(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    return gpu_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -165,6 +165,27 @@ MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const mo
                           const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
                           float *out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Number of events moe_forward_traced records. */
+#define MOE_TRACE_EVENTS 8
+
+/* moe_forward_ex that also records caller-created CUDA events (cudaEvent_t,
+ * created with timing enabled) on `stream` at the kernel boundaries, so the
+ * caller can time each kernel with cudaEventElapsedTime:
+ *   events[0] before the router kernel      events[4] before the shared up GEMM
+ *   events[1] before the dispatch scatter   events[5] before the shared down GEMM
+ *   events[2] before the up GEMM (W1|W3)    events[6] before the combine
+ *   events[3] before the down GEMM (W2)     events[7] after the combine
+ * (events[4..5] mark the same point as events[6] when there is no shared
+ * expert).  n_events must be MOE_TRACE_EVENTS.  While `stream` is being
+ * captured into a CUDA graph the events are recorded as graph event nodes.
+ * The layer's work and results are those of moe_forward_ex. */
+MOE_API moe_status moe_forward_traced(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                                      const moe_bf16 *Wg, const float *router_bias,
+                                      const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2,
+                                      int d_ff_shared, const moe_bf16 *Ws1, const moe_bf16 *Ws3,
+                                      const moe_bf16 *Ws2, float *out, void *ws, size_t ws_bytes,
+                                      moe_stream_t stream, void *const *events, int n_events);
+
 /* Waits for `stream`, then reads the device error word of workspace `ws`
  * into *code (may be NULL).  Returns MOE_OK if it is zero, MOE_ERR_TIMEOUT
  * if a timeout bit is set, MOE_ERR_DEVICE for any other bit, MOE_ERR_CUDA if

@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     moe_expert_ffn,
     moe_forward,
     moe_forward_ex,
+    moe_forward_traced,
     moe_get_device_error,
     moe_permute,
     moe_route,

@@ -26,7 +26,11 @@ DEVERR_BITS = {0x1: "TIMEOUT_TMA", 0x2: "TIMEOUT_MMA", 0x4: "TIMEOUT_EPI", 0x8: 
 #: Every symbol the C header declares (checked against ``include/moe.h`` by the tests).
 ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "moe_permute",
                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_ex",
-                 "moe_get_device_error", "moe_status_string")
+                 "moe_forward_traced", "moe_get_device_error", "moe_status_string")
+TRACE_EVENTS = 8
+#: What each of moe_forward_traced's events marks (event i = start of stage i).
+TRACE_STAGES = ("route", "scatter", "up_gemm", "down_gemm", "shared_up_gemm",
+                "shared_down_gemm", "combine")
 
 
 class MoEError(RuntimeError):
@@ -62,6 +66,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
             "moe_combine": (_I, [_I] * 3 + [_P] * 5 + [_P]),
             "moe_forward": (_I, [_I] * 5 + [_P] * 7 + [_SZ, _P]),
             "moe_forward_ex": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P]),
+            "moe_forward_traced": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P, _P, _I]),
             "moe_get_device_error": (_I, [_P, _P, _P]),
             "moe_status_string": (ctypes.c_char_p, [_I]),
         }
@@ -154,6 +159,22 @@ def moe_forward_ex(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared
                                          _ptr(W1), _ptr(W3), _ptr(W2), d_ff_shared, _ptr(Ws1),
                                          _ptr(Ws3), _ptr(Ws2), _ptr(out), _ptr(ws),
                                          _ws_bytes(ws), _stream(stream)), "moe_forward_ex")
+
+
+def moe_forward_traced(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,
+                       Ws2, out, ws, events, stream=None):
+    """``events``: TRACE_EVENTS torch.cuda.Event(enable_timing=True) objects
+    (or raw cudaEvent_t handles as ints)."""
+    if len(events) != TRACE_EVENTS:
+        raise ValueError(f"need {TRACE_EVENTS} events")
+    arr = (ctypes.c_void_p * TRACE_EVENTS)(
+        *[e if isinstance(e, int) else e.cuda_event for e in events])
+    _check(load_library().moe_forward_traced(T, d, E, d_ff, k, _ptr(x), _ptr(Wg),
+                                             _ptr(router_bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                                             d_ff_shared, _ptr(Ws1), _ptr(Ws3), _ptr(Ws2),
+                                             _ptr(out), _ptr(ws), _ws_bytes(ws),
+                                             _stream(stream), arr, TRACE_EVENTS),
+           "moe_forward_traced")
 
 
 def moe_get_device_error(ws, stream=None) -> tuple[int, int]:

@@ -241,10 +241,12 @@ moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int3
     return from_cuda(launch_scatter(c, s));
 }
 
+static moe_status mark(void *const *events, int i, cudaStream_t s);
+
 static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const moe_bf16 *x_perm,
                            const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
                            const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *err,
-                           cudaStream_t s)
+                           cudaStream_t s, void *const *events = nullptr, int ev0 = 0)
 {
     GemmLaunch g;
     g.up = 1;
@@ -259,8 +261,11 @@ static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const mo
     g.B = x_perm;
     g.out = H;
     g.err = err;
-    moe_status st = from_cuda(launch_gemm(g, s));
+    moe_status st = mark(events, ev0, s);
     if (st != MOE_OK) return st;
+    st = from_cuda(launch_gemm(g, s));
+    if (st != MOE_OK) return st;
+    if ((st = mark(events, ev0 + 1, s)) != MOE_OK) return st;
     g.up = 0;
     g.M_rows = d;
     g.K = d_ff;
@@ -312,11 +317,25 @@ moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *
     return from_cuda(launch_combine(c, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
-                          const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
-                          const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
-                          const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
-                          float *out, void *ws, size_t ws_bytes, moe_stream_t stream)
+// Records event i (if any) on the stream; inside stream capture as a graph
+// event node.
+static moe_status mark(void *const *events, int i, cudaStream_t s)
+{
+    if (events == nullptr || events[i] == nullptr) return MOE_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaEvent_t ev = static_cast<cudaEvent_t>(events[i]);
+    if (cs == cudaStreamCaptureStatusActive)
+        return from_cuda(cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal));
+    return from_cuda(cudaEventRecord(ev, s));
+}
+
+static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                               const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
+                               const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
+                               const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
+                               float *out, void *ws, size_t ws_bytes, moe_stream_t stream,
+                               void *const *events)
 {
     moe_status st = check_shapes(T, d, E, d_ff, k, d_ff_shared);
     if (st != MOE_OK) return st;
@@ -344,6 +363,7 @@ moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *
 
     st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
     if (st != MOE_OK) return st;
+    if ((st = mark(events, 0, s)) != MOE_OK) return st;
     st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
                     reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s);
     if (st != MOE_OK) return st;
@@ -360,21 +380,27 @@ moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *
     c.x_perm = xperm;
     c.row_of_slot = row;
     c.err = err;
+    if ((st = mark(events, 1, s)) != MOE_OK) return st;
     st = from_cuda(launch_scatter(c, s));
     if (st != MOE_OK) return st;
 
     // A token never picks one expert twice, so no segment exceeds T rows.
-    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y, err, s);
+    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y, err, s, events, 2);
     if (st != MOE_OK) return st;
 
     const float *shared_y = nullptr;
     if (d_ff_shared > 0) {
         moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
         float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
-        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys, err, s);
+        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys, err, s, events,
+                      4);
         if (st != MOE_OK) return st;
         shared_y = Ys;
+    } else {
+        if ((st = mark(events, 4, s)) != MOE_OK) return st;
+        if ((st = mark(events, 5, s)) != MOE_OK) return st;
     }
+    if ((st = mark(events, 6, s)) != MOE_OK) return st;
 
     CombineLaunch cb;
     cb.T = T;
@@ -385,7 +411,31 @@ moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *
     cb.w = w;
     cb.shared_y = shared_y;
     cb.out = out;
-    return from_cuda(launch_combine(cb, s));
+    st = from_cuda(launch_combine(cb, s));
+    if (st != MOE_OK) return st;
+    return mark(events, 7, s);
+}
+
+moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                          const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
+                          const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
+                          const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
+                          float *out, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    return forward_impl(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,
+                        Ws2, out, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_traced(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                              const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
+                              const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
+                              const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
+                              float *out, void *ws, size_t ws_bytes, moe_stream_t stream,
+                              void *const *events, int n_events)
+{
+    if (events == nullptr || n_events != MOE_TRACE_EVENTS) return MOE_ERR_INVALID_ARG;
+    return forward_impl(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,
+                        Ws2, out, ws, ws_bytes, stream, events);
 }
 
 moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
