@@ -165,6 +165,30 @@ MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const mo
                           const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
                           float *out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_expert_ffn for callers that cannot allocate device memory: the same
+ * computation, arguments and results as moe_expert_ffn, minus the workspace.
+ * The pages have no counterpart of this entry point; it exists for code that
+ * may not call cudaMalloc (a plugin handed only its tensors by a host program
+ * that owns all device memory, or a loop that must stay out of the
+ * allocator), which still owns x_perm, offsets, the weights and y_perm.
+ *   The intermediate H [S, d_ff] bf16 lives in a fixed 32 MiB device array
+ *   inside the library (every GPU that loads the library keeps it until the
+ *   process exits): S * d_ff * 2 must be at most 32 MiB - 256 bytes, larger
+ *   sizes return MOE_ERR_WORKSPACE.  Nothing is allocated and no allocating
+ *   routine is called.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   All calls share the one array: calls that may overlap on the GPU (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.  The array keeps the last call's contents; the call clears its
+ *   error word itself.  The device error word of this entry point is not
+ *   readable through moe_get_device_error. */
+MOE_API moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
+                                         const int32_t *offsets, const moe_bf16 *W1,
+                                         const moe_bf16 *W3, const moe_bf16 *W2, float *y_perm,
+                                         moe_stream_t stream);
+
 /* Number of events moe_forward_traced records. */
 #define MOE_TRACE_EVENTS 8
 

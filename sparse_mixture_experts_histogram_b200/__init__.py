@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     load_library,
     moe_combine,
     moe_expert_ffn,
+    moe_expert_ffn_static,
     moe_forward,
     moe_forward_ex,
     moe_forward_traced,

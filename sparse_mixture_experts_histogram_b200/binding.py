@@ -26,7 +26,8 @@ DEVERR_BITS = {0x1: "TIMEOUT_TMA", 0x2: "TIMEOUT_MMA", 0x4: "TIMEOUT_EPI", 0x8: 
 #: Every symbol the C header declares (checked against ``include/moe.h`` by the tests).
 ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "moe_permute",
                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_ex",
-                 "moe_forward_traced", "moe_get_device_error", "moe_status_string")
+                 "moe_forward_traced", "moe_get_device_error", "moe_status_string",
+                 "moe_expert_ffn_static")
 TRACE_EVENTS = 8
 #: What each of moe_forward_traced's events marks (event i = start of stage i).
 TRACE_STAGES = ("route", "scatter", "up_gemm", "down_gemm", "shared_up_gemm",
@@ -68,6 +69,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
             "moe_forward_ex": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P]),
             "moe_forward_traced": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P, _P, _I]),
             "moe_get_device_error": (_I, [_P, _P, _P]),
+            "moe_expert_ffn_static": (_I, [_I] * 4 + [_P] * 6 + [_P]),
             "moe_status_string": (ctypes.c_char_p, [_I]),
         }
         for name, (res, args) in sig.items():
@@ -140,6 +142,15 @@ def moe_expert_ffn(S, d, E, d_ff, x_perm, offsets, W1, W3, W2, y_perm, ws, strea
     _check(load_library().moe_expert_ffn(S, d, E, d_ff, _ptr(x_perm), _ptr(offsets), _ptr(W1),
                                          _ptr(W3), _ptr(W2), _ptr(y_perm), _ptr(ws),
                                          _ws_bytes(ws), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_static(S, d, E, d_ff, x_perm, offsets, W1, W3, W2, y_perm, stream=None):
+    """moe_expert_ffn without a workspace argument, for callers that cannot
+    allocate device memory: the intermediate lives in a fixed 32 MiB array
+    inside the library (see include/moe.h for its limit and sharing rules)."""
+    _check(load_library().moe_expert_ffn_static(S, d, E, d_ff, _ptr(x_perm), _ptr(offsets),
+                                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(y_perm),
+                                                _stream(stream)), "moe_expert_ffn_static")
 
 
 def moe_combine(T, d, k, y_perm, row_of_slot, w, shared_y, out, stream=None):
