@@ -12,9 +12,9 @@ E * d_ff = 32768, (E, d_ff, k) in {(8,4096,1), (8,4096,2), (32,1024,1),
 more than the 126 MB L2, so every step streams its weights from HBM.
 
 Metric: MoE-layer tokens/s (tokens x layers per second) and active TFLOP/s.
-Timing: K steps captured in one CUDA graph (with CUDA events recorded at
-every kernel boundary, so each kernel's duration comes from the same timed
-region), bracketed by a barrier and device synchronisation, max over ranks.
+Timing: K steps captured in one CUDA graph, bracketed by a barrier and device
+synchronisation, max over ranks; a second pass of the same K steps, captured
+with CUDA events at every kernel boundary, gives each kernel's duration.
 Multi-GPU is weak scaling: every rank runs the same workload on its own seeded
 batch with its own weights (data parallel replicas, no collective on the data
 path).  ``--impl reference`` times the fp64 CPU oracle instead.
@@ -160,12 +160,19 @@ def dist_init(nccl: bool):
 
 
 def dist_max(v: float, world: int) -> float:
+    """Max of ``v`` over the ranks (the slowest rank's time)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes ``tokens_per_step`` per step."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
 
 
 def barrier(world):
@@ -370,11 +377,15 @@ def gpu_arm(args):
         ms = dist_max(e0.elapsed_time(e1), world)
         return ms, sampler.stop(t_start, tw1)
 
-    ms, clocks = timed(gK)
+    # Timed region: K steps of the plain graph.  A second pass of the same K
+    # steps with events at every kernel boundary gives each kernel's duration
+    # (event nodes add a few microseconds each, so they stay out of the
+    # headline number).
+    ms, clocks = timed(gK_plain)
     if clocks_bad(clocks):
-        ms, clocks = timed(gK)
+        ms, clocks = timed(gK_plain)
         clocks["remeasured"] = True
-    ms_plain, _ = timed(gK_plain, soak_s=0.2)
+    ms_traced, _ = timed(gK, soak_s=0.2)
     st, code = moe.moe_get_device_error(ws, stream)
     if st != 0:
         raise SystemExit(f"device error word {code:#x} after the timed region")
@@ -383,6 +394,7 @@ def gpu_arm(args):
     stages = moe.binding.TRACE_STAGES
     dur = {s: [] for s in stages}        # ms per launch
     per_layer_up = [[] for _ in wls]
+    per_layer = [{s: [] for s in stages} for _ in wls]
     for s in range(args.steps):
         for i, wl in enumerate(wls):
             ev = trace[s][i]
@@ -391,6 +403,7 @@ def gpu_arm(args):
                 if name.startswith("shared") and not wl.d_ff_shared:
                     continue
                 dur[name].append(t)
+                per_layer[i][name].append(t)
                 if name == "up_gemm":
                     per_layer_up[i].append(t)
     kernel_ms = {k: (sum(v) / len(v) if v else None) for k, v in dur.items()}
@@ -403,7 +416,7 @@ def gpu_arm(args):
     bytes_per_step = sum(acc.algorithmic_bytes(w.T, w.d, w.E, w.d_ff, w.k, h, w.d_ff_shared)
                          for w, h in zip(wls, hit))
     sec = ms / 1e3
-    value = world * tokens_per_step * args.steps / sec
+    value = weak_scaling_value(world, tokens_per_step, args.steps, ms)
     pk, pk_src = peaks()
     # dominant kernel: the up-projection GEMM (W1|W3 + SwiGLU)
     up_bytes = [acc.gemm_bytes("up", w.T, w.d, w.d_ff, w.k, h, w.d_ff_shared) for w, h in
@@ -457,7 +470,7 @@ def gpu_arm(args):
         e1.record(stream)
     stream.synchronize()
     e2e_ms = dist_max(e0.elapsed_time(e1), world)
-    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+    e2e_value = weak_scaling_value(world, tokens_per_step, args.steps, e2e_ms)
     h2d = sum(w.T * w.d * 2 for w in wls)
     d2h = sum(w.T * w.d * 4 for w in wls)
     ok = all(torch.isfinite(o).all().item() for o in outs)
@@ -477,7 +490,9 @@ def gpu_arm(args):
         "roofline": roof,
         "kernel_ms": kernel_ms,
         "kernel_share": kernel_share,
-        "ms_per_step_untraced": ms_plain / args.steps,
+        "kernel_ms_per_layer": [{k: round(sum(v) / len(v), 5) for k, v in pl.items() if v}
+                                for pl in per_layer],
+        "ms_per_step_traced": ms_traced / args.steps,
         "experts_hit": hit,
         "gpu_launches": sum(launches_per_layer) * args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

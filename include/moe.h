@@ -116,8 +116,9 @@ MOE_API moe_status moe_route(int T, int d, int E, int k, const moe_bf16 *x, cons
  *   row_of_slot [T,k] int32 out: the x_perm row that holds (token t, slot j)
  *   x_perm [S,d] bf16 out: x_perm[row_of_slot[t,j]] = x[t]
  * Within an expert's rows the order is by token index (stable), so the
- * result is deterministic.  An index outside [0,E) sets MOE_DEVERR_INDEX
- * and that pair is skipped.  Passage: theaiera.top sec. 10.4 (mask,
+ * result is deterministic.  An index outside [0,E), or an expert repeated
+ * within a token, sets MOE_DEVERR_INDEX and that pair is skipped (its
+ * row_of_slot entry is -1).  Passage: theaiera.top sec. 10.4 (mask,
  * nonzero and index_select per expert). */
 MOE_API moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int32_t *idx,
                        int32_t *offsets, int32_t *row_of_slot, moe_bf16 *x_perm, void *ws,

@@ -23,6 +23,7 @@ constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, rank
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
+    size_t tilectr, zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
     size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, xperm, H, Y, Hs, Ys, total;
 };
 
@@ -38,6 +39,8 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     };
     const size_t ntiles = (static_cast<size_t>(T) + 127) / 128;
     const size_t S = static_cast<size_t>(T) * k;
+    L.tilectr = take(ntiles * 4);
+    L.zero_bytes = o;
     L.tilecnt = take(ntiles * E * 4);
     L.tilebase = take(ntiles * E * 4);
     L.rank = take(S * 4);
@@ -48,7 +51,7 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     L.row = take(S * 4);
     L.xperm = take(S * d * 2);
     L.H = take(S * d_ff * 2);
-    L.Y = take(S * d * 4);
+    L.Y = take(S * d * 4 * static_cast<size_t>(down_ksplit(static_cast<int>(S), E, d, d_ff)));
     if (d_ffs > 0) {
         L.Hs = take(static_cast<size_t>(T) * d_ffs * 2);
         L.Ys = take(static_cast<size_t>(T) * d * 4);
@@ -175,6 +178,7 @@ static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, cons
     a.tilebase = reinterpret_cast<int32_t *>(ws + L.tilebase);
     a.rank = reinterpret_cast<int32_t *>(ws + L.rank);
     a.done = reinterpret_cast<uint32_t *>(ws + 4);
+    a.tile_ctr = reinterpret_cast<uint32_t *>(ws + L.tilectr);
     a.err = reinterpret_cast<uint32_t *>(ws);
     return from_cuda(launch_route(a, s));
 }
@@ -192,7 +196,7 @@ moe_status moe_route(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf
     const Layout L = forward_layout(T, d, E, 128, k, 0);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
-    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    st = from_cuda(cudaMemsetAsync(wsb, 0, L.zero_bytes, s));
     if (st != MOE_OK) return st;
     return route_impl(T, d, E, k, x, Wg, router_bias, idx, w, counts,
                       reinterpret_cast<int32_t *>(wsb + L.offsets), wsb, L, s);
@@ -238,6 +242,7 @@ moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int3
     c.x_perm = x_perm;
     c.row_of_slot = row_of_slot;
     c.err = r.err;
+    c.pdl = true;
     return from_cuda(launch_scatter(c, s));
 }
 
@@ -246,7 +251,8 @@ static moe_status mark(void *const *events, int i, cudaStream_t s);
 static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const moe_bf16 *x_perm,
                            const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
                            const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *err,
-                           cudaStream_t s, void *const *events = nullptr, int ev0 = 0)
+                           cudaStream_t s, bool pdl_first, int ksplit,
+                           void *const *events = nullptr, int ev0 = 0)
 {
     GemmLaunch g;
     g.up = 1;
@@ -261,11 +267,15 @@ static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const mo
     g.B = x_perm;
     g.out = H;
     g.err = err;
+    g.ksplit = 1;
+    g.pdl = pdl_first && events == nullptr;
     moe_status st = mark(events, ev0, s);
     if (st != MOE_OK) return st;
     st = from_cuda(launch_gemm(g, s));
     if (st != MOE_OK) return st;
     if ((st = mark(events, ev0 + 1, s)) != MOE_OK) return st;
+    g.pdl = events == nullptr;
+    g.ksplit = ksplit;
     g.up = 0;
     g.M_rows = d;
     g.K = d_ff;
@@ -294,7 +304,7 @@ moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
     if (st != MOE_OK) return st;
     return ffn_impl(S, d, E, d_ff, S, x_perm, offsets, W1, W3, W2,
                     reinterpret_cast<moe_bf16 *>(wsb + kHeaderBytes), y_perm,
-                    reinterpret_cast<uint32_t *>(wsb), s);
+                    reinterpret_cast<uint32_t *>(wsb), s, false, 1);
 }
 
 moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *row_of_slot,
@@ -309,11 +319,13 @@ moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *
     c.T = T;
     c.d = d;
     c.k = k;
+    c.ksplit = 1;
     c.y = y_perm;
     c.row_of_slot = row_of_slot;
     c.w = w;
     c.shared_y = shared_y;
     c.out = out;
+    c.pdl = false;
     return from_cuda(launch_combine(c, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -361,7 +373,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     moe_bf16 *H = reinterpret_cast<moe_bf16 *>(wsb + L.H);
     float *Y = reinterpret_cast<float *>(wsb + L.Y);
 
-    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    st = from_cuda(cudaMemsetAsync(wsb, 0, L.zero_bytes, s));
     if (st != MOE_OK) return st;
     if ((st = mark(events, 0, s)) != MOE_OK) return st;
     st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
@@ -380,20 +392,23 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     c.x_perm = xperm;
     c.row_of_slot = row;
     c.err = err;
+    c.pdl = events == nullptr;
     if ((st = mark(events, 1, s)) != MOE_OK) return st;
     st = from_cuda(launch_scatter(c, s));
     if (st != MOE_OK) return st;
 
     // A token never picks one expert twice, so no segment exceeds T rows.
-    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y, err, s, events, 2);
+    const int ksplit = down_ksplit(S, E, d, d_ff);
+    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y, err, s, true, ksplit,
+                  events, 2);
     if (st != MOE_OK) return st;
 
     const float *shared_y = nullptr;
     if (d_ff_shared > 0) {
         moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
         float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
-        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys, err, s, events,
-                      4);
+        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys, err, s, true, 1,
+                      events, 4);
         if (st != MOE_OK) return st;
         shared_y = Ys;
     } else {
@@ -406,11 +421,13 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     cb.T = T;
     cb.d = d;
     cb.k = k;
+    cb.ksplit = ksplit;
     cb.y = Y;
     cb.row_of_slot = row;
     cb.w = w;
     cb.shared_y = shared_y;
     cb.out = out;
+    cb.pdl = events == nullptr;
     st = from_cuda(launch_combine(cb, s));
     if (st != MOE_OK) return st;
     return mark(events, 7, s);

@@ -10,27 +10,49 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace moe {
 
 namespace {
 
 constexpr int kCombineWarps = 8;
+constexpr int kCombineVec = 2;   // float4 per lane per chunk
+constexpr int kCombineBatch = 8; // (slot, partial) pairs whose loads are in flight together
 
 struct CombineParams {
     int T, d, k;
+    int ksplit;          // partial outputs per row, summed in order before weighting
+    size_t part_stride;  // float4 between consecutive partial outputs
     const float4 *y;
     const int32_t *row_of_slot;
     const float *w;
     const float4 *shared_y;
     float4 *out;
+    int chunks;          // chunks of 32*kCombineVec float4 per row
 };
 
+__device__ __forceinline__ void add4(float4 &a, const float4 &b)
+{
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+}
+
+// One warp per (token, chunk of 32*kCombineVec float4).  The (slot j,
+// partial q) pairs are visited j-major: y_j = sum_q partial_q(row_j), then
+// acc += w_j * y_j, so the order of every addition is fixed.  Loads of
+// kCombineBatch pairs are issued before any of them is used.
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineParams p)
 {
+    ptx::grid_dep_launch();
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    const int gw = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    const int t = gw / p.chunks;
+    const int c = gw - t * p.chunks;
     if (t >= p.T) return;
+    ptx::grid_dep_wait();
     int my_row = -1;
     float my_w = 0.0f;
     if (lane < p.k) {
@@ -38,34 +60,61 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
         my_w = p.w[static_cast<size_t>(t) * p.k + lane];
         if (my_row >= p.T * p.k) my_row = -1;  // rows live in [0, T*k)
     }
-    int rows[kMaxK];
-    float ws[kMaxK];
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-        rows[j] = __shfl_sync(0xffffffffu, my_row, j);
-        ws[j] = __shfl_sync(0xffffffffu, my_w, j);
-    }
     const int nv = p.d >> 2;
-    for (int v = lane; v < nv; v += 32) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int npairs = p.k * p.ksplit;
+    float4 acc[kCombineVec], yj[kCombineVec];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            if (j < p.k && rows[j] >= 0) {
-                const float4 y = __ldg(p.y + static_cast<size_t>(rows[j]) * nv + v);
-                acc.x = fmaf(ws[j], y.x, acc.x);
-                acc.y = fmaf(ws[j], y.y, acc.y);
-                acc.z = fmaf(ws[j], y.z, acc.z);
-                acc.w = fmaf(ws[j], y.w, acc.w);
+    for (int u = 0; u < kCombineVec; ++u) {
+        acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        yj[u] = acc[u];
+    }
+    for (int p0 = 0; p0 < npairs; p0 += kCombineBatch) {
+        float4 val[kCombineBatch][kCombineVec];
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i) {
+            const int pi = p0 + i;
+            const int j = pi / p.ksplit;
+            const int q = pi - j * p.ksplit;
+            const int row = __shfl_sync(0xffffffffu, my_row, j & 31);
+            const bool ok = pi < npairs && row >= 0;
+            const float4 *src = p.y + q * p.part_stride + static_cast<size_t>(ok ? row : 0) * nv;
+#pragma unroll
+            for (int u = 0; u < kCombineVec; ++u) {
+                const int v = (c * kCombineVec + u) * 32 + lane;
+                val[i][u] = (ok && v < nv) ? __ldg(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-        if (p.shared_y != nullptr) {
-            const float4 s = __ldg(p.shared_y + static_cast<size_t>(t) * nv + v);
-            acc.x += s.x;
-            acc.y += s.y;
-            acc.z += s.z;
-            acc.w += s.w;
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i) {
+            const int pi = p0 + i;
+            if (pi < npairs) {
+                const int j = pi / p.ksplit;
+                const int q = pi - j * p.ksplit;
+#pragma unroll
+                for (int u = 0; u < kCombineVec; ++u) {
+                    if (q == 0) yj[u] = val[i][u];
+                    else add4(yj[u], val[i][u]);
+                }
+                if (q == p.ksplit - 1) {
+                    const float wj = __shfl_sync(0xffffffffu, my_w, j & 31);
+#pragma unroll
+                    for (int u = 0; u < kCombineVec; ++u) {
+                        acc[u].x = fmaf(wj, yj[u].x, acc[u].x);
+                        acc[u].y = fmaf(wj, yj[u].y, acc[u].y);
+                        acc[u].z = fmaf(wj, yj[u].z, acc[u].z);
+                        acc[u].w = fmaf(wj, yj[u].w, acc[u].w);
+                    }
+                }
+            }
         }
-        p.out[static_cast<size_t>(t) * nv + v] = acc;
+    }
+#pragma unroll
+    for (int u = 0; u < kCombineVec; ++u) {
+        const int v = (c * kCombineVec + u) * 32 + lane;
+        if (v < nv) {
+            if (p.shared_y != nullptr) add4(acc[u], __ldg(p.shared_y + static_cast<size_t>(t) * nv + v));
+            p.out[static_cast<size_t>(t) * nv + v] = acc[u];
+        }
     }
 }
 
@@ -82,9 +131,13 @@ cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s)
     p.w = a.w;
     p.shared_y = reinterpret_cast<const float4 *>(a.shared_y);
     p.out = reinterpret_cast<float4 *>(a.out);
-    const int blocks = (a.T + kCombineWarps - 1) / kCombineWarps;
-    combine_kernel<<<blocks, 32 * kCombineWarps, 0, s>>>(p);
-    return cudaGetLastError();
+    p.ksplit = a.ksplit < 1 ? 1 : a.ksplit;
+    p.part_stride = static_cast<size_t>(a.T) * a.k * (a.d / 4);
+    const int nv = a.d / 4;
+    p.chunks = (nv + 32 * kCombineVec - 1) / (32 * kCombineVec);
+    const long long warps = static_cast<long long>(a.T) * p.chunks;
+    const int blocks = static_cast<int>((warps + kCombineWarps - 1) / kCombineWarps);
+    return launch_pdl(combine_kernel, dim3(blocks), dim3(32 * kCombineWarps), 0, s, a.pdl, p);
 }
 
 }  // namespace moe

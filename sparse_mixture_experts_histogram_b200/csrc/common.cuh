@@ -88,22 +88,30 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
 {
     const int q = row >> 5;
     const int lane = row & 31;
-    for (int i = row; i < 4 * kMaxE; i += kTileTokens) (&sm.cnt[0][0])[i] = 0;
+    uint32_t *mask = reinterpret_cast<uint32_t *>(&sm.cnt[0][0]);  // [4][kMaxE] lane bitmasks
+    for (int i = row; i < 4 * kMaxE; i += kTileTokens) mask[i] = 0u;
     ptx::named_bar(bar_id, kTileTokens);
 
-    // Each lane owns the experts e == lane (mod 32) of its group and walks the
-    // group's 32 rows in order.
-    for (int t = 32 * q; t < 32 * q + 32; ++t) {
-        for (int j = 0; j < k; ++j) {
-            const int e = sm.sel[t][j];
-            if (e >= 0 && (e & 31) == lane) {
-                sm.rnk[t][j] = sm.cnt[q][e];
-                sm.cnt[q][e] += 1;
-            }
-        }
+    // Bit `lane` of mask[q][e] is set when row 32q+lane chose expert e (a row
+    // never chooses an expert twice).  The rank of (row, j) among its group's
+    // rows with the same expert is the number of lower lanes in that mask.
+    for (int j = 0; j < k; ++j) {
+        const int e = sm.sel[row][j];
+        if (e >= 0) atomicOr(&mask[q * kMaxE + e], 1u << lane);
     }
     ptx::named_bar(bar_id, kTileTokens);
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+        const int e = sm.sel[row][j];
+        if (e >= 0) sm.rnk[row][j] = __popc(mask[q * kMaxE + e] & below);
+    }
+    ptx::named_bar(bar_id, kTileTokens);  // every rank read its mask before it is replaced
+    // cnt[g][e] = popc(mask[g][e]), in place.
+    for (int i = row; i < 4 * kMaxE; i += kTileTokens)
+        sm.cnt[0][i] = __popc(mask[i]);
+    ptx::named_bar(bar_id, kTileTokens);
 
+    const bool single = (o.ntiles == 1);
     for (int e = row; e < E; e += kTileTokens) {
         int run = 0;
 #pragma unroll
@@ -111,7 +119,8 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
             sm.pre[g][e] = run;
             run += sm.cnt[g][e];
         }
-        o.tilecnt[(size_t)tile * E + e] = run;
+        if (single) sm.tot[e] = run;
+        else o.tilecnt[(size_t)tile * E + e] = run;
     }
     ptx::named_bar(bar_id, kTileTokens);
 
@@ -122,34 +131,36 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
             o.rank[(size_t)t * k + j] = (e >= 0) ? sm.pre[q][e] + sm.rnk[row][j] : -1;
         }
     }
-    __threadfence();
-    ptx::named_bar(bar_id, kTileTokens);
-    if (row == 0) sm.is_last = (atomicAdd(o.done, 1u) == (uint32_t)o.ntiles - 1u) ? 1u : 0u;
-    ptx::named_bar(bar_id, kTileTokens);
-    if (!sm.is_last) return;
-    __threadfence();
+    if (!single) {
+        __threadfence();
+        ptx::named_bar(bar_id, kTileTokens);
+        if (row == 0) sm.is_last = (atomicAdd(o.done, 1u) == (uint32_t)o.ntiles - 1u) ? 1u : 0u;
+        ptx::named_bar(bar_id, kTileTokens);
+        if (!sm.is_last) return;
+        __threadfence();
 
-    // Last tile: per expert, exclusive prefix of the tile counts (relative
-    // tile bases) and the expert total.
-    for (int e = row; e < E; e += kTileTokens) {
-        int run = 0;
-        int tl = 0;
-        for (; tl + 8 <= o.ntiles; tl += 8) {
-            int c[8];
+        // Last tile: per expert, exclusive prefix of the tile counts (relative
+        // tile bases) and the expert total.
+        for (int e = row; e < E; e += kTileTokens) {
+            int run = 0;
+            int tl = 0;
+            for (; tl + 8 <= o.ntiles; tl += 8) {
+                int c[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) c[u] = __ldcg(&o.tilecnt[(size_t)(tl + u) * E + e]);
+                for (int u = 0; u < 8; ++u) c[u] = __ldcg(&o.tilecnt[(size_t)(tl + u) * E + e]);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                o.tilebase[(size_t)(tl + u) * E + e] = run;
-                run += c[u];
+                for (int u = 0; u < 8; ++u) {
+                    o.tilebase[(size_t)(tl + u) * E + e] = run;
+                    run += c[u];
+                }
             }
+            for (; tl < o.ntiles; ++tl) {
+                const int c = __ldcg(&o.tilecnt[(size_t)tl * E + e]);
+                o.tilebase[(size_t)tl * E + e] = run;
+                run += c;
+            }
+            sm.tot[e] = run;
         }
-        for (; tl < o.ntiles; ++tl) {
-            const int c = __ldcg(&o.tilecnt[(size_t)tl * E + e]);
-            o.tilebase[(size_t)tl * E + e] = run;
-            run += c;
-        }
-        sm.tot[e] = run;
     }
     ptx::named_bar(bar_id, kTileTokens);
 
@@ -183,9 +194,13 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
         o.offsets[e] = off;
         if (e < E && o.counts) o.counts[e] = ((e + 1 < E) ? sm.tot[e + 1] : sm.total) - off;
     }
-    const int n = o.ntiles * E;
-    for (int i = row; i < n; i += kTileTokens) o.tilebase[i] += sm.tot[i % E];
-    if (row == 0) *o.done = 0u;
+    if (single) {
+        for (int e = row; e < E; e += kTileTokens) o.tilebase[e] = sm.tot[e];
+    } else {
+        const int n = o.ntiles * E;
+        for (int i = row; i < n; i += kTileTokens) o.tilebase[i] += sm.tot[i % E];
+        if (row == 0) *o.done = 0u;
+    }
 }
 
 }  // namespace moe

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -35,7 +36,9 @@ __global__ void __launch_bounds__(kTileTokens) ranks_kernel(const RanksParams p)
         int e = -1;
         if (t < p.T && j < p.k) {
             e = p.idx[static_cast<size_t>(t) * p.k + j];
-            if (e < 0 || e >= p.E) {
+            bool bad = (e < 0 || e >= p.E);
+            for (int jj = 0; jj < j; ++jj) bad |= (ds.sel[row][jj] == e);  // repeated expert
+            if (bad) {
                 atomicOr(p.err, kErrIndex);
                 e = -1;
             }
@@ -53,15 +56,25 @@ struct ScatterParams {
     int32_t *row_of_slot;
     uint32_t *err;
     int S;
+    int chunks;  // 16-byte-vector chunks of kScatterVec*32 per row
 };
 
 constexpr int kScatterWarps = 8;
+constexpr int kScatterVec = 4;  // 16-byte vectors per lane per chunk
 
+// One warp per (token, chunk of 32*kScatterVec 16-byte vectors): the rows of
+// the token's k slots are computed by lanes 0..k-1 and broadcast, then each
+// lane loads its kScatterVec vectors of x (independent loads in flight) and
+// stores them to the k rows.
 __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const ScatterParams p)
 {
+    ptx::grid_dep_launch();
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kScatterWarps + (threadIdx.x >> 5);
+    const int gw = blockIdx.x * kScatterWarps + (threadIdx.x >> 5);
+    const int t = gw / p.chunks;
+    const int c = gw - t * p.chunks;
     if (t >= p.T) return;
+    ptx::grid_dep_wait();
     int my_row = -1;
     if (lane < p.k) {
         const size_t s = static_cast<size_t>(t) * p.k + lane;
@@ -71,19 +84,32 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
             const int row = p.tilebase[static_cast<size_t>(t / kTileTokens) * p.E + e] + r;
             if (row >= 0 && row < p.S) my_row = row;
         }
-        if (my_row < 0) atomicOr(p.err, kErrIndex);
-        p.row_of_slot[s] = my_row;
+        if (c == 0) {
+            if (my_row < 0) atomicOr(p.err, kErrIndex);
+            p.row_of_slot[s] = my_row;
+        }
     }
     int rows[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
     const int nv = p.d >> 3;  // 16-byte vectors per row
     const uint4 *src = p.x + static_cast<size_t>(t) * nv;
-    for (int v = lane; v < nv; v += 32) {
-        const uint4 val = __ldg(src + v);
+    uint4 val[kScatterVec];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-            if (j < p.k && rows[j] >= 0) p.x_perm[static_cast<size_t>(rows[j]) * nv + v] = val;
+    for (int u = 0; u < kScatterVec; ++u) {
+        const int v = (c * kScatterVec + u) * 32 + lane;
+        if (v < nv) val[u] = __ldg(src + v);
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        if (j < p.k && rows[j] >= 0) {
+            uint4 *dst = p.x_perm + static_cast<size_t>(rows[j]) * nv;
+#pragma unroll
+            for (int u = 0; u < kScatterVec; ++u) {
+                const int v = (c * kScatterVec + u) * 32 + lane;
+                if (v < nv) dst[v] = val[u];
+            }
+        }
     }
 }
 
@@ -123,9 +149,11 @@ cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s)
     p.row_of_slot = a.row_of_slot;
     p.err = a.err;
     p.S = a.T * a.k;
-    const int blocks = (a.T + kScatterWarps - 1) / kScatterWarps;
-    scatter_kernel<<<blocks, 32 * kScatterWarps, 0, s>>>(p);
-    return cudaGetLastError();
+    const int nv = a.d / 8;
+    p.chunks = (nv + 32 * kScatterVec - 1) / (32 * kScatterVec);
+    const long long warps = static_cast<long long>(a.T) * p.chunks;
+    const int blocks = static_cast<int>((warps + kScatterWarps - 1) / kScatterWarps);
+    return launch_pdl(scatter_kernel, dim3(blocks), dim3(32 * kScatterWarps), 0, s, a.pdl, p);
 }
 
 }  // namespace moe

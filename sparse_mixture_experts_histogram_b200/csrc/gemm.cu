@@ -27,8 +27,11 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -41,20 +44,22 @@ constexpr size_t kGemmFixedSmem = 1024 /* alignment slack */ + (2 * kGemmMaxStag
                                   2 * (kMaxE + 1) * sizeof(int32_t) + 64;
 constexpr size_t kSmemBudget = 227 * 1024;
 
-template <bool UP, int BN>
+template <bool UP, int BN, int ST>
 struct Cfg {
     static constexpr int kA = UP ? 2 : 1;
     static constexpr uint32_t kBBytes = BN * 128u;
     static constexpr uint32_t kStageBytes = kA * kWTileBytes + kBBytes;
     static constexpr int kAccCols = UP ? 2 * BN : BN;
     static constexpr uint32_t kTmemCols = 2u * kAccCols;
-    static constexpr int kStagesRaw = static_cast<int>((kSmemBudget - kGemmFixedSmem) / kStageBytes);
-    static constexpr int kStages = kStagesRaw > kGemmMaxStages ? kGemmMaxStages : kStagesRaw;
+    static constexpr int kStages = ST;
     static constexpr size_t kSmem = kGemmFixedSmem + static_cast<size_t>(kStages) * kStageBytes;
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "tensor memory allocation must be a power of two in [32, 512]");
-    static_assert(kStages >= 2, "pipeline needs two stages");
+    static_assert(kStages >= 2 && kStages <= kGemmMaxStages, "pipeline depth");
     static_assert(kSmem <= kSmemBudget, "shared memory");
+    // One CTA per SM: the shared memory above keeps a second CTA (and its
+    // tensor-memory allocation) off the SM.
+    static_assert(kSmem > kSmemBudget / 2, "one CTA per SM");
 };
 
 struct GemmParams {
@@ -66,15 +71,20 @@ struct GemmParams {
     void *out;               // [S, M_rows]
     uint32_t *err;
     int stream_weights;      // 1: each weight block feeds one tile; hint L2 to evict it first
+    int ksplit;              // K is split into this many ranges (down only; partial outputs)
+    size_t part_stride;      // elements between the partial outputs of consecutive K ranges
 };
 
 struct Unit {
-    int e, mb, r0, valid;
+    int e, mb, r0, valid, ks;
 };
 
+// Work unit u -> (expert, weight block, token tile, K range).  Units of one
+// expert are numbered weight-block-major, then token tile, then K range, so
+// that CTAs running at the same time share a weight block through L2.
 template <int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const int32_t *s_pre, const int32_t *s_off,
-                                            int E, int MB)
+                                            int E, int ksplit)
 {
     int lo = 0, hi = E - 1;
     while (lo < hi) {
@@ -84,7 +94,9 @@ __device__ __forceinline__ Unit decode_unit(int u, const int32_t *s_pre, const i
     }
     Unit w;
     w.e = lo;
-    const int local = u - s_pre[lo];
+    int local = u - s_pre[lo];
+    w.ks = local % ksplit;
+    local /= ksplit;
     const int cnt = s_off[lo + 1] - s_off[lo];
     const int ntb = (cnt + BN - 1) / BN;
     w.mb = local / ntb;
@@ -103,12 +115,12 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
-template <bool UP, int BN>
+template <bool UP, int BN, int ST>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB, const GemmParams p)
 {
-    using C = Cfg<UP, BN>;
+    using C = Cfg<UP, BN, ST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -128,7 +140,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int E = p.offsets ? p.E : 1;
     const int MB = p.M_rows / 128;
     const int KS = p.K / 64;
+    const int KSPLIT = p.ksplit;
 
+    ptx::grid_dep_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -151,6 +165,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::tmem_alloc(tmem_slot, C::kTmemCols);
         ptx::tmem_relinquish();
     }
+    // Everything above overlaps the previous kernel; from here on its results
+    // (offsets, activations) are read and this kernel's outputs are written.
+    ptx::grid_dep_wait();
     if (warp == 2) {
         // Segment table and the unit prefix (units of expert e =
         // ceil(rows_e / BN) token tiles x MB weight blocks).
@@ -167,7 +184,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (e == E - 1) s_off[E] = o1;
                 const int c = o1 - o0;
                 if (o0 < 0 || c < 0 || o1 > p.S) bad = true;
-                else local += ((c + BN - 1) / BN) * MB;
+                else local += ((c + BN - 1) / BN) * MB * KSPLIT;
             }
         }
         bad = __any_sync(0xffffffffu, bad);
@@ -188,7 +205,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 s_pre[e] = run;
                 if (!bad) {
                     const int c = s_off[e + 1] - s_off[e];
-                    run += ((c + BN - 1) / BN) * MB;
+                    run += ((c + BN - 1) / BN) * MB * KSPLIT;
                 }
             }
         }
@@ -210,9 +227,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 p.stream_weights ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             bool stop = false;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
-                const Unit w = decode_unit<BN>(u, s_pre, s_off, E, MB);
+                const Unit w = decode_unit<BN>(u, s_pre, s_off, E, KSPLIT);
                 const int arow = w.e * p.M_rows + w.mb * 128;
-                for (int ks = 0; ks < KS; ++ks) {
+                const int k_end = (w.ks + 1) * KS / KSPLIT;
+                for (int ks = w.ks * KS / KSPLIT; ks < k_end; ++ks) {
                     if (!bounded_wait(&empty[stage], phase ^ 1u, abort_flag, p.err,
                                       kErrTimeoutMma)) {
                         stop = true;
@@ -243,8 +261,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int i = 0;
             bool stop = false;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x, ++i) {
-                const Unit w = decode_unit<BN>(u, s_pre, s_off, E, MB);
+                const Unit w = decode_unit<BN>(u, s_pre, s_off, E, KSPLIT);
                 const int n = ((w.valid + 15) >> 4) << 4;
+                const int k_beg = w.ks * KS / KSPLIT;
+                const int k_end = (w.ks + 1) * KS / KSPLIT;
                 const uint32_t idesc = ptx::idesc_bf16_f32(128, n);
                 const int buf = i & 1;
                 const uint32_t use = static_cast<uint32_t>(i >> 1);
@@ -253,7 +273,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem + static_cast<uint32_t>(buf * C::kAccCols);
-                for (int ks = 0; ks < KS; ++ks) {
+                for (int ks = k_beg; ks < k_end; ++ks) {
                     if (!bounded_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutTma)) {
                         stop = true;
                         break;
@@ -264,7 +284,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
-                        const uint32_t acc = (ks | kk) ? 1u : 0u;
+                        const uint32_t acc = ((ks - k_beg) | kk) ? 1u : 0u;
                         ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc, idesc,
                                          acc);
                         if (UP)
@@ -289,7 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         int i = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x, ++i) {
-            const Unit w = decode_unit<BN>(u, s_pre, s_off, E, MB);
+            const Unit w = decode_unit<BN>(u, s_pre, s_off, E, KSPLIT);
             const int buf = i & 1;
             const uint32_t use = static_cast<uint32_t>(i >> 1);
             if (!bounded_wait_warp(&tfull[buf], use & 1u, abort_flag, p.err, kErrTimeoutMma))
@@ -317,7 +337,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint32_t y[32];
                     ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), y);
                     ptx::tc_wait_ld();
-                    float *Y = static_cast<float *>(p.out);
+                    float *Y = static_cast<float *>(p.out) + w.ks * p.part_stride;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (c0 + j < w.valid)
@@ -338,10 +358,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 }
 
-template <bool UP, int BN>
-cudaError_t launch_gemm_bn(const GemmLaunch &a, cudaStream_t s)
+template <bool UP, int BN, int ST>
+cudaError_t launch_gemm_cfg(const GemmLaunch &a, cudaStream_t s)
 {
-    using C = Cfg<UP, BN>;
+    using C = Cfg<UP, BN, ST>;
     CUtensorMap tA0, tA1, tB;
     cudaError_t e = make_tmap_bf16(&tA0, a.A0, static_cast<uint64_t>(a.E) * a.M_rows, a.K, 128);
     if (e != cudaSuccess) return e;
@@ -349,7 +369,7 @@ cudaError_t launch_gemm_bn(const GemmLaunch &a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16(&tB, a.B, a.S, a.K, BN);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemm_kernel<UP, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemm_kernel<UP, BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return e;
 
@@ -362,30 +382,72 @@ cudaError_t launch_gemm_bn(const GemmLaunch &a, cudaStream_t s)
     p.out = a.out;
     p.err = a.err;
     p.stream_weights = a.max_rows <= BN ? 1 : 0;
+    p.ksplit = UP ? 1 : (a.ksplit < 1 ? 1 : a.ksplit);
+    p.part_stride = static_cast<size_t>(a.S) * a.M_rows;
     // Upper bound of the work units: every segment rounds up to whole tiles.
     const long long tiles = (static_cast<long long>(a.S) + BN - 1) / BN + p.E;
-    const long long units = tiles * (a.M_rows / 128);
+    const long long units = tiles * (a.M_rows / 128) * p.ksplit;
     long long grid = device_sm_count();
     if (units < grid) grid = units;
     if (grid < 1) grid = 1;
-    gemm_kernel<UP, BN><<<static_cast<int>(grid), kGemmThreads, C::kSmem, s>>>(tA0, tA1, tB, p);
-    return cudaGetLastError();
+    return launch_pdl(gemm_kernel<UP, BN, ST>, dim3(static_cast<unsigned>(grid)),
+                      dim3(kGemmThreads), C::kSmem, s, a.pdl, tA0, tA1, tB, p);
 }
 
 }  // namespace
 
+int gemm_token_tile(int up, int S, int E_seg)
+{
+    // Token tile from the average rows per segment: small tiles waste no
+    // MMA columns and leave room for a deeper weight pipeline.
+    const long long avg = (static_cast<long long>(S) + E_seg - 1) / E_seg;
+    if (avg <= 32) return 32;
+    if (avg <= 64) return 64;
+    if (up || avg <= 128) return 128;
+    return 256;
+}
+
+int down_ksplit(int S, int E_seg, int d, int d_ff)
+{
+    // Split K of the down projection when its (segment x weight block) units
+    // cannot fill the GPU: pick the split whose unit count fills whole waves
+    // of the SMs best, keeping at least 8 K steps per range.
+    const int bn = gemm_token_tile(0, S, E_seg);
+    const long long hit = std::min<long long>(E_seg, S);
+    const long long units = (d / 128) * std::max<long long>(hit, (S + bn - 1) / bn);
+    const long long sms = 148;
+    if (units >= 2 * sms) return 1;
+    const int max_ks = std::max(1, std::min(8, d_ff / 64 / 8));  // 8: the combine sums at most 8 partials
+    int best = 1;
+    double best_eff = 0.0;
+    for (int ks = 1; ks <= max_ks; ++ks) {
+        const long long u = units * ks;
+        const long long waves = (u + sms - 1) / sms;
+        const double eff = static_cast<double>(u) / static_cast<double>(waves * sms);
+        if (eff > best_eff + 0.02) {
+            best = ks;
+            best_eff = eff;
+        }
+    }
+    return best;
+}
+
 cudaError_t launch_gemm(const GemmLaunch &a, cudaStream_t s)
 {
-    const int r = a.max_rows;
+    const int bn = gemm_token_tile(a.up, a.S, a.offsets ? a.E : 1);
     if (a.up) {
-        if (r <= 32) return launch_gemm_bn<true, 32>(a, s);
-        if (r <= 64) return launch_gemm_bn<true, 64>(a, s);
-        return launch_gemm_bn<true, 128>(a, s);
+        switch (bn) {
+        case 32: return launch_gemm_cfg<true, 32, 5>(a, s);
+        case 64: return launch_gemm_cfg<true, 64, 5>(a, s);
+        default: return launch_gemm_cfg<true, 128, 4>(a, s);
+        }
     }
-    if (r <= 32) return launch_gemm_bn<false, 32>(a, s);
-    if (r <= 64) return launch_gemm_bn<false, 64>(a, s);
-    if (r <= 128) return launch_gemm_bn<false, 128>(a, s);
-    return launch_gemm_bn<false, 256>(a, s);
+    switch (bn) {
+    case 32: return launch_gemm_cfg<false, 32, 10>(a, s);
+    case 64: return launch_gemm_cfg<false, 64, 8>(a, s);
+    case 128: return launch_gemm_cfg<false, 128, 6>(a, s);
+    default: return launch_gemm_cfg<false, 256, 4>(a, s);
+    }
 }
 
 }  // namespace moe

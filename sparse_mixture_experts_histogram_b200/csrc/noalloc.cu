@@ -98,7 +98,10 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
     g.B = x_perm;
     g.out = H;
     g.err = err;
+    g.ksplit = 1;
+    g.pdl = false;
     if (launch_gemm(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+    g.pdl = true;
     g.up = 0;
     g.M_rows = d;
     g.K = d_ff;

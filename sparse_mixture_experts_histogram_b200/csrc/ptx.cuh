@@ -213,6 +213,15 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N)
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue now, and wait until the previous kernel's results are visible.
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(int id, int count)
 {

@@ -14,8 +14,11 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -103,6 +106,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     const int tile = blockIdx.x;
     const int ksteps = p.d / 64;
 
+    ptx::grid_dep_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -234,6 +238,244 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Router on the CUDA cores, for batches whose T*E*d is small (decode sizes,
+// narrow layers): a tensor-core tile of 128 tokens would leave most SMs idle
+// and wait on a long serial chain of copies.  One CTA takes kSmallTok tokens:
+// their x rows go to shared memory, warp w computes the logits of experts
+// e = w, w+8, ... for all of them (16-byte loads of Wg, fp32 FMA, warp
+// reduction), then warp i selects token i's top-k by K rounds of a warp-wide
+// (largest value, lowest index) reduction and applies the softmax.  The last
+// CTA of every 128-token tile runs the same tile histogram / stable ranks /
+// offsets step as the tensor-core router.
+constexpr int kSmallTok = 4;
+constexpr int kSmallThreads = 256;
+
+struct SmallRouteParams {
+    int T, d, E;
+    const uint4 *x;
+    const uint4 *Wg;
+    const float *bias;
+    int32_t *idx;
+    float *w;
+    uint32_t *tile_ctr;
+    DispatchOut dout;
+};
+
+// 8 bf16 (one 16-byte vector) to fp32, in element order.
+__device__ __forceinline__ void unpack8(const uint4 &a, float (&f)[8])
+{
+    const uint32_t v[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(v[i] << 16);
+        f[2 * i + 1] = __uint_as_float(v[i] & 0xffff0000u);
+    }
+}
+
+size_t small_route_smem(int d)
+{
+    return static_cast<size_t>(kSmallTok) * d * 2 + kSmallTok * kMaxE * sizeof(float) +
+           sizeof(DispatchSmem);
+}
+
+template <int K, int EPW, int U>
+__global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallRouteParams p)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ uint32_t s_last;
+    const int nv = p.d >> 3;
+    uint4 *sx = reinterpret_cast<uint4 *>(smem_raw);
+    float *slog = reinterpret_cast<float *>(smem_raw + static_cast<size_t>(kSmallTok) * p.d * 2);
+    DispatchSmem &ds = *reinterpret_cast<DispatchSmem *>(slog + kSmallTok * kMaxE);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kSmallTok;
+    const int nt = min(kSmallTok, p.T - t0);
+
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    for (int i = threadIdx.x; i < kSmallTok * nv; i += kSmallThreads) {
+        const int tt = i / nv;
+        sx[i] = (tt < nt) ? __ldg(p.x + static_cast<size_t>(t0) * nv + i) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+
+    // Warp w computes experts w*EPW .. w*EPW+EPW-1, then the next 8*EPW
+    // experts; each lane keeps U*EPW 16-byte loads of Wg in flight.
+    for (int e0 = warp * EPW; e0 < p.E; e0 += (kSmallThreads / 32) * EPW) {
+        float acc[EPW][kSmallTok];
+#pragma unroll
+        for (int q = 0; q < EPW; ++q)
+#pragma unroll
+            for (int tt = 0; tt < kSmallTok; ++tt) acc[q][tt] = 0.0f;
+        for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+            uint4 wv[U][EPW];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + 32 * u;
+#pragma unroll
+                for (int q = 0; q < EPW; ++q)
+                    wv[u][q] = (v < nv && e0 + q < p.E)
+                                   ? __ldg(p.Wg + static_cast<size_t>(e0 + q) * nv + v)
+                                   : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + 32 * u;
+                if (v < nv) {
+                    float wf[EPW][8];
+#pragma unroll
+                    for (int q = 0; q < EPW; ++q) unpack8(wv[u][q], wf[q]);
+#pragma unroll
+                    for (int tt = 0; tt < kSmallTok; ++tt) {
+                        float xf[8];
+                        unpack8(sx[tt * nv + v], xf);
+#pragma unroll
+                        for (int q = 0; q < EPW; ++q)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[q][tt] = fmaf(wf[q][i], xf[i], acc[q][tt]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < EPW; ++q) {
+#pragma unroll
+            for (int tt = 0; tt < kSmallTok; ++tt) {
+                float a = acc[q][tt];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+                acc[q][tt] = a;
+            }
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int q = 0; q < EPW; ++q) {
+                const int e = e0 + q;
+                if (e < p.E) {
+                    const float b = p.bias ? p.bias[e] : 0.0f;
+#pragma unroll
+                    for (int tt = 0; tt < kSmallTok; ++tt) slog[tt * kMaxE + e] = acc[q][tt] + b;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    if (warp < nt) {
+        const int t = t0 + warp;
+        float v[kMaxE / 32];
+#pragma unroll
+        for (int i = 0; i < kMaxE / 32; ++i) {
+            const int e = lane + 32 * i;
+            v[i] = (e < p.E) ? slog[warp * kMaxE + e] : -CUDART_INF_F;
+        }
+        float tv[K];
+        int ti[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            float bv = -CUDART_INF_F;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < kMaxE / 32; ++i) {
+                const int e = lane + 32 * i;
+                if (e < p.E && v[i] > bv) {  // strict: equal values keep the lower index
+                    bv = v[i];
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (ov > bv || (ov == bv && oe < be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            tv[j] = bv;
+            ti[j] = be;
+#pragma unroll
+            for (int i = 0; i < kMaxE / 32; ++i)
+                if (lane + 32 * i == be) v[i] = -CUDART_INF_F;
+        }
+        if (lane == 0) {
+            float ex[K];
+            float s = 0.0f;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                ex[j] = expf(tv[j] - tv[0]);
+                s += ex[j];
+            }
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                p.idx[static_cast<size_t>(t) * K + j] = ti[j];
+                p.w[static_cast<size_t>(t) * K + j] = ex[j] / s;
+            }
+        }
+    }
+
+    // The last CTA of each 128-token tile groups that tile's pairs by expert.
+    __threadfence();
+    __syncthreads();
+    const int tile = t0 / kTileTokens;
+    if (threadIdx.x == 0) {
+        const int tile_tokens = min(kTileTokens, p.T - tile * kTileTokens);
+        const uint32_t nblk = static_cast<uint32_t>((tile_tokens + kSmallTok - 1) / kSmallTok);
+        s_last = (atomicAdd(&p.tile_ctr[tile], 1u) == nblk - 1u) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (!s_last || threadIdx.x >= kTileTokens) return;
+    __threadfence();
+    const int row = threadIdx.x;
+    const int t = tile * kTileTokens + row;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        ds.sel[row][j] = (t < p.T) ? __ldcg(&p.idx[static_cast<size_t>(t) * K + j]) : -1;
+    dispatch_tile(ds, row, tile, p.T, p.E, K, p.dout, 1);
+}
+
+template <int K, int EPW, int U>
+cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
+{
+    const size_t smem = small_route_smem(a.d);
+    cudaError_t e = cudaFuncSetAttribute(route_small_kernel<K, EPW, U>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    SmallRouteParams p;
+    p.T = a.T;
+    p.d = a.d;
+    p.E = a.E;
+    p.x = reinterpret_cast<const uint4 *>(a.x);
+    p.Wg = reinterpret_cast<const uint4 *>(a.Wg);
+    p.bias = a.bias;
+    p.idx = a.idx;
+    p.w = a.w;
+    p.tile_ctr = a.tile_ctr;
+    p.dout.tilecnt = a.tilecnt;
+    p.dout.tilebase = a.tilebase;
+    p.dout.rank = a.rank;
+    p.dout.offsets = a.offsets;
+    p.dout.counts = a.counts;
+    p.dout.done = a.done;
+    p.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
+    const int blocks = (a.T + kSmallTok - 1) / kSmallTok;
+    route_small_kernel<K, EPW, U><<<blocks, kSmallThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// Few experts: one expert per warp and eight loads in flight per lane; many
+// experts: four experts per warp and four loads each.
+template <int K>
+cudaError_t launch_route_small_k(const RouteLaunch &a, cudaStream_t s)
+{
+    if (a.E <= 16) return launch_route_small_cfg<K, 1, 8>(a, s);
+    return launch_route_small_cfg<K, 4, 4>(a, s);
+}
+
 template <int K>
 cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
 {
@@ -280,8 +522,31 @@ cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
 
 }  // namespace
 
+// Tensor cores pay off once the router is a real GEMM; below this many
+// multiply-adds the CUDA-core router is faster (it spreads over more SMs and
+// has a short dependency chain).
+constexpr long long kSmallRouterMacs = 1LL << 30;
+
+bool use_small_router(const RouteLaunch &a)
+{
+    return static_cast<long long>(a.T) * a.E * a.d <= kSmallRouterMacs;
+}
+
 cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s)
 {
+    if (use_small_router(a)) {
+        switch (a.k) {
+        case 1: return launch_route_small_k<1>(a, s);
+        case 2: return launch_route_small_k<2>(a, s);
+        case 3: return launch_route_small_k<3>(a, s);
+        case 4: return launch_route_small_k<4>(a, s);
+        case 5: return launch_route_small_k<5>(a, s);
+        case 6: return launch_route_small_k<6>(a, s);
+        case 7: return launch_route_small_k<7>(a, s);
+        case 8: return launch_route_small_k<8>(a, s);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     switch (a.k) {
     case 1: return launch_route_k<1>(a, s);
     case 2: return launch_route_k<2>(a, s);

@@ -128,6 +128,27 @@ def test_permute_flags_out_of_range_expert():
     assert row.cpu().numpy()[5, 1] == -1
 
 
+def test_permute_flags_repeated_expert_and_keeps_a_bijection():
+    wl = Workload("dup_idx", 40, 128, 8, 128, 3)
+    inp = _inputs(wl)
+    g = np.random.default_rng(9)
+    idx = np.stack([g.choice(8, size=3, replace=False) for _ in range(40)]).astype(np.int32)
+    idx[7, 2] = idx[7, 0]  # token 7 names one expert twice
+    offsets = torch.empty(9, dtype=torch.int32, device=DEV)
+    row = torch.empty(40, 3, dtype=torch.int32, device=DEV)
+    xp = torch.zeros(120, 128, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(wl)
+    moe.moe_permute(40, 128, 8, 3, inp["x"], torch.as_tensor(idx, device=DEV), offsets, row, xp,
+                    ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 5 and code & 0x10
+    r = row.cpu().numpy()
+    assert r[7, 2] == -1
+    valid = r[r >= 0]
+    assert len(np.unique(valid)) == len(valid) == 119     # no two pairs share a row
+    assert offsets.cpu().numpy()[-1] == 119
+
+
 # ------------------------------------------------------------------ experts
 FFN_SEGMENTS = [
     ("ragged", 512, 384, [0, 1, 15, 16, 17, 127, 128, 129, 300, 0, 33]),
