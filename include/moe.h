@@ -191,16 +191,15 @@ MOE_API moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff, const mo
                                          moe_stream_t stream);
 
 /* Number of events moe_forward_traced records. */
-#define MOE_TRACE_EVENTS 8
+#define MOE_TRACE_EVENTS 6
 
 /* moe_forward_ex that also records caller-created CUDA events (cudaEvent_t,
  * created with timing enabled) on `stream` at the kernel boundaries, so the
  * caller can time each kernel with cudaEventElapsedTime:
- *   events[0] before the router kernel      events[4] before the shared up GEMM
- *   events[1] before the dispatch scatter   events[5] before the shared down GEMM
- *   events[2] before the up GEMM (W1|W3)    events[6] before the combine
- *   events[3] before the down GEMM (W2)     events[7] after the combine
- * (events[4..5] mark the same point as events[6] when there is no shared
+ *   events[0] before the router kernel      events[3] before the shared-expert FFN
+ *   events[1] before the dispatch scatter   events[4] before the combine
+ *   events[2] before the expert FFN kernel  events[5] after the combine
+ * (events[3] and events[4] mark the same point when there is no shared
  * expert).  n_events must be MOE_TRACE_EVENTS.  While `stream` is being
  * captured into a CUDA graph the events are recorded as graph event nodes.
  * The layer's work and results are those of moe_forward_ex. */

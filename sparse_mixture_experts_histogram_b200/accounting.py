@@ -63,30 +63,16 @@ def algorithmic_bytes(T: int, d: int, E: int, d_ff: int, k: int, experts_hit: in
             + 2 * expert_params(d, d_ff_shared))
 
 
-def gemm_bytes(kind: str, T: int, d: int, d_ff: int, k: int, experts_hit: int,
-               d_ff_shared: int = 0) -> int:
-    """Algorithmic bytes of one grouped-GEMM launch.
-
-    kind "up":   bf16 W1 and W3 of the hit experts + the permuted bf16 rows
-                 read (S = T*k rows of d) + bf16 H written (S rows of d_ff).
-    kind "down": bf16 W2 of the hit experts + bf16 H read + fp32 Y written
-                 (S rows of d).
-    A shared expert adds one more segment of T rows with its own weights.
-    """
+def ffn_bytes(T: int, d: int, d_ff: int, k: int, experts_hit: int, d_ff_shared: int = 0) -> int:
+    """Algorithmic bytes of the expert feed-forward kernel (both projections):
+    bf16 W1, W3, W2 of the hit experts + the permuted bf16 rows read (S = T*k
+    rows of d) + the fp32 expert outputs written (S rows of d).  The hidden
+    activations H are an intermediate and are not counted.  A shared expert
+    is its own launch over the T token rows with its own weights."""
     S = T * k
-    if kind == "up":
-        return (2 * 2 * experts_hit * d * d_ff + 2 * S * d + 2 * S * d_ff
-                + (2 * 2 * d * d_ff_shared + 2 * T * d + 2 * T * d_ff_shared if d_ff_shared else 0))
-    if kind == "down":
-        return (2 * experts_hit * d * d_ff + 2 * S * d_ff + 4 * S * d
-                + (2 * d * d_ff_shared + 2 * T * d_ff_shared + 4 * T * d if d_ff_shared else 0))
-    raise ValueError(kind)
+    return 2 * 3 * experts_hit * d * d_ff + 2 * S * d + 4 * S * d
 
 
-def gemm_flops(kind: str, T: int, d: int, d_ff: int, k: int, d_ff_shared: int = 0) -> int:
-    S = T * k
-    if kind == "up":
-        return 2 * 2 * S * d * d_ff + 2 * 2 * T * d * d_ff_shared
-    if kind == "down":
-        return 2 * S * d * d_ff + 2 * T * d * d_ff_shared
-    raise ValueError(kind)
+def ffn_flops(T: int, d: int, d_ff: int, k: int) -> int:
+    """FLOPs of the expert feed-forward kernel: 2*3*d*d_ff per routed row."""
+    return 2 * 3 * T * k * d * d_ff

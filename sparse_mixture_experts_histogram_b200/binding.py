@@ -28,10 +28,9 @@ ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "mo
                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_ex",
                  "moe_forward_traced", "moe_get_device_error", "moe_status_string",
                  "moe_expert_ffn_static")
-TRACE_EVENTS = 8
+TRACE_EVENTS = 6
 #: What each of moe_forward_traced's events marks (event i = start of stage i).
-TRACE_STAGES = ("route", "scatter", "up_gemm", "down_gemm", "shared_up_gemm",
-                "shared_down_gemm", "combine")
+TRACE_STAGES = ("route", "scatter", "expert_ffn", "shared_ffn", "combine")
 
 
 class MoEError(RuntimeError):

@@ -23,7 +23,8 @@ constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, rank
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-    size_t tilectr, zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
+    size_t tilectr, hready, hready_s;
+    size_t zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
     size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, xperm, H, Y, Hs, Ys, total;
 };
 
@@ -40,6 +41,8 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     const size_t ntiles = (static_cast<size_t>(T) + 127) / 128;
     const size_t S = static_cast<size_t>(T) * k;
     L.tilectr = take(ntiles * 4);
+    L.hready = take(ffn_ready_counters(static_cast<int>(S), E) * 4);
+    L.hready_s = d_ffs > 0 ? take(ffn_ready_counters(T, 1) * 4) : 0;
     L.zero_bytes = o;
     L.tilecnt = take(ntiles * E * 4);
     L.tilebase = take(ntiles * E * 4);
@@ -248,42 +251,29 @@ moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int3
 
 static moe_status mark(void *const *events, int i, cudaStream_t s);
 
-static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const moe_bf16 *x_perm,
+static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const moe_bf16 *x,
                            const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
-                           const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *err,
-                           cudaStream_t s, bool pdl_first, int ksplit,
-                           void *const *events = nullptr, int ev0 = 0)
+                           const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *h_ready,
+                           uint32_t *err, cudaStream_t s, bool pdl, int ksplit)
 {
-    GemmLaunch g;
-    g.up = 1;
-    g.E = E;
-    g.M_rows = d_ff;
-    g.K = d;
-    g.S = S;
-    g.max_rows = max_rows;
-    g.offsets = offsets;
-    g.A0 = W1;
-    g.A1 = W3;
-    g.B = x_perm;
-    g.out = H;
-    g.err = err;
-    g.ksplit = 1;
-    g.pdl = pdl_first && events == nullptr;
-    moe_status st = mark(events, ev0, s);
-    if (st != MOE_OK) return st;
-    st = from_cuda(launch_gemm(g, s));
-    if (st != MOE_OK) return st;
-    if ((st = mark(events, ev0 + 1, s)) != MOE_OK) return st;
-    g.pdl = events == nullptr;
-    g.ksplit = ksplit;
-    g.up = 0;
-    g.M_rows = d;
-    g.K = d_ff;
-    g.A0 = W2;
-    g.A1 = nullptr;
-    g.B = H;
-    g.out = y;
-    return from_cuda(launch_gemm(g, s));
+    FfnLaunch f;
+    f.E = E;
+    f.d = d;
+    f.d_ff = d_ff;
+    f.S = S;
+    f.max_rows = max_rows;
+    f.ksplit = ksplit;
+    f.offsets = offsets;
+    f.W1 = W1;
+    f.W3 = W3;
+    f.W2 = W2;
+    f.x = x;
+    f.H = H;
+    f.Y = y;
+    f.h_ready = h_ready;
+    f.err = err;
+    f.pdl = pdl;
+    return from_cuda(launch_ffn(f, s));
 }
 
 moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
@@ -296,14 +286,16 @@ moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
     if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
         !ok_ptr(y_perm) || !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
-    const size_t need = kHeaderBytes + align_up(static_cast<size_t>(S) * d_ff * 2);
+    const size_t ctr = align_up(ffn_ready_counters(S, E) * 4);
+    const size_t need = kHeaderBytes + ctr + align_up(static_cast<size_t>(S) * d_ff * 2);
     if (ws_bytes < need) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
-    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes + ctr, s));
     if (st != MOE_OK) return st;
     return ffn_impl(S, d, E, d_ff, S, x_perm, offsets, W1, W3, W2,
-                    reinterpret_cast<moe_bf16 *>(wsb + kHeaderBytes), y_perm,
+                    reinterpret_cast<moe_bf16 *>(wsb + kHeaderBytes + ctr), y_perm,
+                    reinterpret_cast<uint32_t *>(wsb + kHeaderBytes),
                     reinterpret_cast<uint32_t *>(wsb), s, false, 1);
 }
 
@@ -399,23 +391,24 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
 
     // A token never picks one expert twice, so no segment exceeds T rows.
     const int ksplit = down_ksplit(S, E, d, d_ff);
-    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y, err, s, true, ksplit,
-                  events, 2);
+    if ((st = mark(events, 2, s)) != MOE_OK) return st;
+    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
+                  reinterpret_cast<uint32_t *>(wsb + L.hready), err, s, events == nullptr,
+                  ksplit);
     if (st != MOE_OK) return st;
 
     const float *shared_y = nullptr;
+    if ((st = mark(events, 3, s)) != MOE_OK) return st;
     if (d_ff_shared > 0) {
         moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
         float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
-        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys, err, s, true, 1,
-                      events, 4);
+        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys,
+                      reinterpret_cast<uint32_t *>(wsb + L.hready_s), err, s, events == nullptr,
+                      1);
         if (st != MOE_OK) return st;
         shared_y = Ys;
-    } else {
-        if ((st = mark(events, 4, s)) != MOE_OK) return st;
-        if ((st = mark(events, 5, s)) != MOE_OK) return st;
     }
-    if ((st = mark(events, 6, s)) != MOE_OK) return st;
+    if ((st = mark(events, 4, s)) != MOE_OK) return st;
 
     CombineLaunch cb;
     cb.T = T;
@@ -430,7 +423,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     cb.pdl = events == nullptr;
     st = from_cuda(launch_combine(cb, s));
     if (st != MOE_OK) return st;
-    return mark(events, 7, s);
+    return mark(events, 5, s);
 }
 
 moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,

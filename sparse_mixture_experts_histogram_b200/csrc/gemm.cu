@@ -1,22 +1,28 @@
-// gemm.cu -- grouped expert GEMMs on the 5th-generation tensor cores.
+// gemm.cu -- the experts' feed-forward as one persistent kernel on the
+// 5th-generation tensor cores (tcgen05 MMA, accumulators in tensor memory,
+// operands brought in by TMA).
 //
-// For every expert segment e (rows offsets[e] .. offsets[e+1]-1 of the
-// activation matrix B) and every 128-row block of that expert's weights A:
-//   up:   D1 = W1_e[blk] B^T, D3 = W3_e[blk] B^T  (two accumulators),
-//         H[r, blk] = bf16( silu(D1) * D3 )        -- SwiGLU in the epilogue
-//   down: Y[r, blk] = W2_e[blk] H^T                 -- fp32 out
-// The weights are the MMA's A operand (M = 128 weight rows) and the tokens
-// its B operand (N = the segment's rows, rounded up to 16), so a ragged or
-// tiny segment costs only the columns it needs, and decode-sized batches
-// stream each hit expert's weights once.
+// For every expert segment e (rows offsets[e] .. offsets[e+1]-1 of x_perm):
+//   up units:   D0 = W1_e[blk] X^T, D1 = W3_e[blk] X^T   (128 weight rows)
+//               H[r, blk] = bf16( silu(D0) * D1 )         -- SwiGLU epilogue
+//   down units: D0 = W2_e[2m] H^T, D1 = W2_e[2m+1] H^T   (two 128-row blocks)
+//               Y[ks][r, 2m], Y[ks][r, 2m+1] = D0, D1      -- fp32, K range ks
+// The weights are the MMA's A operand (M = 128 weight rows) and the segment's
+// rows its B operand (N = rows, rounded up to 16), so a ragged or tiny
+// segment costs only the columns it needs and small batches stream each hit
+// expert's weights once.  Both kinds of unit load two 128-row weight tiles and
+// one token tile per 64-wide K step, so they share one pipeline.
 //
-// Persistent kernel, one CTA per SM: warp 0 issues TMA copies into a ring of
-// shared-memory stages, warp 1 issues tcgen05 MMAs into a double-buffered
-// tensor-memory accumulator, warps 2..5 drain finished accumulators
-// (tcgen05.ld), apply the epilogue and store; the next tile's MMAs overlap
-// the previous tile's epilogue.  Work units (expert, weight block, token
-// tile) are numbered from the device-side offsets, with consecutive units
-// sharing one weight block so that concurrent CTAs re-read it from L2.
+// One CTA per SM.  Warp 0 issues TMA copies into a ring of shared-memory
+// stages, warp 1 issues the MMAs into a double-buffered tensor-memory
+// accumulator, warps 2..5 drain finished accumulators and store.  Every CTA
+// walks the units numbered up-first (expert, block, token tile) and then
+// down (expert, block pair, token tile, K range).  A down unit needs all of
+// its token tile's H columns: the up epilogues count finished blocks per
+// tile, and the producer waits (bounded) for the count before it copies that
+// H tile.  Since each CTA finishes its up units before its down units, and
+// an up unit never waits, the wait always ends; the down weights stream while
+// the last up units finish.
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward; "Mixtral and MoE
@@ -37,73 +43,83 @@ namespace moe {
 
 namespace {
 
-constexpr int kGemmThreads = 192;
-constexpr int kGemmMaxStages = 12;
-constexpr uint32_t kWTileBytes = 128 * 128;  // 128 weight rows x 64 bf16
-constexpr size_t kGemmFixedSmem = 1024 /* alignment slack */ + (2 * kGemmMaxStages + 5) * 8 + 16 +
-                                  2 * (kMaxE + 1) * sizeof(int32_t) + 64;
+constexpr int kFfnThreads = 192;
+constexpr int kMaxStages = 8;
+constexpr uint32_t kWTile = 128 * 128;  // 128 weight rows x 64 bf16 = 16 KB
+constexpr size_t kFixedSmem = 1024 /* alignment slack */ + (2 * kMaxStages + 5) * 8 + 16 +
+                              4 * (kMaxE + 1) * sizeof(int32_t) + 64;
 constexpr size_t kSmemBudget = 227 * 1024;
 
-template <bool UP, int BN, int ST>
-struct Cfg {
-    static constexpr int kA = UP ? 2 : 1;
-    static constexpr uint32_t kBBytes = BN * 128u;
-    static constexpr uint32_t kStageBytes = kA * kWTileBytes + kBBytes;
-    static constexpr int kAccCols = UP ? 2 * BN : BN;
+template <int BN, int ST>
+struct FfnCfg {
+    static constexpr uint32_t kStageBytes = 2 * kWTile + BN * 128u;
+    static constexpr int kAccCols = 2 * BN;  // accumulators D0 and D1 side by side
     static constexpr uint32_t kTmemCols = 2u * kAccCols;
-    static constexpr int kStages = ST;
-    static constexpr size_t kSmem = kGemmFixedSmem + static_cast<size_t>(kStages) * kStageBytes;
+    static constexpr size_t kSmem = kFixedSmem + static_cast<size_t>(ST) * kStageBytes;
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "tensor memory allocation must be a power of two in [32, 512]");
-    static_assert(kStages >= 2 && kStages <= kGemmMaxStages, "pipeline depth");
+    static_assert(ST >= 2 && ST <= kMaxStages, "pipeline depth");
     static_assert(kSmem <= kSmemBudget, "shared memory");
-    // One CTA per SM: the shared memory above keeps a second CTA (and its
-    // tensor-memory allocation) off the SM.
+    // One CTA per SM: the shared memory keeps a second CTA (and its tensor
+    // memory allocation) off the SM.
     static_assert(kSmem > kSmemBudget / 2, "one CTA per SM");
 };
 
-struct GemmParams {
-    int E;          // segments
-    int M_rows;     // weight rows per expert
-    int K;          // reduction length (multiple of 64)
-    int S;          // rows of B
-    const int32_t *offsets;  // [E+1] or nullptr (one segment [0, S))
-    void *out;               // [S, M_rows]
+struct FfnParams {
+    int E;                  // segments
+    int d, d_ff;
+    int S;                  // rows of x_perm / H / Y
+    int ksplit;             // K ranges of the down projection
+    size_t part_stride;     // floats between the partial outputs of consecutive K ranges
+    const int32_t *offsets; // [E+1] or nullptr (one segment [0, S))
+    __nv_bfloat16 *H;       // [S, d_ff]
+    float *Y;               // [ksplit, S, d]
+    uint32_t *h_ready;      // [tiles] finished (up block x epilogue warp) count per token tile
     uint32_t *err;
-    int stream_weights;      // 1: each weight block feeds one tile; hint L2 to evict it first
-    int ksplit;              // K is split into this many ranges (down only; partial outputs)
-    size_t part_stride;      // elements between the partial outputs of consecutive K ranges
+    int stream_weights;     // each weight block feeds one token tile: L2 evict-first
 };
 
 struct Unit {
-    int e, mb, r0, valid, ks;
+    bool up;
+    int e, blk, r0, valid, tile, k_beg, k_end, ks;
 };
 
-// Work unit u -> (expert, weight block, token tile, K range).  Units of one
-// expert are numbered weight-block-major, then token tile, then K range, so
-// that CTAs running at the same time share a weight block through L2.
 template <int BN>
-__device__ __forceinline__ Unit decode_unit(int u, const int32_t *s_pre, const int32_t *s_off,
-                                            int E, int ksplit)
+__device__ __forceinline__ Unit decode_unit(int u, int u_up, const int32_t *s_off,
+                                            const int32_t *s_pu, const int32_t *s_pd,
+                                            const int32_t *s_tb, int E, int ksplit, int ksu,
+                                            int ksd)
 {
+    Unit w;
+    w.up = u < u_up;
+    const int32_t *pre = w.up ? s_pu : s_pd;
+    const int x = w.up ? u : u - u_up;
     int lo = 0, hi = E - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (s_pre[mid] <= u) lo = mid;
+        if (pre[mid] <= x) lo = mid;
         else hi = mid - 1;
     }
-    Unit w;
     w.e = lo;
-    int local = u - s_pre[lo];
-    w.ks = local % ksplit;
-    local /= ksplit;
+    int local = x - pre[lo];
     const int cnt = s_off[lo + 1] - s_off[lo];
     const int ntb = (cnt + BN - 1) / BN;
-    w.mb = local / ntb;
-    const int tb = local - w.mb * ntb;
+    if (w.up) {
+        w.ks = 0;
+        w.k_beg = 0;
+        w.k_end = ksu;
+    } else {
+        w.ks = local % ksplit;
+        local /= ksplit;
+        w.k_beg = w.ks * ksd / ksplit;
+        w.k_end = (w.ks + 1) * ksd / ksplit;
+    }
+    w.blk = local / ntb;
+    const int tb = local - w.blk * ntb;
     w.r0 = s_off[lo] + tb * BN;
     const int rem = cnt - tb * BN;
     w.valid = rem < BN ? rem : BN;
+    w.tile = s_tb[lo] + tb;
     return w;
 }
 
@@ -115,66 +131,115 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
-template <bool UP, int BN, int ST>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                const __grid_constant__ CUtensorMap tmB, const GemmParams p)
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p)
 {
-    using C = Cfg<UP, BN, ST>;
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Waits until *ctr >= target (written by other CTAs' epilogues).  Bounded
+// like the pipeline waits: gives up after kWaitTimeoutNs or when another role
+// of this CTA has given up.
+__device__ __forceinline__ bool wait_counter(const uint32_t *ctr, uint32_t target,
+                                             volatile uint32_t *abort_flag, uint32_t *gerr)
+{
+    if (ld_acquire(ctr) >= target) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (ld_acquire(ctr) >= target) return true;
+        if (*abort_flag) return false;
+        if ((it & 15u) == 0 && ptx::globaltimer() - t0 > kWaitTimeoutNs) {
+            *abort_flag = 1u;
+            if (gerr) atomicOr(gerr, kErrTimeoutEpi);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane)
+{
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+    }
+    return v;
+}
+
+template <int BN, int ST>
+__global__ void __launch_bounds__(kFfnThreads, 1)
+    ffn_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW3,
+               const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmX,
+               const __grid_constant__ CUtensorMap tmH, const FfnParams p)
+{
+    using C = FfnCfg<BN, ST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
-    uint64_t *empty = full + kGemmMaxStages;
-    uint64_t *tfull = empty + kGemmMaxStages;   // [2]
-    uint64_t *tempty = tfull + 2;               // [2]
-    uint64_t *drain = tempty + 2;               // [1]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ST * C::kStageBytes);
+    uint64_t *empty = full + kMaxStages;
+    uint64_t *tfull = empty + kMaxStages;  // [2]
+    uint64_t *tempty = tfull + 2;          // [2]
+    uint64_t *drain = tempty + 2;          // [1]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     int32_t *s_off = reinterpret_cast<int32_t *>(tmem_slot + 4);
-    int32_t *s_pre = s_off + (kMaxE + 1);
+    int32_t *s_pu = s_off + (kMaxE + 1);   // up-unit prefix per expert
+    int32_t *s_pd = s_pu + (kMaxE + 1);    // down-unit prefix per expert
+    int32_t *s_tb = s_pd + (kMaxE + 1);    // token-tile prefix per expert
 
     const int E = p.offsets ? p.E : 1;
-    const int MB = p.M_rows / 128;
-    const int KS = p.K / 64;
+    const int MBU = p.d_ff / 128;          // up weight blocks per expert
+    const int MBD = (p.d + 255) / 256;     // down weight block pairs per expert
+    const int KSU = p.d / 64;
+    const int KSD = p.d_ff / 64;
     const int KSPLIT = p.ksplit;
+    const uint32_t ready_target = 4u * static_cast<uint32_t>(MBU);
 
     ptx::grid_dep_launch();
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < ST; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&tfull[b], 1);
-            ptx::mbar_init(&tempty[b], 4);   // one arrival per epilogue warp
+            ptx::mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
         ptx::fence_barrier_init();
     }
     if (threadIdx.x == 32) {
-        ptx::prefetch_tensormap(&tmA0);
-        if (UP) ptx::prefetch_tensormap(&tmA1);
-        ptx::prefetch_tensormap(&tmB);
+        ptx::prefetch_tensormap(&tmW1);
+        ptx::prefetch_tensormap(&tmW3);
+        ptx::prefetch_tensormap(&tmW2);
+        ptx::prefetch_tensormap(&tmX);
+        ptx::prefetch_tensormap(&tmH);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, C::kTmemCols);
         ptx::tmem_relinquish();
     }
     // Everything above overlaps the previous kernel; from here on its results
-    // (offsets, activations) are read and this kernel's outputs are written.
+    // (offsets, x_perm) are read and this kernel's outputs are written.
     ptx::grid_dep_wait();
     if (warp == 2) {
-        // Segment table and the unit prefix (units of expert e =
-        // ceil(rows_e / BN) token tiles x MB weight blocks).
+        // Segment table and the unit / tile prefixes per expert.
         const int per = (E + 31) >> 5;
         const int base = lane * per;
         bool bad = false;
-        int local = 0;
+        int nu = 0, nd = 0, nt = 0;
         for (int i = 0; i < per; ++i) {
             const int e = base + i;
             if (e < E) {
@@ -183,54 +248,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 s_off[e] = o0;
                 if (e == E - 1) s_off[E] = o1;
                 const int c = o1 - o0;
-                if (o0 < 0 || c < 0 || o1 > p.S) bad = true;
-                else local += ((c + BN - 1) / BN) * MB * KSPLIT;
+                if (o0 < 0 || c < 0 || o1 > p.S) {
+                    bad = true;
+                } else {
+                    const int ntb = (c + BN - 1) / BN;
+                    nt += ntb;
+                    nu += ntb * MBU;
+                    nd += ntb * MBD * KSPLIT;
+                }
             }
         }
         bad = __any_sync(0xffffffffu, bad);
         if (bad) {
-            local = 0;
+            nu = nd = nt = 0;
             if (lane == 0) atomicOr(p.err, kErrOffsets);
         }
-        int incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
-        int run = incl - local;
+        const int iu = warp_incl_scan(nu, lane);
+        const int id = warp_incl_scan(nd, lane);
+        const int it = warp_incl_scan(nt, lane);
+        int ru = iu - nu, rd = id - nd, rt = it - nt;
         for (int i = 0; i < per; ++i) {
             const int e = base + i;
             if (e < E) {
-                s_pre[e] = run;
+                s_pu[e] = ru;
+                s_pd[e] = rd;
+                s_tb[e] = rt;
                 if (!bad) {
-                    const int c = s_off[e + 1] - s_off[e];
-                    run += ((c + BN - 1) / BN) * MB * KSPLIT;
+                    const int ntb = (s_off[e + 1] - s_off[e] + BN - 1) / BN;
+                    ru += ntb * MBU;
+                    rd += ntb * MBD * KSPLIT;
+                    rt += ntb;
                 }
             }
         }
-        if (lane == 31) s_pre[E] = incl;
+        if (lane == 31) {
+            s_pu[E] = iu;
+            s_pd[E] = id;
+            s_tb[E] = it;
+        }
     }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int total = s_pre[E];
+    const int u_up = s_pu[E];
+    const int total = u_up + s_pd[E];
 
     if (warp == 0) {
         if (lane == 0) {
             uint32_t stage = 0, phase = 0, issued = 0;
-            uint32_t last_parity[kGemmMaxStages];
+            uint32_t last_parity[kMaxStages];
 #pragma unroll
-            for (int s = 0; s < kGemmMaxStages; ++s) last_parity[s] = 0;
+            for (int s = 0; s < kMaxStages; ++s) last_parity[s] = 0;
             const uint64_t pol_w =
                 p.stream_weights ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             bool stop = false;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
-                const Unit w = decode_unit<BN>(u, s_pre, s_off, E, KSPLIT);
-                const int arow = w.e * p.M_rows + w.mb * 128;
-                const int k_end = (w.ks + 1) * KS / KSPLIT;
-                for (int ks = w.ks * KS / KSPLIT; ks < k_end; ++ks) {
+                const Unit w =
+                    decode_unit<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+                const CUtensorMap *ta0 = w.up ? &tmW1 : &tmW2;
+                const CUtensorMap *ta1 = w.up ? &tmW3 : &tmW2;
+                const CUtensorMap *tb = w.up ? &tmX : &tmH;
+                const int arow0 = w.up ? w.e * p.d_ff + w.blk * 128 : w.e * p.d + w.blk * 256;
+                const int arow1 = w.up ? arow0 : arow0 + 128;
+                if (!w.up) {
+                    // The H tile must be complete before any of its copies: every
+                    // up block of this token tile stored by its four epilogue warps.
+                    if (!wait_counter(&p.h_ready[w.tile], ready_target, abort_flag, p.err)) break;
+                    fence_proxy_async_global();
+                }
+                for (int ks = w.k_beg; ks < w.k_end; ++ks) {
                     if (!bounded_wait(&empty[stage], phase ^ 1u, abort_flag, p.err,
                                       kErrTimeoutMma)) {
                         stop = true;
@@ -238,21 +325,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     uint8_t *sa = smem + stage * C::kStageBytes;
                     ptx::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-                    ptx::tma_load_2d_hint(sa, &tmA0, &full[stage], ks * 64, arow, pol_w);
-                    if (UP)
-                        ptx::tma_load_2d_hint(sa + kWTileBytes, &tmA1, &full[stage], ks * 64, arow,
-                                              pol_w);
-                    ptx::tma_load_2d(sa + C::kA * kWTileBytes, &tmB, &full[stage], ks * 64, w.r0);
+                    ptx::tma_load_2d_hint(sa, ta0, &full[stage], ks * 64, arow0, pol_w);
+                    ptx::tma_load_2d_hint(sa + kWTile, ta1, &full[stage], ks * 64, arow1, pol_w);
+                    ptx::tma_load_2d(sa + 2 * kWTile, tb, &full[stage], ks * 64, w.r0);
                     issued |= 1u << stage;
                     last_parity[stage] = phase;
-                    if (++stage == static_cast<uint32_t>(C::kStages)) {
+                    if (++stage == static_cast<uint32_t>(ST)) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             // Make sure no copy is still landing in shared memory at exit.
-            for (int s = 0; s < C::kStages; ++s)
+            for (int s = 0; s < ST; ++s)
                 if (issued & (1u << s)) drain_wait(&full[s], last_parity[s]);
         }
     } else if (warp == 1) {
@@ -261,10 +346,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int i = 0;
             bool stop = false;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x, ++i) {
-                const Unit w = decode_unit<BN>(u, s_pre, s_off, E, KSPLIT);
+                const Unit w =
+                    decode_unit<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
                 const int n = ((w.valid + 15) >> 4) << 4;
-                const int k_beg = w.ks * KS / KSPLIT;
-                const int k_end = (w.ks + 1) * KS / KSPLIT;
                 const uint32_t idesc = ptx::idesc_bf16_f32(128, n);
                 const int buf = i & 1;
                 const uint32_t use = static_cast<uint32_t>(i >> 1);
@@ -273,27 +357,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem + static_cast<uint32_t>(buf * C::kAccCols);
-                for (int ks = k_beg; ks < k_end; ++ks) {
+                for (int ks = w.k_beg; ks < w.k_end; ++ks) {
                     if (!bounded_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutTma)) {
                         stop = true;
                         break;
                     }
                     ptx::tc_fence_after();
                     const uint32_t sa = ptx::smem_addr(smem + stage * C::kStageBytes);
-                    const uint32_t sb = sa + C::kA * kWTileBytes;
+                    const uint32_t sb = sa + 2 * kWTile;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
-                        const uint32_t acc = ((ks - k_beg) | kk) ? 1u : 0u;
+                        const uint32_t acc = ((ks - w.k_beg) | kk) ? 1u : 0u;
                         ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc, idesc,
                                          acc);
-                        if (UP)
-                            ptx::tc_mma_bf16(d0 + BN,
-                                             ptx::sw128_kmajor_desc(sa + kWTileBytes + kk * 32),
-                                             bdesc, idesc, acc);
+                        ptx::tc_mma_bf16(d0 + BN, ptx::sw128_kmajor_desc(sa + kWTile + kk * 32),
+                                         bdesc, idesc, acc);
                     }
                     ptx::tc_commit(&empty[stage]);
-                    if (++stage == static_cast<uint32_t>(C::kStages)) {
+                    if (++stage == static_cast<uint32_t>(ST)) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -309,45 +391,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         int i = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x, ++i) {
-            const Unit w = decode_unit<BN>(u, s_pre, s_off, E, KSPLIT);
+            const Unit w = decode_unit<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
             const int buf = i & 1;
             const uint32_t use = static_cast<uint32_t>(i >> 1);
             if (!bounded_wait_warp(&tfull[buf], use & 1u, abort_flag, p.err, kErrTimeoutMma))
                 break;
             ptx::tc_fence_after();
-            const int f = w.mb * 128 + 32 * q + lane;  // output column of this thread
             const uint32_t tb = tmem + lane_base + static_cast<uint32_t>(buf * C::kAccCols);
+            const int row_in_blk = 32 * q + lane;
             for (int c0 = 0; c0 < w.valid; c0 += 32) {
-                if (UP) {
-                    uint32_t a[32], b[32];
-                    ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), a);
-                    ptx::tmem_ld32(tb + static_cast<uint32_t>(BN + c0), b);
-                    ptx::tc_wait_ld();
-                    __nv_bfloat16 *H = static_cast<__nv_bfloat16 *>(p.out);
+                uint32_t a[32], b[32];
+                ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), a);
+                ptx::tmem_ld32(tb + static_cast<uint32_t>(BN + c0), b);
+                ptx::tc_wait_ld();
+                if (w.up) {
+                    const int f = w.blk * 128 + row_in_blk;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         if (c0 + j < w.valid) {
                             const float g = __uint_as_float(a[j]);
                             const float h = g * __frcp_rn(1.0f + __expf(-g)) * __uint_as_float(b[j]);
-                            H[static_cast<size_t>(w.r0 + c0 + j) * p.M_rows + f] =
+                            p.H[static_cast<size_t>(w.r0 + c0 + j) * p.d_ff + f] =
                                 __float2bfloat16_rn(h);
                         }
                     }
                 } else {
-                    uint32_t y[32];
-                    ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), y);
-                    ptx::tc_wait_ld();
-                    float *Y = static_cast<float *>(p.out) + w.ks * p.part_stride;
+                    const int o0 = w.blk * 256 + row_in_blk;
+                    const bool has1 = o0 + 128 < p.d;
+                    float *Y = p.Y + w.ks * p.part_stride;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < w.valid)
-                            Y[static_cast<size_t>(w.r0 + c0 + j) * p.M_rows + f] =
-                                __uint_as_float(y[j]);
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < w.valid) {
+                            float *yr = Y + static_cast<size_t>(w.r0 + c0 + j) * p.d;
+                            yr[o0] = __uint_as_float(a[j]);
+                            if (has1) yr[o0 + 128] = __uint_as_float(b[j]);
+                        }
+                    }
                 }
             }
             ptx::tc_fence_before();
+            if (w.up) {
+                // Publish this warp's slice of the H block to the down units
+                // (which read it through TMA, the async proxy).
+                fence_proxy_async_global();
+                __threadfence();
+            }
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+            if (lane == 0) {
+                if (w.up) atomicAdd(&p.h_ready[w.tile], 1u);
+                ptx::mbar_arrive(&tempty[buf]);
+            }
         }
     }
 
@@ -358,66 +451,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 }
 
-template <bool UP, int BN, int ST>
-cudaError_t launch_gemm_cfg(const GemmLaunch &a, cudaStream_t s)
+template <int BN, int ST>
+cudaError_t launch_ffn_cfg(const FfnLaunch &a, cudaStream_t s)
 {
-    using C = Cfg<UP, BN, ST>;
-    CUtensorMap tA0, tA1, tB;
-    cudaError_t e = make_tmap_bf16(&tA0, a.A0, static_cast<uint64_t>(a.E) * a.M_rows, a.K, 128);
+    using C = FfnCfg<BN, ST>;
+    const int E = a.offsets ? a.E : 1;
+    CUtensorMap tW1, tW3, tW2, tX, tH;
+    cudaError_t e = make_tmap_bf16(&tW1, a.W1, static_cast<uint64_t>(E) * a.d_ff, a.d, 128);
+    if (e == cudaSuccess) e = make_tmap_bf16(&tW3, a.W3, static_cast<uint64_t>(E) * a.d_ff, a.d, 128);
+    if (e == cudaSuccess) e = make_tmap_bf16(&tW2, a.W2, static_cast<uint64_t>(E) * a.d, a.d_ff, 128);
+    if (e == cudaSuccess) e = make_tmap_bf16(&tX, a.x, a.S, a.d, BN);
+    if (e == cudaSuccess) e = make_tmap_bf16(&tH, a.H, a.S, a.d_ff, BN);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16(&tA1, UP ? a.A1 : a.A0, static_cast<uint64_t>(a.E) * a.M_rows, a.K, 128);
-    if (e != cudaSuccess) return e;
-    e = make_tmap_bf16(&tB, a.B, a.S, a.K, BN);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemm_kernel<UP, BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(ffn_kernel<BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return e;
 
-    GemmParams p;
-    p.E = a.offsets ? a.E : 1;
-    p.M_rows = a.M_rows;
-    p.K = a.K;
+    FfnParams p;
+    p.E = E;
+    p.d = a.d;
+    p.d_ff = a.d_ff;
     p.S = a.S;
+    p.ksplit = a.ksplit < 1 ? 1 : a.ksplit;
+    p.part_stride = static_cast<size_t>(a.S) * a.d;
     p.offsets = a.offsets;
-    p.out = a.out;
+    p.H = reinterpret_cast<__nv_bfloat16 *>(a.H);
+    p.Y = a.Y;
+    p.h_ready = a.h_ready;
     p.err = a.err;
     p.stream_weights = a.max_rows <= BN ? 1 : 0;
-    p.ksplit = UP ? 1 : (a.ksplit < 1 ? 1 : a.ksplit);
-    p.part_stride = static_cast<size_t>(a.S) * a.M_rows;
     // Upper bound of the work units: every segment rounds up to whole tiles.
-    const long long tiles = (static_cast<long long>(a.S) + BN - 1) / BN + p.E;
-    const long long units = tiles * (a.M_rows / 128) * p.ksplit;
+    const long long tiles = (static_cast<long long>(a.S) + BN - 1) / BN + E;
+    const long long units = tiles * (a.d_ff / 128) + tiles * ((a.d + 255) / 256) * p.ksplit;
     long long grid = device_sm_count();
     if (units < grid) grid = units;
     if (grid < 1) grid = 1;
-    return launch_pdl(gemm_kernel<UP, BN, ST>, dim3(static_cast<unsigned>(grid)),
-                      dim3(kGemmThreads), C::kSmem, s, a.pdl, tA0, tA1, tB, p);
+    return launch_pdl(ffn_kernel<BN, ST>, dim3(static_cast<unsigned>(grid)), dim3(kFfnThreads),
+                      C::kSmem, s, a.pdl, tW1, tW3, tW2, tX, tH, p);
 }
 
 }  // namespace
 
-int gemm_token_tile(int up, int S, int E_seg)
+int ffn_token_tile(int S, int E_seg)
 {
     // Token tile from the average rows per segment: small tiles waste no
     // MMA columns and leave room for a deeper weight pipeline.
     const long long avg = (static_cast<long long>(S) + E_seg - 1) / E_seg;
     if (avg <= 32) return 32;
     if (avg <= 64) return 64;
-    if (up || avg <= 128) return 128;
-    return 256;
+    return 128;
+}
+
+size_t ffn_ready_counters(int S, int E_seg)
+{
+    // One counter per token tile; tiles are at least 32 rows and every
+    // segment adds at most one partial tile.
+    return static_cast<size_t>((S + 31) / 32 + E_seg);
 }
 
 int down_ksplit(int S, int E_seg, int d, int d_ff)
 {
-    // Split K of the down projection when its (segment x weight block) units
-    // cannot fill the GPU: pick the split whose unit count fills whole waves
-    // of the SMs best, keeping at least 8 K steps per range.
-    const int bn = gemm_token_tile(0, S, E_seg);
+    // Split K of the down projection when its (segment x weight block pair)
+    // units cannot fill the GPU once: pick the split whose unit count fills
+    // whole waves of the SMs best, keeping at least 8 K steps per range.
+    const int bn = ffn_token_tile(S, E_seg);
     const long long hit = std::min<long long>(E_seg, S);
-    const long long units = (d / 128) * std::max<long long>(hit, (S + bn - 1) / bn);
+    const long long units = ((d + 255) / 256) * std::max<long long>(hit, (S + bn - 1) / bn);
     const long long sms = 148;
-    if (units >= 2 * sms) return 1;
-    const int max_ks = std::max(1, std::min(8, d_ff / 64 / 8));  // 8: the combine sums at most 8 partials
+    if (units >= sms) return 1;
+    const int max_ks = std::max(1, std::min(8, d_ff / 64 / 8));
     int best = 1;
     double best_eff = 0.0;
     for (int ks = 1; ks <= max_ks; ++ks) {
@@ -432,21 +534,12 @@ int down_ksplit(int S, int E_seg, int d, int d_ff)
     return best;
 }
 
-cudaError_t launch_gemm(const GemmLaunch &a, cudaStream_t s)
+cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s)
 {
-    const int bn = gemm_token_tile(a.up, a.S, a.offsets ? a.E : 1);
-    if (a.up) {
-        switch (bn) {
-        case 32: return launch_gemm_cfg<true, 32, 5>(a, s);
-        case 64: return launch_gemm_cfg<true, 64, 5>(a, s);
-        default: return launch_gemm_cfg<true, 128, 4>(a, s);
-        }
-    }
-    switch (bn) {
-    case 32: return launch_gemm_cfg<false, 32, 10>(a, s);
-    case 64: return launch_gemm_cfg<false, 64, 8>(a, s);
-    case 128: return launch_gemm_cfg<false, 128, 6>(a, s);
-    default: return launch_gemm_cfg<false, 256, 4>(a, s);
+    switch (ffn_token_tile(a.S, a.offsets ? a.E : 1)) {
+    case 32: return launch_ffn_cfg<32, 6>(a, s);
+    case 64: return launch_ffn_cfg<64, 5>(a, s);
+    default: return launch_ffn_cfg<128, 4>(a, s);
     }
 }
 

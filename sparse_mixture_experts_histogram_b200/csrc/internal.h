@@ -41,19 +41,20 @@ struct ScatterLaunch {
     bool pdl;  // launched right after another kernel of this library
 };
 
-struct GemmLaunch {
-    int up;               // 1: H = silu(W1 x) * (W3 x) (bf16 out); 0: Y = W2 H (fp32 out)
-    int E;                // experts (segments)
-    int M_rows;           // weight rows per expert: d_ff (up) or d (down)
-    int K;                // reduction length: d (up) or d_ff (down)
-    int S;                // rows of the activation operand
-    int max_rows;         // upper bound of rows in one segment (weights streamed once if <= tile)
-    int ksplit;           // down only: K split into this many ranges, partial outputs
-                          // [ksplit, S, M_rows] summed by the caller (the combine)
-    const int32_t *offsets;   // [E+1] device, or nullptr for one segment [0, S)
-    const uint16_t *A0, *A1;  // W1, W3 (up) or W2 (down, A1 unused)
-    const uint16_t *B;        // x_perm (up) or H (down)
-    void *out;                // H [S, M_rows] bf16 or Y [S, M_rows] fp32
+struct FfnLaunch {
+    int E;                    // segments (ignored when offsets is null: one segment [0, S))
+    int d, d_ff;
+    int S;                    // rows of x / H / Y
+    int max_rows;             // upper bound of rows in one segment (weights streamed once if <= tile)
+    int ksplit;               // K ranges of the down projection: partial outputs
+                              // [ksplit, S, d] summed by the caller (the combine)
+    const int32_t *offsets;   // [E+1] device, or nullptr
+    const uint16_t *W1, *W3;  // [E, d_ff, d]
+    const uint16_t *W2;       // [E, d, d_ff]
+    const uint16_t *x;        // [S, d]
+    uint16_t *H;              // [S, d_ff] intermediate
+    float *Y;                 // [ksplit, S, d]
+    uint32_t *h_ready;        // ffn_ready_counters(S, E) counters, zero before the launch
     uint32_t *err;
     bool pdl;                 // launched right after another kernel of this library
 };
@@ -72,8 +73,9 @@ struct CombineLaunch {
 cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s);
 cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s);
 cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s);
-cudaError_t launch_gemm(const GemmLaunch &a, cudaStream_t s);
-int gemm_token_tile(int up, int S, int E_seg);
+cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s);
+int ffn_token_tile(int S, int E_seg);
+size_t ffn_ready_counters(int S, int E_seg);
 int down_ksplit(int S, int E_seg, int d, int d_ff);
 cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s);
 

@@ -69,9 +69,11 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
     const void *ptrs[] = {x_perm, offsets, W1, W3, W2, y_perm};
     for (const void *p : ptrs)
         if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
-    // H [S, d_ff] bf16 must fit in the fixed scratch behind the header.
+    // The tile counters and H [S, d_ff] bf16 must fit in the fixed scratch
+    // behind the header.
+    const size_t ctr_bytes = (ffn_ready_counters(S, E) * 4 + 255) / 256 * 256;
     const size_t h_bytes = static_cast<size_t>(S) * d_ff * 2;
-    if (h_bytes > kStaticScratchBytes - kStaticHeaderBytes) return MOE_ERR_WORKSPACE;
+    if (ctr_bytes + h_bytes > kStaticScratchBytes - kStaticHeaderBytes) return MOE_ERR_WORKSPACE;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStaticMaxDevices)
@@ -80,35 +82,27 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
     if (scratch == nullptr) return MOE_ERR_CUDA;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // The error word must start at zero; H is fully written before it is read.
-    if (cudaMemsetAsync(scratch, 0, kStaticHeaderBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
-    uint32_t *err = reinterpret_cast<uint32_t *>(scratch);
-    uint16_t *H = reinterpret_cast<uint16_t *>(scratch + kStaticHeaderBytes);
-
-    GemmLaunch g;
-    g.up = 1;
-    g.E = E;
-    g.M_rows = d_ff;
-    g.K = d;
-    g.S = S;
-    g.max_rows = S;
-    g.offsets = offsets;
-    g.A0 = W1;
-    g.A1 = W3;
-    g.B = x_perm;
-    g.out = H;
-    g.err = err;
-    g.ksplit = 1;
-    g.pdl = false;
-    if (launch_gemm(g, s) != cudaSuccess) return MOE_ERR_CUDA;
-    g.pdl = true;
-    g.up = 0;
-    g.M_rows = d;
-    g.K = d_ff;
-    g.A0 = W2;
-    g.A1 = nullptr;
-    g.B = H;
-    g.out = y_perm;
-    if (launch_gemm(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // The error word and the tile counters must start at zero; H is fully
+    // written before it is read.
+    if (cudaMemsetAsync(scratch, 0, kStaticHeaderBytes + ctr_bytes, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    FfnLaunch f;
+    f.E = E;
+    f.d = d;
+    f.d_ff = d_ff;
+    f.S = S;
+    f.max_rows = S;
+    f.ksplit = 1;
+    f.offsets = offsets;
+    f.W1 = W1;
+    f.W3 = W3;
+    f.W2 = W2;
+    f.x = x_perm;
+    f.H = reinterpret_cast<uint16_t *>(scratch + kStaticHeaderBytes + ctr_bytes);
+    f.Y = y_perm;
+    f.h_ready = reinterpret_cast<uint32_t *>(scratch + kStaticHeaderBytes);
+    f.err = reinterpret_cast<uint32_t *>(scratch);
+    f.pdl = false;
+    if (launch_ffn(f, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -99,9 +99,12 @@ def test_null_misaligned_and_small_workspace(lib):
     assert lib.moe_forward_ex(16, 512, 8, 1024, 2, FAKE, FAKE, None, FAKE, FAKE, FAKE, 256,
                               None, None, None, FAKE, FAKE, 1 << 40, None) == 1
     # traced forward needs exactly MOE_TRACE_EVENTS events
-    evs = (ctypes.c_void_p * 8)()
+    evs = (ctypes.c_void_p * binding.TRACE_EVENTS)()
     assert lib.moe_forward_traced(16, 512, 8, 1024, 2, FAKE, FAKE, None, FAKE, FAKE, FAKE, 0,
-                                  None, None, None, FAKE, FAKE, 1 << 40, None, evs, 7) == 1
+                                  None, None, None, FAKE, FAKE, 1 << 40, None, evs,
+                                  binding.TRACE_EVENTS - 1) == 1
+    assert "#define MOE_TRACE_EVENTS %d" % binding.TRACE_EVENTS in open(
+        os.path.join(ROOT, "include", "moe.h")).read()
     assert lib.moe_get_device_error(None, None, None) == 1
 
 

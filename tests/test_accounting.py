@@ -60,10 +60,12 @@ def test_flops_and_bytes_closed_forms():
     assert abs(acc.active_flops(512, 512, 8, 4096, 2) / 1e9 - 12.89) < 0.01
     # Mixtral prefill T=8192: 5.773 TFLOP
     assert abs(acc.active_flops(8192, 4096, 8, 14336, 2) / 1e12 - 5.773) < 0.001
-    # the two grouped GEMMs carry all expert FLOPs
+    # the expert FFN kernels (routed + shared) carry all expert FLOPs
     for (T, d, f, k, fs) in [(512, 512, 4096, 2, 0), (8192, 7168, 2048, 8, 2048)]:
-        assert acc.gemm_flops("up", T, d, f, k, fs) + acc.gemm_flops("down", T, d, f, k, fs) == \
+        assert acc.ffn_flops(T, d, f, k) + acc.ffn_flops(T, d, fs, 1) == \
             acc.active_flops(T, d, 1, f, k, fs) - 2 * T * d
+    # the FFN kernel's bytes: all hit experts' weights once, rows in, fp32 rows out
+    assert acc.ffn_bytes(512, 512, 4096, 2, 8) == 2 * 3 * 8 * 512 * 4096 + 6 * 1024 * 512
     # decode T=1 streams the two hit experts: 0.70 GB
     b = acc.algorithmic_bytes(1, 4096, 8, 14336, 2, experts_hit=2)
     assert abs(b / 1e9 - 0.705) < 0.001
