@@ -41,8 +41,8 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     const size_t ntiles = (static_cast<size_t>(T) + 127) / 128;
     const size_t S = static_cast<size_t>(T) * k;
     L.tilectr = take(ntiles * 4);
-    L.hready = take(ffn_ready_counters(static_cast<int>(S), E) * 4);
-    L.hready_s = d_ffs > 0 ? take(ffn_ready_counters(T, 1) * 4) : 0;
+    L.hready = take(ffn_ready_counters(static_cast<int>(S), E, d_ff) * 4);
+    L.hready_s = d_ffs > 0 ? take(ffn_ready_counters(T, 1, d_ffs) * 4) : 0;
     L.zero_bytes = o;
     L.tilecnt = take(ntiles * E * 4);
     L.tilebase = take(ntiles * E * 4);
@@ -286,7 +286,7 @@ moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
     if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
         !ok_ptr(y_perm) || !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
-    const size_t ctr = align_up(ffn_ready_counters(S, E) * 4);
+    const size_t ctr = align_up(ffn_ready_counters(S, E, d_ff) * 4);
     const size_t need = kHeaderBytes + ctr + align_up(static_cast<size_t>(S) * d_ff * 2);
     if (ws_bytes < need) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -403,8 +403,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
         float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
         st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys,
-                      reinterpret_cast<uint32_t *>(wsb + L.hready_s), err, s, events == nullptr,
-                      1);
+                      reinterpret_cast<uint32_t *>(wsb + L.hready_s), err, s, false, 1);
         if (st != MOE_OK) return st;
         shared_y = Ys;
     }
@@ -420,7 +419,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     cb.w = w;
     cb.shared_y = shared_y;
     cb.out = out;
-    cb.pdl = events == nullptr;
+    cb.pdl = false;  // after a persistent kernel an early launch only takes SM slots
     st = from_cuda(launch_combine(cb, s));
     if (st != MOE_OK) return st;
     return mark(events, 5, s);

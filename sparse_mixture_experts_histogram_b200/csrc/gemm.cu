@@ -17,12 +17,14 @@
 // stages, warp 1 issues the MMAs into a double-buffered tensor-memory
 // accumulator, warps 2..5 drain finished accumulators and store.  Every CTA
 // walks the units numbered up-first (expert, block, token tile) and then
-// down (expert, block pair, token tile, K range).  A down unit needs all of
-// its token tile's H columns: the up epilogues count finished blocks per
-// tile, and the producer waits (bounded) for the count before it copies that
-// H tile.  Since each CTA finishes its up units before its down units, and
-// an up unit never waits, the wait always ends; the down weights stream while
-// the last up units finish.
+// down (expert, block pair, token tile, K range).  A down unit reads, per K
+// step, 64 columns of its token tile's H: the up epilogues mark each finished
+// (token tile, 128-column block) of H, and the producer waits (bounded) for
+// that mark before it copies the columns -- after it has already issued the
+// step's W2 copies.  A unit only ever waits for units numbered before it, and
+// every CTA takes its units in increasing order, so the lowest unfinished
+// unit can always proceed: the waits always end.  Down work starts on the
+// first finished H blocks while later up blocks are still running.
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward; "Mixtral and MoE
@@ -74,7 +76,7 @@ struct FfnParams {
     const int32_t *offsets; // [E+1] or nullptr (one segment [0, S))
     __nv_bfloat16 *H;       // [S, d_ff]
     float *Y;               // [ksplit, S, d]
-    uint32_t *h_ready;      // [tiles] finished (up block x epilogue warp) count per token tile
+    uint32_t *h_ready;      // [tiles, d_ff/128]: epilogue warps done with (token tile, H block)
     uint32_t *err;
     int stream_weights;     // each weight block feeds one token tile: L2 evict-first
 };
@@ -204,9 +206,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     const int KSU = p.d / 64;
     const int KSD = p.d_ff / 64;
     const int KSPLIT = p.ksplit;
-    const uint32_t ready_target = 4u * static_cast<uint32_t>(MBU);
+    const uint32_t ready_target = 4u;  // the four epilogue warps of the up unit
 
-    ptx::grid_dep_launch();
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -311,12 +312,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                 const CUtensorMap *tb = w.up ? &tmX : &tmH;
                 const int arow0 = w.up ? w.e * p.d_ff + w.blk * 128 : w.e * p.d + w.blk * 256;
                 const int arow1 = w.up ? arow0 : arow0 + 128;
-                if (!w.up) {
-                    // The H tile must be complete before any of its copies: every
-                    // up block of this token tile stored by its four epilogue warps.
-                    if (!wait_counter(&p.h_ready[w.tile], ready_target, abort_flag, p.err)) break;
-                    fence_proxy_async_global();
-                }
+                int ready_blk = -1;
                 for (int ks = w.k_beg; ks < w.k_end; ++ks) {
                     if (!bounded_wait(&empty[stage], phase ^ 1u, abort_flag, p.err,
                                       kErrTimeoutMma)) {
@@ -327,9 +323,20 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                     ptx::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
                     ptx::tma_load_2d_hint(sa, ta0, &full[stage], ks * 64, arow0, pol_w);
                     ptx::tma_load_2d_hint(sa + kWTile, ta1, &full[stage], ks * 64, arow1, pol_w);
-                    ptx::tma_load_2d(sa + 2 * kWTile, tb, &full[stage], ks * 64, w.r0);
                     issued |= 1u << stage;
                     last_parity[stage] = phase;
+                    if (!w.up && (ks >> 1) != ready_blk) {
+                        // These 64 columns of H belong to 128-column block ks/2:
+                        // wait until its up unit has stored and published it.
+                        ready_blk = ks >> 1;
+                        if (!wait_counter(&p.h_ready[w.tile * MBU + ready_blk], ready_target,
+                                          abort_flag, p.err)) {
+                            stop = true;
+                            break;
+                        }
+                        fence_proxy_async_global();
+                    }
+                    ptx::tma_load_2d(sa + 2 * kWTile, tb, &full[stage], ks * 64, w.r0);
                     if (++stage == static_cast<uint32_t>(ST)) {
                         stage = 0;
                         phase ^= 1u;
@@ -438,12 +445,15 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
             }
             __syncwarp();
             if (lane == 0) {
-                if (w.up) atomicAdd(&p.h_ready[w.tile], 1u);
+                if (w.up) atomicAdd(&p.h_ready[w.tile * MBU + w.blk], 1u);
                 ptx::mbar_arrive(&tempty[buf]);
             }
         }
     }
 
+    // Dependents (the shared expert, the combine) need this kernel's results:
+    // let them launch only once its work is done.
+    ptx::grid_dep_launch();
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
@@ -494,19 +504,21 @@ cudaError_t launch_ffn_cfg(const FfnLaunch &a, cudaStream_t s)
 
 int ffn_token_tile(int S, int E_seg)
 {
-    // Token tile from the average rows per segment: small tiles waste no
-    // MMA columns and leave room for a deeper weight pipeline.
-    const long long avg = (static_cast<long long>(S) + E_seg - 1) / E_seg;
-    if (avg <= 32) return 32;
-    if (avg <= 64) return 64;
+    // Token tile from the rows a segment is expected to hold (1.5x the
+    // average, so that few segments spill into a second, mostly empty tile
+    // that streams the same weights again); small tiles waste no MMA columns
+    // and leave room for a deeper weight pipeline.
+    const long long expect = (3LL * S + 2LL * E_seg - 1) / (2LL * E_seg);
+    if (expect <= 32) return 32;
+    if (expect <= 64) return 64;
     return 128;
 }
 
-size_t ffn_ready_counters(int S, int E_seg)
+size_t ffn_ready_counters(int S, int E_seg, int d_ff)
 {
-    // One counter per token tile; tiles are at least 32 rows and every
-    // segment adds at most one partial tile.
-    return static_cast<size_t>((S + 31) / 32 + E_seg);
+    // One counter per (token tile, 128-column block of H); tiles are at least
+    // 32 rows and every segment adds at most one partial tile.
+    return static_cast<size_t>((S + 31) / 32 + E_seg) * static_cast<size_t>(d_ff / 128);
 }
 
 int down_ksplit(int S, int E_seg, int d, int d_ff)

@@ -54,7 +54,7 @@ struct FfnLaunch {
     const uint16_t *x;        // [S, d]
     uint16_t *H;              // [S, d_ff] intermediate
     float *Y;                 // [ksplit, S, d]
-    uint32_t *h_ready;        // ffn_ready_counters(S, E) counters, zero before the launch
+    uint32_t *h_ready;        // ffn_ready_counters(S, E, d_ff) counters, zero before the launch
     uint32_t *err;
     bool pdl;                 // launched right after another kernel of this library
 };
@@ -75,7 +75,7 @@ cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s);
 cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s);
 cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s);
 int ffn_token_tile(int S, int E_seg);
-size_t ffn_ready_counters(int S, int E_seg);
+size_t ffn_ready_counters(int S, int E_seg, int d_ff);
 int down_ksplit(int S, int E_seg, int d, int d_ff);
 cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s);
 

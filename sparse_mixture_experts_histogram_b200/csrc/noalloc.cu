@@ -71,7 +71,7 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
         if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
     // The tile counters and H [S, d_ff] bf16 must fit in the fixed scratch
     // behind the header.
-    const size_t ctr_bytes = (ffn_ready_counters(S, E) * 4 + 255) / 256 * 256;
+    const size_t ctr_bytes = (ffn_ready_counters(S, E, d_ff) * 4 + 255) / 256 * 256;
     const size_t h_bytes = static_cast<size_t>(S) * d_ff * 2;
     if (ctr_bytes + h_bytes > kStaticScratchBytes - kStaticHeaderBytes) return MOE_ERR_WORKSPACE;
 
