@@ -18,7 +18,8 @@ namespace moe {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, ranks counter @8
+constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, ranks counter @8,
+                                      // partial outputs per row of the expert kernel @12
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -27,6 +28,14 @@ struct Layout {
     size_t zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
     size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, xperm, H, Y, Hs, Ys, total;
 };
+
+// Partial expert outputs the routed experts' kernel writes per row: the
+// narrow-layer kernel splits the hidden width, the general one may split the
+// down projection's K.
+int ffn_splits(int S, int E, int d, int d_ff)
+{
+    return ffn_small_supported(d) ? ffn_small_splits(S, E, d, d_ff) : down_ksplit(S, E, d, d_ff);
+}
 
 // Workspace of moe_forward_ex (a superset of every other entry point's need).
 Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
@@ -54,7 +63,7 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     L.row = take(S * 4);
     L.xperm = take(S * d * 2);
     L.H = take(S * d_ff * 2);
-    L.Y = take(S * d * 4 * static_cast<size_t>(down_ksplit(static_cast<int>(S), E, d, d_ff)));
+    L.Y = take(S * d * 4 * static_cast<size_t>(ffn_splits(static_cast<int>(S), E, d, d_ff)));
     if (d_ffs > 0) {
         L.Hs = take(static_cast<size_t>(T) * d_ffs * 2);
         L.Ys = take(static_cast<size_t>(T) * d * 4);
@@ -165,7 +174,7 @@ static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, cons
                              const float *bias, int32_t *idx, float *w, int32_t *counts,
                              int32_t *offsets, uint8_t *ws, const Layout &L, cudaStream_t s)
 {
-    RouteLaunch a;
+    RouteLaunch a{};
     a.T = T;
     a.d = d;
     a.E = E;
@@ -220,7 +229,7 @@ moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int3
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
     if (st != MOE_OK) return st;
-    RanksLaunch r;
+    RanksLaunch r{};
     r.T = T;
     r.E = E;
     r.k = k;
@@ -233,7 +242,7 @@ moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int3
     r.err = reinterpret_cast<uint32_t *>(wsb);
     st = from_cuda(launch_ranks(r, s));
     if (st != MOE_OK) return st;
-    ScatterLaunch c;
+    ScatterLaunch c{};
     c.T = T;
     c.d = d;
     c.E = E;
@@ -256,7 +265,7 @@ static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const mo
                            const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *h_ready,
                            uint32_t *err, cudaStream_t s, bool pdl, int ksplit)
 {
-    FfnLaunch f;
+    FfnLaunch f{};
     f.E = E;
     f.d = d;
     f.d_ff = d_ff;
@@ -307,7 +316,7 @@ moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *
     if (!ok_ptr(y_perm) || !ok_ptr(row_of_slot) || !ok_ptr(w) || !ok_ptr(out))
         return MOE_ERR_INVALID_ARG;
     if (shared_y != nullptr && !aligned16(shared_y)) return MOE_ERR_INVALID_ARG;
-    CombineLaunch c;
+    CombineLaunch c{};
     c.T = T;
     c.d = d;
     c.k = k;
@@ -372,7 +381,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
                     reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s);
     if (st != MOE_OK) return st;
 
-    ScatterLaunch c;
+    ScatterLaunch c{};
     c.T = T;
     c.d = d;
     c.E = E;
@@ -390,11 +399,32 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     if (st != MOE_OK) return st;
 
     // A token never picks one expert twice, so no segment exceeds T rows.
-    const int ksplit = down_ksplit(S, E, d, d_ff);
+    const int ksplit = ffn_splits(S, E, d, d_ff);
     if ((st = mark(events, 2, s)) != MOE_OK) return st;
-    st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
-                  reinterpret_cast<uint32_t *>(wsb + L.hready), err, s, events == nullptr,
-                  ksplit);
+    if (ffn_small_supported(d)) {
+        FfnLaunch f{};
+        f.E = E;
+        f.d = d;
+        f.d_ff = d_ff;
+        f.S = S;
+        f.max_rows = T;
+        f.ksplit = ksplit;
+        f.offsets = offsets;
+        f.W1 = W1;
+        f.W3 = W3;
+        f.W2 = W2;
+        f.x = xperm;
+        f.H = nullptr;
+        f.Y = Y;
+        f.h_ready = nullptr;
+        f.err = err;
+        f.pdl = events == nullptr;
+        st = from_cuda(launch_ffn_small(f, ksplit, reinterpret_cast<int *>(wsb + 12), s));
+    } else {
+        st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
+                      reinterpret_cast<uint32_t *>(wsb + L.hready), err, s, events == nullptr,
+                      ksplit);
+    }
     if (st != MOE_OK) return st;
 
     const float *shared_y = nullptr;
@@ -409,11 +439,12 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     }
     if ((st = mark(events, 4, s)) != MOE_OK) return st;
 
-    CombineLaunch cb;
+    CombineLaunch cb{};
     cb.T = T;
     cb.d = d;
     cb.k = k;
     cb.ksplit = ksplit;
+    cb.ksplit_dev = ffn_small_supported(d) ? reinterpret_cast<const int *>(wsb + 12) : nullptr;
     cb.y = Y;
     cb.row_of_slot = row;
     cb.w = w;

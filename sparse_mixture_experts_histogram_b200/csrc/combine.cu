@@ -23,6 +23,7 @@ constexpr int kCombineBatch = 8; // (slot, partial) pairs whose loads are in fli
 struct CombineParams {
     int T, d, k;
     int ksplit;          // partial outputs per row, summed in order before weighting
+    const int *ksplit_dev; // if set, the count is read here (written by the previous kernel)
     size_t part_stride;  // float4 between consecutive partial outputs
     const float4 *y;
     const int32_t *row_of_slot;
@@ -61,7 +62,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
         if (my_row >= p.T * p.k) my_row = -1;  // rows live in [0, T*k)
     }
     const int nv = p.d >> 2;
-    const int npairs = p.k * p.ksplit;
+    const int ksplit = p.ksplit_dev ? *p.ksplit_dev : p.ksplit;
+    const int npairs = p.k * ksplit;
     float4 acc[kCombineVec], yj[kCombineVec];
 #pragma unroll
     for (int u = 0; u < kCombineVec; ++u) {
@@ -73,8 +75,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
 #pragma unroll
         for (int i = 0; i < kCombineBatch; ++i) {
             const int pi = p0 + i;
-            const int j = pi / p.ksplit;
-            const int q = pi - j * p.ksplit;
+            const int j = pi / ksplit;
+            const int q = pi - j * ksplit;
             const int row = __shfl_sync(0xffffffffu, my_row, j & 31);
             const bool ok = pi < npairs && row >= 0;
             const float4 *src = p.y + q * p.part_stride + static_cast<size_t>(ok ? row : 0) * nv;
@@ -88,14 +90,14 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
         for (int i = 0; i < kCombineBatch; ++i) {
             const int pi = p0 + i;
             if (pi < npairs) {
-                const int j = pi / p.ksplit;
-                const int q = pi - j * p.ksplit;
+                const int j = pi / ksplit;
+                const int q = pi - j * ksplit;
 #pragma unroll
                 for (int u = 0; u < kCombineVec; ++u) {
                     if (q == 0) yj[u] = val[i][u];
                     else add4(yj[u], val[i][u]);
                 }
-                if (q == p.ksplit - 1) {
+                if (q == ksplit - 1) {
                     const float wj = __shfl_sync(0xffffffffu, my_w, j & 31);
 #pragma unroll
                     for (int u = 0; u < kCombineVec; ++u) {
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
 
 cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s)
 {
-    CombineParams p;
+    CombineParams p{};
     p.T = a.T;
     p.d = a.d;
     p.k = a.k;
@@ -132,6 +134,7 @@ cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s)
     p.shared_y = reinterpret_cast<const float4 *>(a.shared_y);
     p.out = reinterpret_cast<float4 *>(a.out);
     p.ksplit = a.ksplit < 1 ? 1 : a.ksplit;
+    p.ksplit_dev = a.ksplit_dev;
     p.part_stride = static_cast<size_t>(a.T) * a.k * (a.d / 4);
     const int nv = a.d / 4;
     p.chunks = (nv + 32 * kCombineVec - 1) / (32 * kCombineVec);

@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
 
 cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s)
 {
-    RanksParams p;
+    RanksParams p{};
     p.T = a.T;
     p.E = a.E;
     p.k = a.k;
@@ -136,7 +136,7 @@ cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s)
 
 cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s)
 {
-    ScatterParams p;
+    ScatterParams p{};
     p.T = a.T;
     p.d = a.d;
     p.E = a.E;

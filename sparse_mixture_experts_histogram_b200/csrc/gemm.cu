@@ -477,7 +477,7 @@ cudaError_t launch_ffn_cfg(const FfnLaunch &a, cudaStream_t s)
                              static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return e;
 
-    FfnParams p;
+    FfnParams p{};
     p.E = E;
     p.d = a.d;
     p.d_ff = a.d_ff;

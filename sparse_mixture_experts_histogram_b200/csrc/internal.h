@@ -62,6 +62,7 @@ struct FfnLaunch {
 struct CombineLaunch {
     int T, d, k;
     int ksplit;            // partial outputs per row of y, summed in order before weighting
+    const int *ksplit_dev; // or read from device memory (written by the expert kernel), if set
     const float *y;        // [ksplit, T*k, d]
     const int32_t *row_of_slot;
     const float *w;
@@ -74,6 +75,12 @@ cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s);
 cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s);
 cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s);
 cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s);
+// Narrow layers (d <= 1024): every CTA runs whole hidden chunks (up, H in
+// shared memory, down) and writes `nsplit` partial outputs [nsplit, S, d].
+cudaError_t launch_ffn_small(const FfnLaunch &a, int nsplit_max, int *nsplit_out,
+                             cudaStream_t s);
+bool ffn_small_supported(int d);
+int ffn_small_splits(int S, int E, int d, int d_ff);
 int ffn_token_tile(int S, int E_seg);
 size_t ffn_ready_counters(int S, int E_seg, int d_ff);
 int down_ksplit(int S, int E_seg, int d, int d_ff);

@@ -86,7 +86,7 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
     // written before it is read.
     if (cudaMemsetAsync(scratch, 0, kStaticHeaderBytes + ctr_bytes, s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    FfnLaunch f;
+    FfnLaunch f{};
     f.E = E;
     f.d = d;
     f.d_ff = d_ff;

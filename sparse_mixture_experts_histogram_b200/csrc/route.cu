@@ -445,7 +445,7 @@ cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    SmallRouteParams p;
+    SmallRouteParams p{};
     p.T = a.T;
     p.d = a.d;
     p.E = a.E;
@@ -497,7 +497,7 @@ cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
 
-    RouteParams p;
+    RouteParams p{};
     p.T = a.T;
     p.d = a.d;
     p.E = a.E;
