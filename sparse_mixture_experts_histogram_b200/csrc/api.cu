@@ -393,7 +393,10 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     c.x_perm = xperm;
     c.row_of_slot = row;
     c.err = err;
-    c.pdl = events == nullptr;
+    // Overlapping launches pay off for small layers; for large ones they only
+    // take SM slots early (measured: neutral to slightly negative).
+    const bool pdl = events == nullptr && S <= 4096;
+    c.pdl = pdl;
     if ((st = mark(events, 1, s)) != MOE_OK) return st;
     st = from_cuda(launch_scatter(c, s));
     if (st != MOE_OK) return st;
@@ -418,12 +421,11 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         f.Y = Y;
         f.h_ready = nullptr;
         f.err = err;
-        f.pdl = events == nullptr;
+        f.pdl = pdl;
         st = from_cuda(launch_ffn_small(f, ksplit, reinterpret_cast<int *>(wsb + 12), s));
     } else {
         st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
-                      reinterpret_cast<uint32_t *>(wsb + L.hready), err, s, events == nullptr,
-                      ksplit);
+                      reinterpret_cast<uint32_t *>(wsb + L.hready), err, s, pdl, ksplit);
     }
     if (st != MOE_OK) return st;
 
