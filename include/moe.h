@@ -85,6 +85,7 @@ typedef enum {
 #define MOE_DEVERR_TIMEOUT_EPI 0x4u  /* a wait for the epilogue ran out */
 #define MOE_DEVERR_OFFSETS 0x8u      /* offsets[] not non-decreasing within [0, S] */
 #define MOE_DEVERR_INDEX 0x10u       /* an expert index or row index out of range */
+#define MOE_DEVERR_LAYOUT 0x20u      /* a kernel found its shared memory misplaced and did nothing */
 
 /* Bytes of workspace every entry point below needs for these shapes
  * (the largest need over all of them).  0 if the shapes are unsupported. */

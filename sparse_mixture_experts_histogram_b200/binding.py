@@ -21,7 +21,7 @@ STATUS_NAMES = {
     4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE", 6: "MOE_ERR_TIMEOUT",
 }
 DEVERR_BITS = {0x1: "TIMEOUT_TMA", 0x2: "TIMEOUT_MMA", 0x4: "TIMEOUT_EPI", 0x8: "OFFSETS",
-               0x10: "INDEX"}
+               0x10: "INDEX", 0x20: "LAYOUT"}
 
 #: Every symbol the C header declares (checked against ``include/moe.h`` by the tests).
 ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "moe_permute",

@@ -24,10 +24,14 @@ constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, rank
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-    size_t tilectr, hready, hready_s;
+    size_t tilectr, hready, hready_s, gcnt;
     size_t zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
-    size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, xperm, H, Y, Hs, Ys, total;
+    size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, slotpos, perm, xperm, H, Y, Hs,
+        Ys, total;
 };
+
+// Token lists of the slot mode: one row of perm_stride entries per expert.
+int perm_stride(int T) { return (T + 15) / 16 * 16; }
 
 // Partial expert outputs the routed experts' kernel writes per row: the
 // narrow-layer kernel splits the hidden width, the general one may split the
@@ -52,6 +56,7 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     L.tilectr = take(ntiles * 4);
     L.hready = take(ffn_ready_counters(static_cast<int>(S), E, d_ff) * 4);
     L.hready_s = d_ffs > 0 ? take(ffn_ready_counters(T, 1, d_ffs) * 4) : 0;
+    L.gcnt = take(static_cast<size_t>(E) * 4);
     L.zero_bytes = o;
     L.tilecnt = take(ntiles * E * 4);
     L.tilebase = take(ntiles * E * 4);
@@ -61,6 +66,8 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     L.idx = take(S * 4);
     L.w = take(S * 4);
     L.row = take(S * 4);
+    L.slotpos = take(S * 4);
+    L.perm = take(static_cast<size_t>(E) * perm_stride(T) * 4);
     L.xperm = take(S * d * 2);
     L.H = take(S * d_ff * 2);
     L.Y = take(S * d * 4 * static_cast<size_t>(ffn_splits(static_cast<int>(S), E, d, d_ff)));
@@ -172,7 +179,8 @@ const char *moe_status_string(moe_status s)
 
 static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
                              const float *bias, int32_t *idx, float *w, int32_t *counts,
-                             int32_t *offsets, uint8_t *ws, const Layout &L, cudaStream_t s)
+                             int32_t *offsets, uint8_t *ws, const Layout &L, cudaStream_t s,
+                             bool slots = false)
 {
     RouteLaunch a{};
     a.T = T;
@@ -192,6 +200,12 @@ static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, cons
     a.done = reinterpret_cast<uint32_t *>(ws + 4);
     a.tile_ctr = reinterpret_cast<uint32_t *>(ws + L.tilectr);
     a.err = reinterpret_cast<uint32_t *>(ws);
+    if (slots) {
+        a.slot_pos = reinterpret_cast<int32_t *>(ws + L.slotpos);
+        a.perm = reinterpret_cast<int32_t *>(ws + L.perm);
+        a.gcnt = reinterpret_cast<int32_t *>(ws + L.gcnt);
+        a.perm_stride = perm_stride(T);
+    }
     return from_cuda(launch_route(a, s));
 }
 
@@ -376,35 +390,41 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
 
     st = from_cuda(cudaMemsetAsync(wsb, 0, L.zero_bytes, s));
     if (st != MOE_OK) return st;
-    if ((st = mark(events, 0, s)) != MOE_OK) return st;
-    st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
-                    reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s);
-    if (st != MOE_OK) return st;
-
-    ScatterLaunch c{};
-    c.T = T;
-    c.d = d;
-    c.E = E;
-    c.k = k;
-    c.x = x;
-    c.idx = idx;
-    c.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
-    c.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
-    c.x_perm = xperm;
-    c.row_of_slot = row;
-    c.err = err;
+    // Narrow layers run the slot mode: the router hands every expert its
+    // token list and the expert kernel gathers the rows of x itself, so there
+    // is no permuted copy of x and no scatter launch in between.
+    const bool narrow = ffn_small_supported(d);
     // Overlapping launches pay off for small layers; for large ones they only
     // take SM slots early (measured: neutral to slightly negative).
     const bool pdl = events == nullptr && S <= 4096;
-    c.pdl = pdl;
-    if ((st = mark(events, 1, s)) != MOE_OK) return st;
-    st = from_cuda(launch_scatter(c, s));
+    if ((st = mark(events, 0, s)) != MOE_OK) return st;
+    st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
+                    reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s, narrow);
     if (st != MOE_OK) return st;
+
+    if ((st = mark(events, 1, s)) != MOE_OK) return st;
+    if (!narrow) {
+        ScatterLaunch c{};
+        c.T = T;
+        c.d = d;
+        c.E = E;
+        c.k = k;
+        c.x = x;
+        c.idx = idx;
+        c.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
+        c.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
+        c.x_perm = xperm;
+        c.row_of_slot = row;
+        c.err = err;
+        c.pdl = pdl;
+        st = from_cuda(launch_scatter(c, s));
+        if (st != MOE_OK) return st;
+    }
 
     // A token never picks one expert twice, so no segment exceeds T rows.
     const int ksplit = ffn_splits(S, E, d, d_ff);
     if ((st = mark(events, 2, s)) != MOE_OK) return st;
-    if (ffn_small_supported(d)) {
+    if (narrow) {
         FfnLaunch f{};
         f.E = E;
         f.d = d;
@@ -416,12 +436,15 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         f.W1 = W1;
         f.W3 = W3;
         f.W2 = W2;
-        f.x = xperm;
+        f.x = x;
         f.H = nullptr;
         f.Y = Y;
         f.h_ready = nullptr;
         f.err = err;
         f.pdl = pdl;
+        f.perm = reinterpret_cast<const int32_t *>(wsb + L.perm);
+        f.perm_stride = perm_stride(T);
+        f.x_rows = T;
         st = from_cuda(launch_ffn_small(f, ksplit, reinterpret_cast<int *>(wsb + 12), s));
     } else {
         st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
@@ -446,9 +469,15 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     cb.d = d;
     cb.k = k;
     cb.ksplit = ksplit;
-    cb.ksplit_dev = ffn_small_supported(d) ? reinterpret_cast<const int *>(wsb + 12) : nullptr;
+    cb.ksplit_dev = narrow ? reinterpret_cast<const int *>(wsb + 12) : nullptr;
     cb.y = Y;
-    cb.row_of_slot = row;
+    if (narrow) {
+        cb.idx = idx;
+        cb.slot_pos = reinterpret_cast<const int32_t *>(wsb + L.slotpos);
+        cb.offsets = offsets;
+    } else {
+        cb.row_of_slot = row;
+    }
     cb.w = w;
     cb.shared_y = shared_y;
     cb.out = out;

@@ -27,6 +27,7 @@ struct CombineParams {
     size_t part_stride;  // float4 between consecutive partial outputs
     const float4 *y;
     const int32_t *row_of_slot;
+    const int32_t *idx, *slot_pos, *offsets;  // used when row_of_slot is null
     const float *w;
     const float4 *shared_y;
     float4 *out;
@@ -57,8 +58,15 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
     int my_row = -1;
     float my_w = 0.0f;
     if (lane < p.k) {
-        my_row = p.row_of_slot[static_cast<size_t>(t) * p.k + lane];
-        my_w = p.w[static_cast<size_t>(t) * p.k + lane];
+        const size_t sl = static_cast<size_t>(t) * p.k + lane;
+        if (p.row_of_slot) {
+            my_row = p.row_of_slot[sl];
+        } else {
+            const int e = p.idx[sl];
+            const int q = p.slot_pos[sl];
+            my_row = (e >= 0 && q >= 0) ? p.offsets[e] + q : -1;
+        }
+        my_w = p.w[sl];
         if (my_row >= p.T * p.k) my_row = -1;  // rows live in [0, T*k)
     }
     const int nv = p.d >> 2;
@@ -130,6 +138,9 @@ cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s)
     p.k = a.k;
     p.y = reinterpret_cast<const float4 *>(a.y);
     p.row_of_slot = a.row_of_slot;
+    p.idx = a.idx;
+    p.slot_pos = a.slot_pos;
+    p.offsets = a.offsets;
     p.w = a.w;
     p.shared_y = reinterpret_cast<const float4 *>(a.shared_y);
     p.out = reinterpret_cast<float4 *>(a.out);

@@ -16,6 +16,7 @@ constexpr uint32_t kErrTimeoutMma = 0x2u;
 constexpr uint32_t kErrTimeoutEpi = 0x4u;
 constexpr uint32_t kErrOffsets = 0x8u;
 constexpr uint32_t kErrIndex = 0x10u;
+constexpr uint32_t kErrLayout = 0x20u;
 
 constexpr int kTileTokens = 128;   // tokens per routing tile (= MMA M of the router)
 constexpr int kMaxK = 8;
@@ -200,6 +201,102 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
         const int n = o.ntiles * E;
         for (int i = row; i < n; i += kTileTokens) o.tilebase[i] += sm.tot[i % E];
         if (row == 0) *o.done = 0u;
+    }
+}
+
+// Slot assignment without a token order: every (token, slot) pair gets a
+// position inside its expert's segment from one global atomic per (CTA,
+// expert) plus its rank among the CTA's own pairs.  Positions are unique and
+// dense but their order inside a segment depends on scheduling; a row's
+// expert output does not depend on where the row sits, so the layer's result
+// is the same whatever order comes out.  The last CTA to finish turns the
+// per-expert totals into offsets and clears the totals for the next call.
+struct SlotOut {
+    int32_t *gcnt;     // [E] pairs per expert (zero before the launch, cleared again at the end)
+    int32_t *pos;      // [T, k] position of the pair inside its expert's segment (-1: none)
+    int32_t *perm;     // [E, perm_stride] token at each position of each expert
+    int32_t *offsets;  // [E+1] segment starts
+    int32_t *counts;   // [E] or nullptr
+    uint32_t *done;    // CTA completion counter (zero before the launch, cleared at the end)
+    int perm_stride;   // a multiple of 64, >= T
+    int nblocks;       // CTAs taking part
+};
+
+// Called by threads tid = 0..nthr-1 (a multiple of 32, >= 32) of a CTA whose
+// tokens t0 .. t0+ntok-1 chose ds.sel[r][j] (-1 = none); `bar_id` is a named
+// barrier over exactly those threads.
+__device__ __forceinline__ void assign_slots(DispatchSmem &ds, int t0, int ntok, int T, int E,
+                                             int k, const SlotOut &o, int tid, int nthr,
+                                             int bar_id)
+{
+    int32_t *hist = ds.cnt[0];
+    int32_t *base = ds.pre[0];
+    for (int e = tid; e < E; e += nthr) hist[e] = 0;
+    ptx::named_bar(bar_id, nthr);
+    const int npairs = ntok * k;
+    for (int i = tid; i < npairs; i += nthr) {
+        const int r = i / k;
+        const int j = i - r * k;
+        const int e = ds.sel[r][j];
+        ds.rnk[r][j] = e >= 0 ? atomicAdd(&hist[e], 1) : -1;
+    }
+    ptx::named_bar(bar_id, nthr);
+    for (int e = tid; e < E; e += nthr) {
+        const int c = hist[e];
+        base[e] = c ? atomicAdd(&o.gcnt[e], c) : 0;
+    }
+    ptx::named_bar(bar_id, nthr);
+    for (int i = tid; i < npairs; i += nthr) {
+        const int r = i / k;
+        const int j = i - r * k;
+        const int t = t0 + r;
+        if (t < T) {
+            const int e = ds.sel[r][j];
+            int p = -1;
+            if (e >= 0) {
+                p = base[e] + ds.rnk[r][j];
+                o.perm[static_cast<size_t>(e) * o.perm_stride + p] = t;
+            }
+            o.pos[static_cast<size_t>(t) * k + j] = p;
+        }
+    }
+    __threadfence();
+    ptx::named_bar(bar_id, nthr);
+    if (tid == 0) ds.is_last = (atomicAdd(o.done, 1u) == static_cast<uint32_t>(o.nblocks) - 1u);
+    ptx::named_bar(bar_id, nthr);
+    if (!ds.is_last) return;
+    __threadfence();
+    if (tid < 32) {
+        // Exclusive scan of the E <= 256 totals by one warp, then clear them.
+        const int lane = tid;
+        const int per = (E + 31) >> 5;
+        const int b0 = lane * per;
+        int c[kMaxE / 32];
+        int local = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxE / 32; ++i) {
+            c[i] = (i < per && b0 + i < E) ? __ldcg(&o.gcnt[b0 + i]) : 0;
+            local += c[i];
+        }
+        int incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        int run = incl - local;
+#pragma unroll
+        for (int i = 0; i < kMaxE / 32; ++i) {
+            const int e = b0 + i;
+            if (i < per && e < E) {
+                o.offsets[e] = run;
+                if (o.counts) o.counts[e] = c[i];
+                o.gcnt[e] = 0;
+                run += c[i];
+            }
+        }
+        if (lane == 31) o.offsets[E] = incl;
+        if (lane == 0) *o.done = 0u;
     }
 }
 

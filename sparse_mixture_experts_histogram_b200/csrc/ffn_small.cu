@@ -2,27 +2,32 @@
 // one persistent kernel with no dependency between CTAs.
 //
 // A work item is (expert e, token tile of BN rows, a range of 128-column
-// chunks of the hidden width).  For every chunk c of its range the CTA
+// chunks of the hidden width).  The item's BN rows of x (the tokens at
+// positions r0.. of e's token list) are gathered once into shared memory, in
+// the K-major 128-byte-swizzled layout the tensor cores read, and stay there
+// for the whole item.  For every chunk c of its range the CTA then runs
 //   up:    D0 = W1_e[c] X^T, D1 = W3_e[c] X^T        (tensor memory)
-//   H:     silu(D0) * D1 -> bf16 -> shared memory, already in the K-major
-//          128-byte-swizzled layout the tensor cores read as an operand
+//   H:     silu(D0) * D1 -> bf16 -> shared memory, in the same operand layout
 //   down:  Y += W2_e[:, c] H^T for every 128-row block of d (Y lives in
 //          tensor memory for the whole item)
 // and after its last chunk writes Y as one fp32 partial output
-// [split, S, d]; the combine sums the splits of a row in a fixed order.
-// Every weight byte is read once, H never leaves the SM, and a CTA waits only
-// on its own warps.  The MMA warp issues up(c+1) before down(c), so the
-// epilogue warps turn chunk c into H while the tensor cores already work on
-// chunk c+1 (two up accumulators, two H buffers).
+// [split, S, d], rows offsets[e] + position; the combine sums the splits of
+// a row in a fixed order.  Every weight byte is read once, x rows are read
+// once per item, H never leaves the SM, and a CTA waits only on its own
+// warps.  The MMA warp issues up(c+1) before down(c), so the epilogue warps
+// turn chunk c into H while the tensor cores already work on chunk c+1 (two
+// up accumulators, two H buffers).
 //
 // Tensor memory: 2 up accumulators of 2*BN columns + (d/128) Y blocks of BN
-// columns, at most 512.  Roles: warp 0 TMA producer, warp 1 MMA issuer,
-// warps 2..5 epilogue (one TMEM lane quarter each), as in gemm.cu.
+// columns, at most 512.  Roles: warp 0 TMA producer (weights only), warp 1
+// MMA issuer, warps 2..5 gather the item's x rows (16-byte cp.async) and run
+// the epilogues (one TMEM lane quarter each), as in gemm.cu.
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward) on each expert's own tokens
-// ("MoE" (theaiera.top) sec. 10.4); splitting the hidden width and summing
-// the partial down projections is the same sum over the hidden units.
+// ("MoE" (theaiera.top) sec. 10.4: index the tokens routed to the expert);
+// splitting the hidden width and summing the partial down projections is the
+// same sum over the hidden units.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -37,28 +42,40 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 6;
 constexpr uint32_t kWTile = 128 * 128;  // 128 weight rows x 64 bf16
 constexpr size_t kSmemBudget = 227 * 1024;
+constexpr int kMaxTile = 64;            // token rows per item, at most
 // barriers: full/empty [kMaxStages], ub_full/ub_empty/h_full/h_empty [2],
-// y_full, y_empty, drain
-constexpr size_t kFixedSmem = 1024 + (2 * kMaxStages + 11) * 8 + 16 + (2 * (kMaxE + 1) + 4) * 4 + 64;
+// y_full, y_empty, x_full, drain; then the TMEM address, the abort flag and
+// the segment tables.  No alignment slack: the dynamic shared memory window
+// starts on a 1024-byte boundary (the kernel checks it), which the 128-byte
+// swizzled operand tiles need; without the slack a d = 512 layer keeps four
+// weight stages next to its resident x rows.
+constexpr size_t kFixedSmem = (2 * kMaxStages + 12) * 8 + 16 + (2 * (kMaxE + 1) + 4) * 4;
 
-template <int BN, int ST, int MBD>
+template <int BN, int MBD>
 struct SmallCfg {
-    static constexpr uint32_t kStageBytes = 2 * kWTile + BN * 128u;
-    static constexpr uint32_t kHAtom = BN * 128u;        // BN rows x 64 bf16
+    static constexpr int KSU = 2 * MBD;                  // 64-column steps of d
+    static constexpr uint32_t kStageBytes = 2 * kWTile;  // two 128-row weight tiles
+    static constexpr uint32_t kXAtom = BN * 128u;        // BN rows x 64 bf16
+    static constexpr uint32_t kXBytes = KSU * kXAtom;    // the item's rows of x, all of d
+    static constexpr uint32_t kHAtom = BN * 128u;
     static constexpr uint32_t kHBytes = 2 * kHAtom;      // one H chunk: 128 hidden columns
     static constexpr int kUpCols = 2 * BN;               // D0 | D1
     static constexpr int kYCol0 = 2 * kUpCols;           // after two up accumulators
     static constexpr int kCols = kYCol0 + MBD * BN;      // MBD = d / 128 Y blocks
     static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128
                                         : kCols <= 256 ? 256 : 512;
-    static constexpr size_t kSmem = kFixedSmem + size_t(ST) * kStageBytes + 2 * kHBytes;
+    static constexpr size_t kRest = kFixedSmem + kXBytes + 2 * kHBytes;
+    static constexpr int kFit = static_cast<int>((kSmemBudget - kRest) / kStageBytes);
+    static constexpr int ST = kFit < kMaxStages ? kFit : kMaxStages;
+    static constexpr size_t kSmem = kRest + static_cast<size_t>(ST) * kStageBytes;
     static_assert(kCols <= 512, "tensor memory");
-    static_assert(kSmem <= kSmemBudget, "shared memory");
+    static_assert(kRest < kSmemBudget, "shared memory");
     static_assert(kSmem > kSmemBudget / 2, "one CTA per SM");
-    static_assert(ST >= 2 && ST <= kMaxStages, "pipeline depth");
+    static_assert(ST >= 3, "pipeline depth");
+    static_assert(BN <= kMaxTile && BN % 16 == 0, "token rows per item");
 };
 
 struct SmallParams {
@@ -68,6 +85,10 @@ struct SmallParams {
     int *nsplit_out;        // the count chosen (= partial outputs per row), for the combine
     size_t part_stride;     // floats between partial outputs
     const int32_t *offsets; // [E+1]
+    const int32_t *perm;    // [E, perm_stride] token at each position of each segment
+    int perm_stride;
+    const __nv_bfloat16 *x; // [x_rows, d]
+    int x_rows;
     float *Y;               // [nsplit, S, d]
     uint32_t *err;
 };
@@ -113,21 +134,36 @@ __device__ __forceinline__ void fence_proxy_async_shared()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int BN, int ST, int MBD>
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+template <int BN, int MBD>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_small_kernel(const __grid_constant__ CUtensorMap tmW1,
                      const __grid_constant__ CUtensorMap tmW3,
-                     const __grid_constant__ CUtensorMap tmW2,
-                     const __grid_constant__ CUtensorMap tmX, const SmallParams p)
+                     const __grid_constant__ CUtensorMap tmW2, const SmallParams p)
 {
-    using C = SmallCfg<BN, ST, MBD>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~static_cast<uintptr_t>(1023));
+    using C = SmallCfg<BN, MBD>;
+    constexpr int ST = C::ST;
+    constexpr int KSU = C::KSU;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (ptx::smem_addr(smem) & 1023u) {
+        // Nothing is set up yet; every thread leaves.
+        if (threadIdx.x == 0) atomicOr(p.err, kErrLayout);
+        return;
+    }
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    uint8_t *hbuf = smem + ST * C::kStageBytes;  // 2 H chunks, 1024-aligned
+    uint8_t *xbuf = smem + ST * C::kStageBytes;  // the item's x rows, KSU atoms
+    uint8_t *hbuf = xbuf + C::kXBytes;           // 2 H chunks
     uint64_t *full = reinterpret_cast<uint64_t *>(hbuf + 2 * C::kHBytes);
     uint64_t *empty = full + kMaxStages;
     uint64_t *ub_full = empty + kMaxStages;  // [2]
@@ -136,7 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *h_empty = h_full + 2;          // [2]
     uint64_t *y_full = h_empty + 2;
     uint64_t *y_empty = y_full + 1;
-    uint64_t *drain = y_empty + 1;
+    uint64_t *x_full = y_empty + 1;
+    uint64_t *drain = x_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     int32_t *s_off = reinterpret_cast<int32_t *>(tmem_slot + 4);
@@ -145,8 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int E = p.E;
     const int MBU = p.d_ff / 128;
-    const int KSU = p.d / 64;
-    const int NPAIR = (MBD + 1) / 2;
+    constexpr int NPAIR = (MBD + 1) / 2;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
@@ -161,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::mbar_init(y_full, 1);
         ptx::mbar_init(y_empty, 4);
+        ptx::mbar_init(x_full, 4);
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
         ptx::fence_barrier_init();
@@ -169,7 +206,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tensormap(&tmW1);
         ptx::prefetch_tensormap(&tmW3);
         ptx::prefetch_tensormap(&tmW2);
-        ptx::prefetch_tensormap(&tmX);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, C::kTmemCols);
@@ -192,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_off[e] = o0;
                 if (e == E - 1) s_off[E] = o1;
                 const int c = o1 - o0;
-                if (o0 < 0 || c < 0 || o1 > p.S) bad = true;
+                if (o0 < 0 || c < 0 || o1 > p.S || c > p.perm_stride) bad = true;
                 else nt += (c + BN - 1) / BN;
             }
         }
@@ -240,10 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < kMaxStages; ++s) last_parity[s] = 0;
             const uint64_t pol = ptx::policy_evict_normal();
             bool stop = false;
-            auto next_stage = [&](uint32_t bytes) -> uint8_t * {
+            auto next_stage = [&]() -> uint8_t * {
                 if (!bounded_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrTimeoutMma))
                     return nullptr;
-                ptx::mbar_arrive_expect_tx(&full[stage], bytes);
+                ptx::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
                 return smem + stage * C::kStageBytes;
             };
             auto advance = [&]() {
@@ -258,14 +294,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const Item it = decode_item<BN>(u, s_off, s_pre, E, nsplit, MBU);
                 const int nc = it.c_end - it.c_beg;
                 for (int j = 0; j <= nc && !stop; ++j) {
-                    if (j < nc) {  // up: W1, W3 rows of chunk c, token tile
+                    if (j < nc) {  // up: W1, W3 rows of chunk c
                         const int arow = it.e * p.d_ff + (it.c_beg + j) * 128;
                         for (int ks = 0; ks < KSU; ++ks) {
-                            uint8_t *sa = next_stage(C::kStageBytes);
+                            uint8_t *sa = next_stage();
                             if (!sa) { stop = true; break; }
                             ptx::tma_load_2d_hint(sa, &tmW1, &full[stage], ks * 64, arow, pol);
                             ptx::tma_load_2d_hint(sa + kWTile, &tmW3, &full[stage], ks * 64, arow, pol);
-                            ptx::tma_load_2d(sa + 2 * kWTile, &tmX, &full[stage], ks * 64, it.r0);
                             advance();
                         }
                     }
@@ -274,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int pr = 0; pr < NPAIR && !stop; ++pr) {
                             const int arow = it.e * p.d + pr * 256;
                             for (int kh = 0; kh < 2; ++kh) {
-                                uint8_t *sa = next_stage(2 * kWTile);
+                                uint8_t *sa = next_stage();
                                 if (!sa) { stop = true; break; }
                                 ptx::tma_load_2d_hint(sa, &tmW2, &full[stage], col + kh * 64, arow, pol);
                                 ptx::tma_load_2d_hint(sa + kWTile, &tmW2, &full[stage], col + kh * 64,
@@ -294,10 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t stage = 0, phase = 0;
             int n = 0, items = 0;
             bool stop = false;
+            const uint32_t sx = ptx::smem_addr(xbuf);
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
                 const Item it = decode_item<BN>(u, s_off, s_pre, E, nsplit, MBU);
                 const int nc = it.c_end - it.c_beg;
                 const uint32_t idesc = ptx::idesc_bf16_f32(128, ((it.valid + 15) >> 4) << 4);
+                if (!bounded_wait(x_full, static_cast<uint32_t>(items) & 1u, abort_flag, p.err,
+                                  kErrTimeoutEpi))
+                    break;
                 for (int j = 0; j <= nc && !stop; ++j) {
                     if (j < nc) {
                         const int ub = (n + j) & 1;
@@ -313,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             ptx::tc_fence_after();
                             const uint32_t sa = ptx::smem_addr(smem + stage * C::kStageBytes);
-                            const uint32_t sb = sa + 2 * kWTile;
+                            const uint32_t sb = sx + static_cast<uint32_t>(ks) * C::kXAtom;
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 const uint64_t bd = ptx::sw128_kmajor_desc(sb + kk * 32);
@@ -379,6 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (stop) break;
+                // Arrives when every MMA of the item is done: Y is complete and
+                // the x rows may be replaced by the next item's.
                 ptx::tc_commit(y_full);
                 n += nc;
                 ++items;
@@ -387,18 +428,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             drain_wait(drain, 0u);
         }
     } else {
-        // ---------------------------------------------------------------- epilogue
+        // ---------------------------------------------------------------- gather + epilogue
         const int q = warp & 3;
-        const int f = 32 * q + lane;  // hidden column of the chunk / row of a Y block
+        const int g = threadIdx.x - 64;  // 0..127
+        const int f = 32 * q + lane;     // hidden column of the chunk / row of a Y block
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         const uint32_t kk = static_cast<uint32_t>(f & 63);
         const uint32_t hcol_off = (f >> 6) * C::kHAtom + (kk & 7u) * 2u;
         const uint32_t hchunk = kk >> 3;
+        const uint32_t sx = ptx::smem_addr(xbuf);
+        // Gather share of this thread: 16-byte piece gc of rows gr, gr+16, ...
+        // of every 64-column atom.
+        const uint32_t gc = static_cast<uint32_t>(g & 7);
+        const int gr = g >> 3;
         int n = 0, items = 0;
         bool stop = false;
         for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
             const Item it = decode_item<BN>(u, s_off, s_pre, E, nsplit, MBU);
             const int nc = it.c_end - it.c_beg;
+            {
+                // x rows of the item's tokens; rows past the segment's end
+                // repeat its first token (their columns are never stored).
+                // The previous item's MMAs are all done (its y_full was seen).
+                const int32_t *pl = p.perm + static_cast<size_t>(it.e) * p.perm_stride +
+                                    (it.r0 - s_off[it.e]);
+                int tok[BN / 16];
+#pragma unroll
+                for (int m = 0; m < BN / 16; ++m) {
+                    const int r = gr + 16 * m;
+                    int t = __ldg(pl + (r < it.valid ? r : 0));
+                    if (static_cast<unsigned>(t) >= static_cast<unsigned>(p.x_rows)) {
+                        atomicOr(p.err, kErrIndex);
+                        t = 0;
+                    }
+                    tok[m] = t;
+                }
+#pragma unroll
+                for (int m = 0; m < BN / 16; ++m) {
+                    const int r = gr + 16 * m;
+                    const __nv_bfloat16 *src = p.x + static_cast<size_t>(tok[m]) * p.d + gc * 8;
+                    const uint32_t dst = sx + static_cast<uint32_t>(r) * 128u +
+                                         ((gc ^ (static_cast<uint32_t>(r) & 7u)) << 4);
+#pragma unroll
+                    for (int ks = 0; ks < KSU; ++ks)
+                        cp_async16(dst + static_cast<uint32_t>(ks) * C::kXAtom, src + ks * 64);
+                }
+                cp_async_wait_all();
+                fence_proxy_async_shared();  // x rows are read by the tensor cores (async proxy)
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(x_full);
+            }
             for (int j = 0; j < nc; ++j) {
                 const int ub = (n + j) & 1;
                 const uint32_t use = static_cast<uint32_t>((n + j) >> 1);
@@ -411,21 +490,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after();
                 const uint32_t tb = tmem + lane_base + static_cast<uint32_t>(ub * C::kUpCols);
                 uint8_t *hb = hbuf + ub * C::kHBytes + hcol_off;
-                for (int c0 = 0; c0 < it.valid; c0 += 32) {
-                    uint32_t a[32], b[32];
-                    ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), a);
-                    ptx::tmem_ld32(tb + static_cast<uint32_t>(BN + c0), b);
+                // Eight tokens per step: a short loop body keeps the code the
+                // epilogue runs small (it is cold at the start of every launch).
+#pragma unroll 1
+                for (int c0 = 0; c0 < it.valid; c0 += 8) {
+                    uint32_t a[8], b[8];
+                    ptx::tmem_ld8(tb + static_cast<uint32_t>(c0), a);
+                    ptx::tmem_ld8(tb + static_cast<uint32_t>(BN + c0), b);
                     ptx::tc_wait_ld();
+                    uint8_t *hrow = hb + c0 * 128;
 #pragma unroll
-                    for (int jt = 0; jt < 32; ++jt) {
-                        const int t = c0 + jt;
-                        if (t < it.valid) {
-                            const float g = __uint_as_float(a[jt]);
-                            const float h = g * __frcp_rn(1.0f + __expf(-g)) * __uint_as_float(b[jt]);
-                            // row t, column f of the chunk in the 128-byte-swizzled layout
-                            const uint32_t off = static_cast<uint32_t>(t) * 128u +
-                                                 ((hchunk ^ (static_cast<uint32_t>(t) & 7u)) << 4);
-                            *reinterpret_cast<__nv_bfloat16 *>(hb + off) = __float2bfloat16_rn(h);
+                    for (int jt = 0; jt < 8; ++jt) {
+                        if (c0 + jt < it.valid) {
+                            const float gv = __uint_as_float(a[jt]);
+                            const float h = __fdividef(gv * __uint_as_float(b[jt]), 1.0f + __expf(-gv));
+                            // row c0+jt (c0 is a multiple of 8, so the row's swizzle
+                            // phase is jt), column f, 128-byte-swizzled layout
+                            *reinterpret_cast<__nv_bfloat16 *>(hrow + jt * 128 + ((hchunk ^ jt) << 4)) =
+                                __float2bfloat16_rn(h);
                         }
                     }
                 }
@@ -446,17 +528,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_after();
             float *Y = p.Y + it.sp * p.part_stride;
+#pragma unroll 1
             for (int m = 0; m < MBD; ++m) {
                 const uint32_t yb = tmem + lane_base + static_cast<uint32_t>(C::kYCol0 + m * BN);
-                const int col = m * 128 + f;
-                for (int c0 = 0; c0 < it.valid; c0 += 32) {
-                    uint32_t y[32];
-                    ptx::tmem_ld32(yb + static_cast<uint32_t>(c0), y);
+                float *yc = Y + static_cast<size_t>(it.r0) * p.d + m * 128 + f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < it.valid; c0 += 8) {
+                    uint32_t y[8];
+                    ptx::tmem_ld8(yb + static_cast<uint32_t>(c0), y);
                     ptx::tc_wait_ld();
 #pragma unroll
-                    for (int jt = 0; jt < 32; ++jt)
+                    for (int jt = 0; jt < 8; ++jt)
                         if (c0 + jt < it.valid)
-                            Y[static_cast<size_t>(it.r0 + c0 + jt) * p.d + col] = __uint_as_float(y[jt]);
+                            yc[static_cast<size_t>(c0 + jt) * p.d] = __uint_as_float(y[jt]);
                 }
             }
             ptx::tc_fence_before();
@@ -475,18 +559,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, int ST, int MBD>
+template <int BN, int MBD>
 cudaError_t launch_small_cfg(const FfnLaunch &a, int nsplit_max, int *nsplit_out, cudaStream_t s)
 {
-    using C = SmallCfg<BN, ST, MBD>;
-    CUtensorMap tW1, tW3, tW2, tX;
+    using C = SmallCfg<BN, MBD>;
+    if (a.perm == nullptr || a.x_rows < 1) return cudaErrorInvalidValue;
+    CUtensorMap tW1, tW3, tW2;
     cudaError_t e = make_tmap_bf16(&tW1, a.W1, static_cast<uint64_t>(a.E) * a.d_ff, a.d, 128);
     if (e == cudaSuccess) e = make_tmap_bf16(&tW3, a.W3, static_cast<uint64_t>(a.E) * a.d_ff, a.d, 128);
     if (e == cudaSuccess) e = make_tmap_bf16(&tW2, a.W2, static_cast<uint64_t>(a.E) * a.d, a.d_ff, 128);
-    if (e == cudaSuccess) e = make_tmap_bf16(&tX, a.x, a.S, a.d, BN);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ffn_small_kernel<BN, ST, MBD>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::kSmem));
+    e = cudaFuncSetAttribute(ffn_small_kernel<BN, MBD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return e;
     SmallParams p{};
     p.E = a.E;
@@ -498,22 +582,25 @@ cudaError_t launch_small_cfg(const FfnLaunch &a, int nsplit_max, int *nsplit_out
     p.nsplit_out = nsplit_out;
     p.part_stride = static_cast<size_t>(a.S) * a.d;
     p.offsets = a.offsets;
+    p.perm = a.perm;
+    p.perm_stride = a.perm_stride;
+    p.x = reinterpret_cast<const __nv_bfloat16 *>(a.x);
+    p.x_rows = a.x_rows;
     p.Y = a.Y;
     p.err = a.err;
     const long long items = ((static_cast<long long>(a.S) + BN - 1) / BN + a.E) * nsplit_max;
     long long grid = device_sm_count();
     if (items < grid) grid = items;
     if (grid < 1) grid = 1;
-    return launch_pdl(ffn_small_kernel<BN, ST, MBD>, dim3(static_cast<unsigned>(grid)),
-                      dim3(kThreads), C::kSmem, s, a.pdl, tW1, tW3, tW2, tX, p);
+    return launch_pdl(ffn_small_kernel<BN, MBD>, dim3(static_cast<unsigned>(grid)),
+                      dim3(kThreads), C::kSmem, s, a.pdl, tW1, tW3, tW2, p);
 }
 
 template <int MBD>
 cudaError_t launch_small_d(const FfnLaunch &a, int nsplit_max, int *nsplit_out, cudaStream_t s)
 {
     constexpr int kBN = (4 + MBD) * 64 <= 512 ? 64 : 32;
-    constexpr int kST = kBN == 64 ? 4 : 5;
-    return launch_small_cfg<kBN, kST, MBD>(a, nsplit_max, nsplit_out, s);
+    return launch_small_cfg<kBN, MBD>(a, nsplit_max, nsplit_out, s);
 }
 
 }  // namespace

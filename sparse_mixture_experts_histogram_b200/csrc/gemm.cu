@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                     for (int j = 0; j < 32; ++j) {
                         if (c0 + j < w.valid) {
                             const float g = __uint_as_float(a[j]);
-                            const float h = g * __frcp_rn(1.0f + __expf(-g)) * __uint_as_float(b[j]);
+                            const float h = __fdividef(g * __uint_as_float(b[j]), 1.0f + __expf(-g));
                             p.H[static_cast<size_t>(w.r0 + c0 + j) * p.d_ff + f] =
                                 __float2bfloat16_rn(h);
                         }

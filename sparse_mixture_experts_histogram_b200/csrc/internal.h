@@ -22,6 +22,13 @@ struct RouteLaunch {
     uint32_t *done;      // counter, zero before the launch
     uint32_t *tile_ctr;  // [ntiles] counters, zero before the launch
     uint32_t *err;       // device error word
+    // Slot mode (slot_pos set): instead of the token-ordered tile histogram,
+    // positions from atomics (common.cuh assign_slots) and the token list of
+    // every expert; tilecnt, tilebase, rank and tile_ctr are not used.
+    int32_t *slot_pos;   // [T,k]
+    int32_t *perm;       // [E, perm_stride]
+    int32_t *gcnt;       // [E] zero before the launch (left zero)
+    int perm_stride;
 };
 
 struct RanksLaunch {
@@ -57,6 +64,12 @@ struct FfnLaunch {
     uint32_t *h_ready;        // ffn_ready_counters(S, E, d_ff) counters, zero before the launch
     uint32_t *err;
     bool pdl;                 // launched right after another kernel of this library
+    // Narrow kernel only: when set, the rows of segment e are gathered from x
+    // ([x_rows, d]) through the token list perm[e * perm_stride + position]
+    // instead of being read from a permuted copy.
+    const int32_t *perm;
+    int perm_stride;
+    int x_rows;
 };
 
 struct CombineLaunch {
@@ -65,6 +78,8 @@ struct CombineLaunch {
     const int *ksplit_dev; // or read from device memory (written by the expert kernel), if set
     const float *y;        // [ksplit, T*k, d]
     const int32_t *row_of_slot;
+    // or, when row_of_slot is null: row of (t, j) = offsets[idx[t,j]] + slot_pos[t,j]
+    const int32_t *idx, *slot_pos, *offsets;
     const float *w;
     const float *shared_y;
     float *out;

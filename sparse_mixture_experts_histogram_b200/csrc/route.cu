@@ -36,6 +36,8 @@ struct RouteParams {
     float *w;
     uint32_t *err;
     DispatchOut dout;
+    int slots;      // slot mode: assign_slots instead of dispatch_tile
+    SlotOut sout;
 };
 
 __host__ __device__ constexpr uint32_t route_stage_bytes(int Npad)
@@ -45,6 +47,19 @@ __host__ __device__ constexpr uint32_t route_stage_bytes(int Npad)
 
 constexpr size_t kRouteFixedSmem = 1024 /* alignment slack */ + 2 * kRouteMaxStages * 8 + 8 + 16 +
                                    kMaxE * sizeof(float) + sizeof(DispatchSmem) + 64;
+
+void fill_slots(const RouteLaunch &a, int blocks, int *slots, SlotOut *o)
+{
+    *slots = a.slot_pos != nullptr ? 1 : 0;
+    o->gcnt = a.gcnt;
+    o->pos = a.slot_pos;
+    o->perm = a.perm;
+    o->offsets = a.offsets;
+    o->counts = a.counts;
+    o->done = a.done;
+    o->perm_stride = a.perm_stride;
+    o->nblocks = blocks;
+}
 
 template <int K>
 __device__ __forceinline__ void topk_insert(float (&tv)[K], int (&ti)[K], float v, int e)
@@ -228,7 +243,11 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         }
 #pragma unroll
         for (int j = 0; j < K; ++j) ds.sel[row][j] = valid ? ti[j] : -1;
-        dispatch_tile(ds, row, tile, p.T, p.E, K, p.dout, 1);
+        if (p.slots)
+            assign_slots(ds, tile * kTileTokens, kTileTokens, p.T, p.E, K, p.sout, row,
+                         kTileTokens, 1);
+        else
+            dispatch_tile(ds, row, tile, p.T, p.E, K, p.dout, 1);
     }
 
     __syncthreads();
@@ -261,6 +280,8 @@ struct SmallRouteParams {
     float *w;
     uint32_t *tile_ctr;
     DispatchOut dout;
+    int slots;      // slot mode: assign_slots instead of the per-tile dispatch
+    SlotOut sout;
 };
 
 // 8 bf16 (one 16-byte vector) to fp32, in element order.
@@ -413,8 +434,14 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
             for (int j = 0; j < K; ++j) {
                 p.idx[static_cast<size_t>(t) * K + j] = ti[j];
                 p.w[static_cast<size_t>(t) * K + j] = ex[j] / s;
+                ds.sel[warp][j] = ti[j];
             }
         }
+    }
+    if (p.slots) {
+        __syncthreads();
+        assign_slots(ds, t0, nt, p.T, p.E, K, p.sout, threadIdx.x, kSmallThreads, 1);
+        return;
     }
 
     // The last CTA of each 128-token tile groups that tile's pairs by expert.
@@ -463,6 +490,7 @@ cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
     p.dout.done = a.done;
     p.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
     const int blocks = (a.T + kSmallTok - 1) / kSmallTok;
+    fill_slots(a, blocks, &p.slots, &p.sout);
     route_small_kernel<K, EPW, U><<<blocks, kSmallThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -516,6 +544,7 @@ cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
     p.dout.counts = a.counts;
     p.dout.done = a.done;
     p.dout.ntiles = p.ntiles;
+    fill_slots(a, p.ntiles, &p.slots, &p.sout);
     route_kernel<K><<<p.ntiles, kRouteThreads, smem, s>>>(tmX, tmWg, p);
     return cudaGetLastError();
 }

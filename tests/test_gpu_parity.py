@@ -155,6 +155,9 @@ FFN_SEGMENTS = [
     ("one_big", 256, 256, [700]),
     ("tiny", 128, 128, [1, 2, 3]),
     ("wide_ff", 384, 1024, [40, 0, 200, 5]),
+    # a few hundred rows per segment: 256-row token tiles with ragged spills
+    ("tile256", 256, 256, [300, 257, 511, 0, 256, 200, 12]),
+    ("tile256_wide", 1152, 384, [520, 256, 255, 1]),
 ]
 
 
