@@ -496,11 +496,15 @@ cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
 }
 
 // Few experts: one expert per warp and eight loads in flight per lane; many
-// experts: four experts per warp and four loads each.
+// experts: four (eight for narrow rows) experts per warp.
 template <int K>
 cudaError_t launch_route_small_k(const RouteLaunch &a, cudaStream_t s)
 {
     if (a.E <= 16) return launch_route_small_cfg<K, 1, 8>(a, s);
+    // Narrow rows (d <= 512: 64 vectors, two loads per lane cover a row):
+    // eight experts per warp, so a pass covers 64 experts with all of its
+    // loads in flight at once.
+    if (a.d <= 512) return launch_route_small_cfg<K, 8, 2>(a, s);
     return launch_route_small_cfg<K, 4, 4>(a, s);
 }
 
