@@ -402,6 +402,8 @@ def gpu_arm(args):
                 t = ev[j].elapsed_time(ev[j + 1])
                 if name.startswith("shared") and not wl.d_ff_shared:
                     continue
+                if name == "scatter" and wl.d <= 1024:
+                    continue  # no scatter launch: the expert kernel gathers x itself
                 dur[name].append(t)
                 per_layer[i][name].append(t)
                 if name == "expert_ffn":
@@ -475,7 +477,8 @@ def gpu_arm(args):
     d2h = sum(w.T * w.d * 4 for w in wls)
     ok = all(torch.isfinite(o).all().item() for o in outs)
 
-    launches_per_layer = [4 + (1 if w.d_ff_shared else 0) for w in wls]
+    # router, [scatter: only layers with d > 1024], expert FFN, [shared FFN], combine
+    launches_per_layer = [(3 if w.d <= 1024 else 4) + (1 if w.d_ff_shared else 0) for w in wls]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,

@@ -150,7 +150,12 @@ MOE_API moe_status moe_combine(int T, int d, int k, const float *y_perm, const i
 /* The whole layer: route, dispatch, experts and combine in one call.
  * out [T,d] fp32 out.  Equivalent to moe_route + moe_permute +
  * moe_expert_ffn + moe_combine, without leaving the GPU and without any
- * host synchronisation (the call can be captured in a CUDA graph). */
+ * host synchronisation (the call can be captured in a CUDA graph).  For
+ * d <= 1024 the dispatch inside the call does not build a permuted copy of x:
+ * the router gives every expert its token list and the expert kernel reads
+ * the rows of x through it; the rows of an expert are then not in token
+ * order inside the workspace, which does not change out (each row's expert
+ * output does not depend on its position; slots are summed in order). */
 MOE_API moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
                        const moe_bf16 *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
                        const moe_bf16 *W2, float *out, void *ws, size_t ws_bytes,
