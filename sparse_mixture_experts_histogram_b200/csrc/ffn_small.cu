@@ -20,8 +20,10 @@
 //
 // Tensor memory: 2 up accumulators of 2*BN columns + (d/128) Y blocks of BN
 // columns, at most 512.  Roles: warp 0 TMA producer (weights only), warp 1
-// MMA issuer, warps 2..5 gather the item's x rows (16-byte cp.async) and run
-// the epilogues (one TMEM lane quarter each), as in gemm.cu.
+// MMA issuer, warps 2..9 gather the item's x rows (16-byte cp.async) and run
+// the epilogues, two warps per TMEM lane quarter taking alternate 8-token
+// steps, so that the epilogue the tensor cores wait for after an item's last
+// chunk, and the partial-output write, take half as long.
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward) on each expert's own tokens
@@ -41,7 +43,8 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                      // two per tensor-memory lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxStages = 6;
 constexpr uint32_t kWTile = 128 * 128;  // 128 weight rows x 64 bf16
 constexpr size_t kSmemBudget = 227 * 1024;
@@ -75,7 +78,7 @@ struct SmallCfg {
     static_assert(kRest < kSmemBudget, "shared memory");
     static_assert(kSmem > kSmemBudget / 2, "one CTA per SM");
     static_assert(ST >= 3, "pipeline depth");
-    static_assert(BN <= kMaxTile && BN % 16 == 0, "token rows per item");
+    static_assert(BN <= kMaxTile && BN % 32 == 0, "token rows per item");
 };
 
 struct SmallParams {
@@ -191,13 +194,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&ub_full[b], 1);
-            ptx::mbar_init(&ub_empty[b], 4);
-            ptx::mbar_init(&h_full[b], 4);
+            ptx::mbar_init(&ub_empty[b], kEpiWarps);
+            ptx::mbar_init(&h_full[b], kEpiWarps);
             ptx::mbar_init(&h_empty[b], 1);
         }
         ptx::mbar_init(y_full, 1);
-        ptx::mbar_init(y_empty, 4);
-        ptx::mbar_init(x_full, 4);
+        ptx::mbar_init(y_empty, kEpiWarps);
+        ptx::mbar_init(x_full, kEpiWarps);
         ptx::mbar_init(drain, 1);
         *abort_flag = 0u;
         ptx::fence_barrier_init();
@@ -429,18 +432,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- gather + epilogue
+        // Warps 2..9: lane quarter q = warp % 4 of tensor memory; the two
+        // warps of a quarter take alternate eight-token steps (half).
         const int q = warp & 3;
-        const int g = threadIdx.x - 64;  // 0..127
+        const int half = (warp - 2) >> 2;
+        const int g = threadIdx.x - 64;  // 0..255
         const int f = 32 * q + lane;     // hidden column of the chunk / row of a Y block
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         const uint32_t kk = static_cast<uint32_t>(f & 63);
         const uint32_t hcol_off = (f >> 6) * C::kHAtom + (kk & 7u) * 2u;
         const uint32_t hchunk = kk >> 3;
         const uint32_t sx = ptx::smem_addr(xbuf);
-        // Gather share of this thread: 16-byte piece gc of rows gr, gr+16, ...
+        // Gather share of this thread: 16-byte piece gc of rows gr, gr+32, ...
         // of every 64-column atom.
         const uint32_t gc = static_cast<uint32_t>(g & 7);
-        const int gr = g >> 3;
+        const int gr = g >> 3;  // 0..31
         int n = 0, items = 0;
         bool stop = false;
         for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
@@ -452,10 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // The previous item's MMAs are all done (its y_full was seen).
                 const int32_t *pl = p.perm + static_cast<size_t>(it.e) * p.perm_stride +
                                     (it.r0 - s_off[it.e]);
-                int tok[BN / 16];
+                int tok[BN / 32];
 #pragma unroll
-                for (int m = 0; m < BN / 16; ++m) {
-                    const int r = gr + 16 * m;
+                for (int m = 0; m < BN / 32; ++m) {
+                    const int r = gr + 32 * m;
                     int t = __ldg(pl + (r < it.valid ? r : 0));
                     if (static_cast<unsigned>(t) >= static_cast<unsigned>(p.x_rows)) {
                         atomicOr(p.err, kErrIndex);
@@ -464,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tok[m] = t;
                 }
 #pragma unroll
-                for (int m = 0; m < BN / 16; ++m) {
-                    const int r = gr + 16 * m;
+                for (int m = 0; m < BN / 32; ++m) {
+                    const int r = gr + 32 * m;
                     const __nv_bfloat16 *src = p.x + static_cast<size_t>(tok[m]) * p.d + gc * 8;
                     const uint32_t dst = sx + static_cast<uint32_t>(r) * 128u +
                                          ((gc ^ (static_cast<uint32_t>(r) & 7u)) << 4);
@@ -493,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Eight tokens per step: a short loop body keeps the code the
                 // epilogue runs small (it is cold at the start of every launch).
 #pragma unroll 1
-                for (int c0 = 0; c0 < it.valid; c0 += 8) {
+                for (int c0 = 8 * half; c0 < it.valid; c0 += 16) {
                     uint32_t a[8], b[8];
                     ptx::tmem_ld8(tb + static_cast<uint32_t>(c0), a);
                     ptx::tmem_ld8(tb + static_cast<uint32_t>(BN + c0), b);
@@ -533,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t yb = tmem + lane_base + static_cast<uint32_t>(C::kYCol0 + m * BN);
                 float *yc = Y + static_cast<size_t>(it.r0) * p.d + m * 128 + f;
 #pragma unroll 1
-                for (int c0 = 0; c0 < it.valid; c0 += 8) {
+                for (int c0 = 8 * half; c0 < it.valid; c0 += 16) {
                     uint32_t y[8];
                     ptx::tmem_ld8(yb + static_cast<uint32_t>(c0), y);
                     ptx::tc_wait_ld();
