@@ -20,10 +20,10 @@
 //
 // Tensor memory: 2 up accumulators of 2*BN columns + (d/128) Y blocks of BN
 // columns, at most 512.  Roles: warp 0 TMA producer (weights only), warp 1
-// MMA issuer, warps 2..9 gather the item's x rows (16-byte cp.async) and run
-// the epilogues, two warps per TMEM lane quarter taking alternate 8-token
+// MMA issuer, warps 2..17 gather the item's x rows (16-byte cp.async) and
+// run the epilogues, four warps per TMEM lane quarter taking turns at 8-token
 // steps, so that the epilogue the tensor cores wait for after an item's last
-// chunk, and the partial-output write, take half as long.
+// chunk, and the partial-output write, are short.
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward) on each expert's own tokens
@@ -43,7 +43,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kEpiWarps = 8;                      // two per tensor-memory lane quarter
+constexpr int kEpiWarps = 16;                     // four per tensor-memory lane quarter
+constexpr int kEpiPer = kEpiWarps / 4;            // warps per lane quarter
+constexpr int kGatherRows = 4 * kEpiWarps;        // rows one gather pass covers
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxStages = 6;
 constexpr uint32_t kWTile = 128 * 128;  // 128 weight rows x 64 bf16
@@ -432,10 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- gather + epilogue
-        // Warps 2..9: lane quarter q = warp % 4 of tensor memory; the two
-        // warps of a quarter take alternate eight-token steps (half).
+        // Warps 2..17: lane quarter q = warp % 4 of tensor memory; the
+        // kEpiPer warps of a quarter take turns at eight-token steps.
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
+        const int half = (warp - 2) >> 2;  // 0 .. kEpiPer-1
         const int g = threadIdx.x - 64;  // 0..255
         const int f = 32 * q + lane;     // hidden column of the chunk / row of a Y block
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
@@ -458,10 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // The previous item's MMAs are all done (its y_full was seen).
                 const int32_t *pl = p.perm + static_cast<size_t>(it.e) * p.perm_stride +
                                     (it.r0 - s_off[it.e]);
-                int tok[BN / 32];
+                constexpr int kPasses = (BN + kGatherRows - 1) / kGatherRows;
+                int tok[kPasses];
 #pragma unroll
-                for (int m = 0; m < BN / 32; ++m) {
-                    const int r = gr + 32 * m;
+                for (int m = 0; m < kPasses; ++m) {
+                    const int r = gr + kGatherRows * m;
                     int t = __ldg(pl + (r < it.valid ? r : 0));
                     if (static_cast<unsigned>(t) >= static_cast<unsigned>(p.x_rows)) {
                         atomicOr(p.err, kErrIndex);
@@ -470,8 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tok[m] = t;
                 }
 #pragma unroll
-                for (int m = 0; m < BN / 32; ++m) {
-                    const int r = gr + 32 * m;
+                for (int m = 0; m < kPasses; ++m) {
+                    const int r = gr + kGatherRows * m;
+                    if (r >= BN) break;
                     const __nv_bfloat16 *src = p.x + static_cast<size_t>(tok[m]) * p.d + gc * 8;
                     const uint32_t dst = sx + static_cast<uint32_t>(r) * 128u +
                                          ((gc ^ (static_cast<uint32_t>(r) & 7u)) << 4);
@@ -499,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Eight tokens per step: a short loop body keeps the code the
                 // epilogue runs small (it is cold at the start of every launch).
 #pragma unroll 1
-                for (int c0 = 8 * half; c0 < it.valid; c0 += 16) {
+                for (int c0 = 8 * half; c0 < it.valid; c0 += 8 * kEpiPer) {
                     uint32_t a[8], b[8];
                     ptx::tmem_ld8(tb + static_cast<uint32_t>(c0), a);
                     ptx::tmem_ld8(tb + static_cast<uint32_t>(BN + c0), b);
@@ -539,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t yb = tmem + lane_base + static_cast<uint32_t>(C::kYCol0 + m * BN);
                 float *yc = Y + static_cast<size_t>(it.r0) * p.d + m * 128 + f;
 #pragma unroll 1
-                for (int c0 = 8 * half; c0 < it.valid; c0 += 16) {
+                for (int c0 = 8 * half; c0 < it.valid; c0 += 8 * kEpiPer) {
                     uint32_t y[8];
                     ptx::tmem_ld8(yb + static_cast<uint32_t>(c0), y);
                     ptx::tc_wait_ld();
