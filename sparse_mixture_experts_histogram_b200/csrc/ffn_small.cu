@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Warps 2..17: lane quarter q = warp % 4 of tensor memory; the
         // kEpiPer warps of a quarter take turns at eight-token steps.
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;  // 0 .. kEpiPer-1
+        const int turn = (warp - 2) >> 2;  // 0 .. kEpiPer-1
         const int g = threadIdx.x - 64;  // 0..255
         const int f = 32 * q + lane;     // hidden column of the chunk / row of a Y block
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
@@ -503,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Eight tokens per step: a short loop body keeps the code the
                 // epilogue runs small (it is cold at the start of every launch).
 #pragma unroll 1
-                for (int c0 = 8 * half; c0 < it.valid; c0 += 8 * kEpiPer) {
+                for (int c0 = 8 * turn; c0 < it.valid; c0 += 8 * kEpiPer) {
                     uint32_t a[8], b[8];
                     ptx::tmem_ld8(tb + static_cast<uint32_t>(c0), a);
                     ptx::tmem_ld8(tb + static_cast<uint32_t>(BN + c0), b);
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t yb = tmem + lane_base + static_cast<uint32_t>(C::kYCol0 + m * BN);
                 float *yc = Y + static_cast<size_t>(it.r0) * p.d + m * 128 + f;
 #pragma unroll 1
-                for (int c0 = 8 * half; c0 < it.valid; c0 += 8 * kEpiPer) {
+                for (int c0 = 8 * turn; c0 < it.valid; c0 += 8 * kEpiPer) {
                     uint32_t y[8];
                     ptx::tmem_ld8(yb + static_cast<uint32_t>(c0), y);
                     ptx::tc_wait_ld();
