@@ -325,7 +325,13 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
 
     // Warp w computes experts w*EPW .. w*EPW+EPW-1, then the next 8*EPW
     // experts; each lane keeps U*EPW 16-byte loads of Wg in flight.
+    // Every CTA reads all of Wg; starting each CTA at a different group of
+    // experts spreads the simultaneous reads over the L2 slices instead of
+    // sending all CTAs to the same rows at once.  (Only when E is a multiple
+    // of EPW, so that a rotated group never wraps.)
+    const int rot = (p.E % EPW == 0) ? static_cast<int>((blockIdx.x * EPW) % p.E) : 0;
     for (int e0 = warp * EPW; e0 < p.E; e0 += (kSmallThreads / 32) * EPW) {
+        const int eb = e0 + rot < p.E ? e0 + rot : e0 + rot - p.E;  // first expert of the group
         float acc[EPW][kSmallTok];
 #pragma unroll
         for (int q = 0; q < EPW; ++q)
@@ -339,7 +345,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
 #pragma unroll
                 for (int q = 0; q < EPW; ++q)
                     wv[u][q] = (v < nv && e0 + q < p.E)
-                                   ? __ldg(p.Wg + static_cast<size_t>(e0 + q) * nv + v)
+                                   ? __ldg(p.Wg + static_cast<size_t>(eb + q) * nv + v)
                                    : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
@@ -374,8 +380,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
         if (lane == 0) {
 #pragma unroll
             for (int q = 0; q < EPW; ++q) {
-                const int e = e0 + q;
-                if (e < p.E) {
+                const int e = eb + q;
+                if (e0 + q < p.E) {
                     const float b = p.bias ? p.bias[e] : 0.0f;
 #pragma unroll
                     for (int tt = 0; tt < kSmallTok; ++tt) slog[tt * kMaxE + e] = acc[q][tt] + b;
