@@ -391,8 +391,9 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     st = from_cuda(cudaMemsetAsync(wsb, 0, L.zero_bytes, s));
     if (st != MOE_OK) return st;
     // Narrow layers run the slot mode: the router hands every expert its
-    // token list and the expert kernel gathers the rows of x itself, so there
-    // is no permuted copy of x and no scatter launch in between.
+    // token list and its total, and the expert kernel derives the segment
+    // starts and gathers the rows of x itself, so there is no permuted copy
+    // of x and no scatter launch in between.
     const bool narrow = ffn_small_supported(d);
     // Overlapping launches pay off for small layers; for large ones they only
     // take SM slots early (measured: neutral to slightly negative).
@@ -445,6 +446,8 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         f.perm = reinterpret_cast<const int32_t *>(wsb + L.perm);
         f.perm_stride = perm_stride(T);
         f.x_rows = T;
+        f.counts = reinterpret_cast<const int32_t *>(wsb + L.gcnt);
+        f.offsets_out = offsets;
         st = from_cuda(launch_ffn_small(f, ksplit, reinterpret_cast<int *>(wsb + 12), s));
     } else {
         st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,

@@ -209,21 +209,18 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
 // expert) plus its rank among the CTA's own pairs.  Positions are unique and
 // dense but their order inside a segment depends on scheduling; a row's
 // expert output does not depend on where the row sits, so the layer's result
-// is the same whatever order comes out.  The last CTA to finish turns the
-// per-expert totals into offsets and clears the totals for the next call.
+// is the same whatever order comes out.  When the grid has finished, gcnt
+// holds every expert's total; the expert kernel turns the totals into
+// segment starts itself, so no CTA of the router waits for the others.
 struct SlotOut {
-    int32_t *gcnt;     // [E] pairs per expert (zero before the launch, cleared again at the end)
+    int32_t *gcnt;     // [E] pairs per expert (zero before the launch)
     int32_t *pos;      // [T, k] position of the pair inside its expert's segment (-1: none)
     int32_t *perm;     // [E, perm_stride] token at each position of each expert
-    int32_t *offsets;  // [E+1] segment starts
-    int32_t *counts;   // [E] or nullptr
-    uint32_t *done;    // CTA completion counter (zero before the launch, cleared at the end)
-    int perm_stride;   // a multiple of 64, >= T
-    int nblocks;       // CTAs taking part
+    int perm_stride;   // >= T
 };
 
-// Called by threads tid = 0..nthr-1 (a multiple of 32, >= 32) of a CTA whose
-// tokens t0 .. t0+ntok-1 chose ds.sel[r][j] (-1 = none); `bar_id` is a named
+// Called by threads tid = 0..nthr-1 (a multiple of 32) of a CTA whose tokens
+// t0 .. t0+ntok-1 chose ds.sel[r][j] (-1 = none); `bar_id` is a named
 // barrier over exactly those threads.
 __device__ __forceinline__ void assign_slots(DispatchSmem &ds, int t0, int ntok, int T, int E,
                                              int k, const SlotOut &o, int tid, int nthr,
@@ -259,44 +256,6 @@ __device__ __forceinline__ void assign_slots(DispatchSmem &ds, int t0, int ntok,
             }
             o.pos[static_cast<size_t>(t) * k + j] = p;
         }
-    }
-    __threadfence();
-    ptx::named_bar(bar_id, nthr);
-    if (tid == 0) ds.is_last = (atomicAdd(o.done, 1u) == static_cast<uint32_t>(o.nblocks) - 1u);
-    ptx::named_bar(bar_id, nthr);
-    if (!ds.is_last) return;
-    __threadfence();
-    if (tid < 32) {
-        // Exclusive scan of the E <= 256 totals by one warp, then clear them.
-        const int lane = tid;
-        const int per = (E + 31) >> 5;
-        const int b0 = lane * per;
-        int c[kMaxE / 32];
-        int local = 0;
-#pragma unroll
-        for (int i = 0; i < kMaxE / 32; ++i) {
-            c[i] = (i < per && b0 + i < E) ? __ldcg(&o.gcnt[b0 + i]) : 0;
-            local += c[i];
-        }
-        int incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
-        int run = incl - local;
-#pragma unroll
-        for (int i = 0; i < kMaxE / 32; ++i) {
-            const int e = b0 + i;
-            if (i < per && e < E) {
-                o.offsets[e] = run;
-                if (o.counts) o.counts[e] = c[i];
-                o.gcnt[e] = 0;
-                run += c[i];
-            }
-        }
-        if (lane == 31) o.offsets[E] = incl;
-        if (lane == 0) *o.done = 0u;
     }
 }
 

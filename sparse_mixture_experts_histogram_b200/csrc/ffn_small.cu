@@ -89,7 +89,8 @@ struct SmallParams {
     int sms;                // SMs the work should cover in one wave
     int *nsplit_out;        // the count chosen (= partial outputs per row), for the combine
     size_t part_stride;     // floats between partial outputs
-    const int32_t *offsets; // [E+1]
+    const int32_t *counts;  // [E] rows of every segment (the router's totals)
+    int32_t *offsets_out;   // [E+1] segment starts, written by CTA 0 for the combine
     const int32_t *perm;    // [E, perm_stride] token at each position of each segment
     int perm_stride;
     const __nv_bfloat16 *x; // [x_rows, d]
@@ -218,30 +219,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::grid_dep_wait();
     if (warp == 2) {
-        // Token tiles per expert from the offsets, then the number of chunk
-        // ranges per tile: as many as fit one wave of items on the SMs (the
-        // same choice in every CTA, since all read the same offsets).
+        // Segment starts are the exclusive prefix of the router's per-expert
+        // totals (CTA 0 writes them out for the combine).  Then token tiles
+        // per expert and the number of chunk ranges per tile: as many as fit
+        // one wave of items on the SMs (the same choice in every CTA, since
+        // all read the same totals).
         const int per = (E + 31) >> 5;
         const int base = lane * per;
         bool bad = false;
-        int nt = 0;
-        for (int i = 0; i < per; ++i) {
+        int cnt[kMaxE / 32];
+        int rows = 0, nt = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxE / 32; ++i) {
             const int e = base + i;
-            if (e < E) {
-                const int o0 = p.offsets[e];
-                const int o1 = p.offsets[e + 1];
-                s_off[e] = o0;
-                if (e == E - 1) s_off[E] = o1;
-                const int c = o1 - o0;
-                if (o0 < 0 || c < 0 || o1 > p.S || c > p.perm_stride) bad = true;
-                else nt += (c + BN - 1) / BN;
+            int c = 0;
+            if (i < per && e < E) {
+                c = p.counts[e];
+                if (c < 0 || c > p.perm_stride) {
+                    bad = true;
+                    c = 0;
+                }
             }
+            cnt[i] = c;
+            rows += c;
+            nt += (c + BN - 1) / BN;
         }
+        int incl_rows = rows;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl_rows, off);
+            if (lane >= off) incl_rows += v;
+        }
+        if (__shfl_sync(0xffffffffu, incl_rows, 31) > p.S) bad = true;
         bad = __any_sync(0xffffffffu, bad);
         if (bad) {
             nt = 0;
             if (lane == 0) atomicOr(p.err, kErrOffsets);
         }
+        int o = incl_rows - rows;
+#pragma unroll
+        for (int i = 0; i < kMaxE / 32; ++i) {
+            const int e = base + i;
+            if (i < per && e < E) {
+                const int oe = bad ? 0 : o;
+                s_off[e] = oe;
+                if (blockIdx.x == 0) p.offsets_out[e] = oe;
+                o += cnt[i];
+            }
+        }
+        if (lane == 31) {
+            const int end = bad ? 0 : incl_rows;
+            s_off[E] = end;
+            if (blockIdx.x == 0) p.offsets_out[E] = end;
+        }
+        __syncwarp();
         int incl = nt;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -573,7 +604,8 @@ template <int BN, int MBD>
 cudaError_t launch_small_cfg(const FfnLaunch &a, int nsplit_max, int *nsplit_out, cudaStream_t s)
 {
     using C = SmallCfg<BN, MBD>;
-    if (a.perm == nullptr || a.x_rows < 1) return cudaErrorInvalidValue;
+    if (a.perm == nullptr || a.counts == nullptr || a.offsets_out == nullptr || a.x_rows < 1)
+        return cudaErrorInvalidValue;
     CUtensorMap tW1, tW3, tW2;
     cudaError_t e = make_tmap_bf16(&tW1, a.W1, static_cast<uint64_t>(a.E) * a.d_ff, a.d, 128);
     if (e == cudaSuccess) e = make_tmap_bf16(&tW3, a.W3, static_cast<uint64_t>(a.E) * a.d_ff, a.d, 128);
@@ -591,7 +623,8 @@ cudaError_t launch_small_cfg(const FfnLaunch &a, int nsplit_max, int *nsplit_out
     p.sms = device_sm_count();
     p.nsplit_out = nsplit_out;
     p.part_stride = static_cast<size_t>(a.S) * a.d;
-    p.offsets = a.offsets;
+    p.counts = a.counts;
+    p.offsets_out = a.offsets_out;
     p.perm = a.perm;
     p.perm_stride = a.perm_stride;
     p.x = reinterpret_cast<const __nv_bfloat16 *>(a.x);

@@ -23,8 +23,9 @@ struct RouteLaunch {
     uint32_t *tile_ctr;  // [ntiles] counters, zero before the launch
     uint32_t *err;       // device error word
     // Slot mode (slot_pos set): instead of the token-ordered tile histogram,
-    // positions from atomics (common.cuh assign_slots) and the token list of
-    // every expert; tilecnt, tilebase, rank and tile_ctr are not used.
+    // positions from atomics (common.cuh assign_slots), the token list of
+    // every expert and the per-expert totals in gcnt; offsets, counts,
+    // tilecnt, tilebase, rank, done and tile_ctr are not written.
     int32_t *slot_pos;   // [T,k]
     int32_t *perm;       // [E, perm_stride]
     int32_t *gcnt;       // [E] zero before the launch (left zero)
@@ -70,6 +71,8 @@ struct FfnLaunch {
     const int32_t *perm;
     int perm_stride;
     int x_rows;
+    const int32_t *counts;    // [E] rows per segment (the router's totals); offsets are
+    int32_t *offsets_out;     // their exclusive prefix, written here [E+1]
 };
 
 struct CombineLaunch {

@@ -48,17 +48,13 @@ __host__ __device__ constexpr uint32_t route_stage_bytes(int Npad)
 constexpr size_t kRouteFixedSmem = 1024 /* alignment slack */ + 2 * kRouteMaxStages * 8 + 8 + 16 +
                                    kMaxE * sizeof(float) + sizeof(DispatchSmem) + 64;
 
-void fill_slots(const RouteLaunch &a, int blocks, int *slots, SlotOut *o)
+void fill_slots(const RouteLaunch &a, int *slots, SlotOut *o)
 {
     *slots = a.slot_pos != nullptr ? 1 : 0;
     o->gcnt = a.gcnt;
     o->pos = a.slot_pos;
     o->perm = a.perm;
-    o->offsets = a.offsets;
-    o->counts = a.counts;
-    o->done = a.done;
     o->perm_stride = a.perm_stride;
-    o->nblocks = blocks;
 }
 
 template <int K>
@@ -496,7 +492,7 @@ cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
     p.dout.done = a.done;
     p.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
     const int blocks = (a.T + kSmallTok - 1) / kSmallTok;
-    fill_slots(a, blocks, &p.slots, &p.sout);
+    fill_slots(a, &p.slots, &p.sout);
     route_small_kernel<K, EPW, U><<<blocks, kSmallThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -554,7 +550,7 @@ cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
     p.dout.counts = a.counts;
     p.dout.done = a.done;
     p.dout.ntiles = p.ntiles;
-    fill_slots(a, p.ntiles, &p.slots, &p.sout);
+    fill_slots(a, &p.slots, &p.sout);
     route_kernel<K><<<p.ntiles, kRouteThreads, smem, s>>>(tmX, tmWg, p);
     return cudaGetLastError();
 }
