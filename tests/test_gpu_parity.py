@@ -264,6 +264,21 @@ def test_forward_is_deterministic_and_graph_capturable():
     assert torch.equal(out, a)
 
 
+@pytest.mark.parametrize("wl", [synth.sweep()[-1], Workload("E64_k4_T1000", 1000, 384, 64, 256, 4)],
+                         ids=lambda w: w.name)
+def test_forward_narrow_repeatable_whatever_the_slot_order(wl):
+    # Narrow layers place each expert's rows in the order the router's
+    # atomics hand out positions, which differs from run to run; the output
+    # must not (each row's expert output is independent of its position and
+    # slots are summed in order).
+    inp = _inputs(wl)
+    ws = workspace(wl)
+    first = gpu_forward(wl, inp, ws).clone()
+    for _ in range(4):
+        assert torch.equal(gpu_forward(wl, inp, ws), first)
+    check_forward(wl, inp)
+
+
 @pytest.mark.parametrize("T", [1, 8, 32, 128])
 def test_forward_mixtral_decode(T):
     wl = synth.mixtral_decode(T)
