@@ -292,6 +292,9 @@ def gpu_arm(args):
     ws_bytes = max(moe.moe_workspace_size_ex(w.T, w.d, w.E, w.d_ff, w.k, w.d_ff_shared)
                    for w in wls)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    # The inputs were drawn on the default stream; everything below runs on
+    # its own stream, so wait for them first.
+    torch.cuda.synchronize(dev)
     stream = torch.cuda.Stream(device=dev)
 
     # ---- routing pre-pass: experts each batch hits (for the algorithmic bytes)

@@ -389,11 +389,17 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
 
     if (warp < nt) {
         const int t = t0 + warp;
+        // A NaN logit (only from non-finite inputs) ranks like -inf, and
+        // every round takes the largest remaining value with the lower index
+        // on ties, so each slot gets a distinct expert in [0, E) whatever
+        // the values are (k <= E).
         float v[kMaxE / 32];
+        uint32_t taken = 0u;  // bit i: expert lane + 32*i already selected
 #pragma unroll
         for (int i = 0; i < kMaxE / 32; ++i) {
             const int e = lane + 32 * i;
-            v[i] = (e < p.E) ? slog[warp * kMaxE + e] : -CUDART_INF_F;
+            const float l = (e < p.E) ? slog[warp * kMaxE + e] : -CUDART_INF_F;
+            v[i] = (l == l) ? l : -CUDART_INF_F;
         }
         float tv[K];
         int ti[K];
@@ -404,7 +410,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
 #pragma unroll
             for (int i = 0; i < kMaxE / 32; ++i) {
                 const int e = lane + 32 * i;
-                if (e < p.E && v[i] > bv) {  // strict: equal values keep the lower index
+                // e ascends with i: equal values keep the lower index
+                if (e < p.E && !(taken & (1u << i)) && (v[i] > bv || be == 0x7fffffff)) {
                     bv = v[i];
                     be = e;
                 }
@@ -422,7 +429,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
             ti[j] = be;
 #pragma unroll
             for (int i = 0; i < kMaxE / 32; ++i)
-                if (lane + 32 * i == be) v[i] = -CUDART_INF_F;
+                if (lane + 32 * i == be) taken |= 1u << i;
         }
         if (lane == 0) {
             float ex[K];
@@ -463,6 +470,9 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
 #pragma unroll
     for (int j = 0; j < K; ++j)
         ds.sel[row][j] = (t < p.T) ? __ldcg(&p.idx[static_cast<size_t>(t) * K + j]) : -1;
+#pragma unroll
+    for (int j = 0; j < K; ++j)  // the selection above always yields [0, E); keep dispatch in bounds regardless
+        if (static_cast<unsigned>(ds.sel[row][j]) >= static_cast<unsigned>(p.E)) ds.sel[row][j] = -1;
     dispatch_tile(ds, row, tile, p.T, p.E, K, p.dout, 1);
 }
 

@@ -9,8 +9,8 @@ import sparse_mixture_experts_histogram_b200 as moe
 from sparse_mixture_experts_histogram_b200 import synth
 from sparse_mixture_experts_histogram_b200.synth import Workload, bits
 
-from gpu_util import (assert_close, check_forward, check_routing, gpu_forward, sample_tokens,
-                      workspace)
+from gpu_util import (assert_close, check_forward, check_routing, gpu_forward, gpu_route,
+                      sample_tokens, workspace)
 
 pytestmark = pytest.mark.gpu
 
@@ -250,6 +250,7 @@ def test_forward_is_deterministic_and_graph_capturable():
     assert torch.equal(a, b)
     out = torch.empty_like(a)
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         moe.moe_forward(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["W1"],
                         inp["W3"], inp["W2"], out, ws, stream=s)
@@ -277,6 +278,30 @@ def test_forward_narrow_repeatable_whatever_the_slot_order(wl):
     for _ in range(4):
         assert torch.equal(gpu_forward(wl, inp, ws), first)
     check_forward(wl, inp)
+
+
+@pytest.mark.parametrize("wl", [Workload("nonfinite_narrow", 64, 256, 8, 256, 2),
+                                Workload("nonfinite_wide", 40, 1152, 8, 256, 3)],
+                         ids=lambda w: w.name)
+def test_nonfinite_rows_route_in_bounds(wl):
+    # Inputs are finite by construction everywhere else; a NaN or Inf row must
+    # still give every slot of its token a distinct expert in [0, E) (NaN ranks
+    # like -inf, ties go to the lower index), raise no device error, and leave
+    # the other tokens' outputs as they were.
+    inp = _inputs(wl, seed=5)
+    bad = inp["x"].clone()
+    bad[3] = float("nan")
+    bad[17] = float("inf")
+    inp_bad = dict(inp, x=bad)
+    idx, _, counts = gpu_route(wl, inp_bad)
+    assert idx.min() >= 0 and idx.max() < wl.E
+    assert all(len(set(r)) == wl.k for r in idx.tolist())
+    assert counts.sum() == wl.T * wl.k
+    assert idx[3].tolist() == list(range(wl.k))  # every logit NaN: all tied, lowest indices win
+    out_bad = gpu_forward(wl, inp_bad).cpu().numpy()
+    out = gpu_forward(wl, inp).cpu().numpy()
+    keep = [t for t in range(wl.T) if t not in (3, 17)]
+    assert_close(out_bad[keep], out[keep], "finite tokens next to non-finite ones")
 
 
 @pytest.mark.parametrize("T", [1, 8, 32, 128])
