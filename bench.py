@@ -440,7 +440,13 @@ def gpu_arm(args):
     roof["frac"] = roof["achieved"] / roof["peak"]
     tr = traffic_record(f"expert_ffn:{args.workload}")
     roof["traffic"] = None if tr is None else tr["bytes_per_launch"]
-    roof["kernel"] = "ffn_kernel (grouped W1|W3 + SwiGLU, then W2, one persistent launch)"
+    kinds = []
+    if any(w.d <= 1024 for w in wls):
+        kinds.append("ffn_small_kernel (d <= 1024: x rows gathered through the experts' token "
+                     "lists, W1|W3 + SwiGLU and W2 per hidden chunk, one persistent launch)")
+    if any(w.d > 1024 for w in wls):
+        kinds.append("ffn_kernel (grouped W1|W3 + SwiGLU, then W2, one persistent launch)")
+    roof["kernel"] = "; ".join(kinds)
     roof["algorithmic_bytes_per_launch"] = sum(up_bytes) / len(up_bytes)
     roof["flops_per_launch"] = sum(up_flops) / len(up_flops)
     roof["launch_ms"] = sum(up_time) / len(up_time)
