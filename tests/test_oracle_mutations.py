@@ -29,6 +29,14 @@ MUTANTS = {
                               "for (int i = 0; i < d; ++i) o[i] += 0.0 * y[i];"),
     "unnormalised_weights": ("for (int j = 0; j < k; ++j) w[j] /= s;\n}",
                              "for (int j = 0; j < k; ++j) w[j] /= 1.0;\n}"),
+    "gap_from_top1": ("*gap = l[sel[k - 1]] - l[next];", "*gap = l[sel[0]] - l[next];"),
+    "gap_next_is_smallest": ("if (!taken[e] && (next < 0 || l[e] > l[next])) next = e;",
+                             "if (!taken[e] && (next < 0 || l[e] < l[next])) next = e;"),
+    "gap_skips_a_place": ("*gap = l[sel[k - 1]] - l[next];",
+                          "*gap = (k > 1 ? l[sel[k - 2]] : l[sel[k - 1]]) - l[next];"),
+    "logits_without_bias": ("if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);",
+                            "if (logits) { memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);"
+                            " if (bias) for (int e = 0; e < E; ++e) logits[(size_t)t * E + e] -= bias[e]; }"),
 }
 
 

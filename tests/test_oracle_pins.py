@@ -281,3 +281,40 @@ def test_expert_call_statistics_plausible():
     assert int(r["counts"].sum()) == p["calls"]
     assert int((r["counts"] > 0).sum()) >= p["experts_hit"] - 4
     assert r["counts"].min() >= 5 and r["counts"].max() <= 80
+
+
+@pytest.mark.parametrize("case", ["k1", "k2", "kE-1"])
+@pytest.mark.parametrize("ties", [False, True])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_logits_and_gap_match_library_formulation(case, ties, with_bias):
+    # The oracle's `logits` output is the router's linear layer x Wg^T
+    # (+ bias) -- here a torch fp64 matmul, a library routine that shares no
+    # code with the oracle -- and its `gap` is the k-th largest minus the
+    # (k+1)-th largest logit of the token, taken here from a numpy sort.  The
+    # gap decides which tokens count as near ties (their selected set may
+    # differ between two correct implementations), so a gap measured from the
+    # wrong pair of logits would silently change which tokens are checked.
+    E = 9
+    k = {"k1": 1, "k2": 2, "kE-1": E - 1}[case]
+    wl, inp = _inputs(T=120, d=40, E=E, dff=8, k=k, seed=13)
+    Wg = inp["Wg"].clone()
+    if ties:
+        Wg[5] = Wg[2]     # bit-identical logits for experts 2, 5 and 7
+        Wg[7] = Wg[2]
+    bias = np.linspace(-0.4, 0.6, E) if with_bias else None
+    if ties and with_bias:
+        bias[5] = bias[7] = bias[2]
+    r = oracle.route(bits(inp["x"]), bits(Wg), k=k, bias=bias)
+    L = (_f64(inp["x"]) @ _f64(Wg).T).numpy()
+    if with_bias:
+        L = L + bias[None, :]
+    assert np.max(np.abs(r["logits"] - L)) <= 1e-12 * np.max(np.abs(L))
+    Ls = -np.sort(-L, axis=1)
+    gap = Ls[:, k - 1] - Ls[:, k]
+    assert np.max(np.abs(r["gap"] - gap)) <= 1e-12 * np.max(np.abs(L))
+    if ties:
+        # wherever the k-th and (k+1)-th places go to two of the twins, the
+        # gap is exactly zero
+        twin = np.isin(np.argsort(-L, axis=1, kind="stable")[:, k - 1:k + 1], [2, 5, 7]).all(1)
+        assert twin.any()
+        assert (r["gap"][twin] == 0).all()
