@@ -5,7 +5,13 @@ of the benchmark are the only callers.  The product path never imports this
 package, and this package imports nothing from the product.
 """
 from .oracle import (  # noqa: F401
+    ACT_SIGMOID,
+    ACT_SILU,
+    W_SIGMOID,
+    W_SOFTMAX_ALL,
+    W_SOFTMAX_TOPK,
     build,
+    capacity_limit,
     num_threads,
     route,
     forward,

@@ -97,10 +97,16 @@ static void route_one(int d, int E, int k, const double *xt, const uint16_t *Wg,
     for (int j = 0; j < k; ++j) w[j] /= s;
 }
 
-/* One SwiGLU expert on one token: y = W2 (silu(W1 x) * (W3 x)).
- * W1, W3 are [dff, d] and W2 is [d, dff], row-major (nn.Linear's [out, in]). */
-static void swiglu_one(int d, int dff, const uint16_t *W1, const uint16_t *W3,
-                       const uint16_t *W2, const double *xt, double *h, double *y)
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/* One gated expert on one token: y = W2 (act(W1 x) * (W3 x)) with
+ * act = silu (act_mode 0, SwiGLU) or act = the logistic sigmoid (act_mode 1:
+ * the "万亿 MoE" forward listing's h = a * sigmoid(g), whose gate g is the
+ * W1 half and whose linear half a is the W3 half of its concatenated
+ * up-projection).  W1, W3 are [dff, d] and W2 is [d, dff], row-major
+ * (nn.Linear's [out, in]). */
+static void expert_one(int d, int dff, const uint16_t *W1, const uint16_t *W3,
+                       const uint16_t *W2, const double *xt, double *h, double *y, int act_mode)
 {
     for (int f = 0; f < dff; ++f) {
         const uint16_t *r1 = W1 + (size_t)f * d;
@@ -108,13 +114,44 @@ static void swiglu_one(int d, int dff, const uint16_t *W1, const uint16_t *W3,
         double a = 0.0, b = 0.0;
         for (int i = 0; i < d; ++i) a += bf16_bits_to_double(r1[i]) * xt[i];
         for (int i = 0; i < d; ++i) b += bf16_bits_to_double(r3[i]) * xt[i];
-        h[f] = silu(a) * b;
+        if (act_mode == 1) h[f] = sigmoid(a) * b;
+        else h[f] = silu(a) * b;
     }
     for (int o = 0; o < d; ++o) {
         const uint16_t *r2 = W2 + (size_t)o * dff;
         double acc = 0.0;
         for (int f = 0; f < dff; ++f) acc += bf16_bits_to_double(r2[f]) * h[f];
         y[o] = acc;
+    }
+}
+
+/* The method's expert: SwiGLU. */
+static void swiglu_one(int d, int dff, const uint16_t *W1, const uint16_t *W3,
+                       const uint16_t *W2, const double *xt, double *h, double *y)
+{
+    expert_one(d, dff, W1, W3, W2, xt, h, y, 0);
+}
+
+/* Gate weights of the selected experts sel[0..k) for the routing variants
+ * (w_mode 0, the softmax over the selected logits, is computed by route_one
+ * or the forced-set code):
+ *   w_mode 1: softmax over all E logits; the selected experts keep their
+ *             probabilities, not renormalised ("Mixtral 8x7B模型架构解析"
+ *             (bjdmk.com.cn), Router.forward: softmax, then top-k of the
+ *             probabilities)
+ *   w_mode 2: the logistic sigmoid of each selected logit ("万亿 MoE"
+ *             (m.xxqk.cn) forward listing: w = 1 / (1 + exp(-logit))) */
+static void variant_weights(int E, int k, const double *l, const int32_t *sel, int w_mode,
+                            double *w)
+{
+    if (w_mode == 1) {
+        double m = l[0], s = 0.0;
+        for (int e = 1; e < E; ++e)
+            if (l[e] > m) m = l[e];
+        for (int e = 0; e < E; ++e) s += exp(l[e] - m);
+        for (int j = 0; j < k; ++j) w[j] = exp(l[sel[j]] - m) / s;
+    } else if (w_mode == 2) {
+        for (int j = 0; j < k; ++j) w[j] = sigmoid(l[sel[j]]);
     }
 }
 
@@ -133,10 +170,25 @@ int oracle_num_threads(void)
  *   idx [T,k] int32, w [T,k], gap [T] (may be NULL), logits [T,E] (may be
  *   NULL), counts [E] (may be NULL): number of (token, slot) pairs per expert.
  * Returns 0, or -1 on bad arguments. */
+int oracle_route_v(int T, int d, int E, int k, const uint16_t *x, const uint16_t *Wg,
+                   const double *bias, int w_mode, int32_t *idx, double *w, double *gap,
+                   double *logits, int64_t *counts);
+
 int oracle_route(int T, int d, int E, int k, const uint16_t *x, const uint16_t *Wg,
                  const double *bias, int32_t *idx, double *w, double *gap,
                  double *logits, int64_t *counts)
 {
+    return oracle_route_v(T, d, E, k, x, Wg, bias, 0, idx, w, gap, logits, counts);
+}
+
+/* oracle_route with the gate weights of routing variant w_mode (0, 1, 2 as
+ * in variant_weights; the selected set and the gap do not depend on it:
+ * the softmax over all logits and the sigmoid keep the logits' order). */
+int oracle_route_v(int T, int d, int E, int k, const uint16_t *x, const uint16_t *Wg,
+                   const double *bias, int w_mode, int32_t *idx, double *w, double *gap,
+                   double *logits, int64_t *counts)
+{
+    if (w_mode < 0 || w_mode > 2) return -1;
     if (T < 0 || d < 1 || E < 1 || k < 1 || k > E || !x || !Wg || !idx || !w) return -1;
     int err = 0;
 #pragma omp parallel
@@ -153,6 +205,8 @@ int oracle_route(int T, int d, int E, int k, const uint16_t *x, const uint16_t *
                 for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)t * d + i]);
                 route_one(d, E, k, xt, Wg, bias, l, idx + (size_t)t * k, w + (size_t)t * k,
                           gap ? gap + t : NULL, taken);
+                if (w_mode)
+                    variant_weights(E, k, l, idx + (size_t)t * k, w_mode, w + (size_t)t * k);
                 if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);
             }
         }
@@ -180,21 +234,85 @@ int oracle_route(int T, int d, int E, int k, const uint16_t *x, const uint16_t *
  *   (used where the k-th and (k+1)-th logits nearly tie).
  *   out [n,d] double.
  * Returns 0, or -1 on bad arguments. */
+int oracle_forward_v(int n, const int32_t *tokens, int T, int d, int E, int dff, int k,
+                     const uint16_t *x, const uint16_t *Wg, const double *bias,
+                     const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
+                     int dffs, const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
+                     const int32_t *forced, int w_mode, int act_mode, long long cap,
+                     const int32_t *route_all, double *out);
+
 int oracle_forward(int n, const int32_t *tokens, int T, int d, int E, int dff, int k,
                    const uint16_t *x, const uint16_t *Wg, const double *bias,
                    const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
                    int dffs, const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
                    const int32_t *forced, double *out)
 {
+    return oracle_forward_v(n, tokens, T, d, E, dff, k, x, Wg, bias, W1, W3, W2, dffs, Ws1, Ws3,
+                            Ws2, forced, 0, 0, -1, NULL, out);
+}
+
+/* oracle_forward for the variants the pages describe besides the method:
+ *   w_mode, act_mode: gate weights and expert activation (variant_weights,
+ *     expert_one); with forced experts the weights are those of the forced
+ *     set under the same rule
+ *   cap >= 0: expert capacity ("Mistral 8x7B SMoE" (jsqmd.com) sec. 2.4,
+ *     capacity factor): of the (token, slot) pairs routed to an expert only
+ *     the first cap in token order are computed, the others add nothing to
+ *     their token's output (the other slots keep their weights).  The ranks
+ *     need the routing of all T tokens: route_all [T,k] (e.g. a routing with
+ *     forced near ties), or NULL for the oracle's own top-k.  cap < 0:
+ *     dropless. */
+int oracle_forward_v(int n, const int32_t *tokens, int T, int d, int E, int dff, int k,
+                     const uint16_t *x, const uint16_t *Wg, const double *bias,
+                     const uint16_t *W1, const uint16_t *W3, const uint16_t *W2,
+                     int dffs, const uint16_t *Ws1, const uint16_t *Ws3, const uint16_t *Ws2,
+                     const int32_t *forced, int w_mode, int act_mode, long long cap,
+                     const int32_t *route_all, double *out)
+{
     if (n < 0 || T < 1 || d < 1 || E < 1 || dff < 1 || k < 1 || k > E) return -1;
     if (!x || !Wg || !W1 || !W3 || !W2 || !out) return -1;
     if (dffs < 0 || (dffs > 0 && (!Ws1 || !Ws3 || !Ws2))) return -1;
+    if (w_mode < 0 || w_mode > 2 || act_mode < 0 || act_mode > 1) return -1;
     for (int r = 0; r < n; ++r) {
         int t = tokens ? tokens[r] : r;
         if (t < 0 || t >= T) return -1;
         if (forced)
             for (int j = 0; j < k; ++j)
                 if (forced[(size_t)r * k + j] < 0 || forced[(size_t)r * k + j] >= E) return -1;
+    }
+    /* Capacity: which (token, slot) pairs are kept. */
+    unsigned char *keep = NULL;
+    if (cap >= 0) {
+        int32_t *sel_all = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * k);
+        double *w_all = (double *)malloc(sizeof(double) * (size_t)T * k);
+        int64_t *cnt = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+        keep = (unsigned char *)malloc((size_t)T * k);
+        int bad = !sel_all || !w_all || !cnt || !keep;
+        if (!bad) {
+            if (route_all) {
+                for (size_t s = 0; s < (size_t)T * k; ++s) {
+                    if (route_all[s] < 0 || route_all[s] >= E) bad = 1;
+                    sel_all[s] = route_all[s];
+                }
+            } else if (oracle_route(T, d, E, k, x, Wg, bias, sel_all, w_all, NULL, NULL, NULL)) {
+                bad = 1;
+            }
+        }
+        if (!bad) {
+            for (int t = 0; t < T; ++t)
+                for (int j = 0; j < k; ++j) {
+                    int e = sel_all[(size_t)t * k + j];
+                    keep[(size_t)t * k + j] = cnt[e] < cap;
+                    cnt[e] += 1;
+                }
+        }
+        free(sel_all);
+        free(w_all);
+        free(cnt);
+        if (bad) {
+            free(keep);
+            return -1;
+        }
     }
     int hmax = dff > dffs ? dff : dffs;
     int err = 0;
@@ -229,16 +347,18 @@ int oracle_forward(int n, const int32_t *tokens, int T, int d, int E, int dff, i
                     }
                     for (int j = 0; j < k; ++j) w[j] /= s;
                 }
+                if (w_mode) variant_weights(E, k, l, sel, w_mode, w);
                 double *o = out + (size_t)r * d;
                 for (int i = 0; i < d; ++i) o[i] = 0.0;
                 for (int j = 0; j < k; ++j) {
+                    if (keep && !keep[(size_t)t * k + j]) continue;
                     int e = sel[j];
-                    swiglu_one(d, dff, W1 + (size_t)e * dff * d, W3 + (size_t)e * dff * d,
-                               W2 + (size_t)e * d * dff, xt, h, y);
+                    expert_one(d, dff, W1 + (size_t)e * dff * d, W3 + (size_t)e * dff * d,
+                               W2 + (size_t)e * d * dff, xt, h, y, act_mode);
                     for (int i = 0; i < d; ++i) o[i] += w[j] * y[i];
                 }
                 if (dffs > 0) {
-                    swiglu_one(d, dffs, Ws1, Ws3, Ws2, xt, h, y);
+                    expert_one(d, dffs, Ws1, Ws3, Ws2, xt, h, y, act_mode);
                     for (int i = 0; i < d; ++i) o[i] += y[i];
                 }
             }
@@ -251,6 +371,7 @@ int oracle_forward(int n, const int32_t *tokens, int T, int d, int E, int dff, i
         free(sel);
         free(taken);
     }
+    free(keep);
     return err ? -1 : 0;
 }
 

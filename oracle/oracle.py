@@ -8,6 +8,7 @@ outputs are float64 / int32 numpy arrays.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -46,6 +47,11 @@ def _load():
         lib.oracle_num_threads.restype = _I
         lib.oracle_route.restype = _I
         lib.oracle_route.argtypes = [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]
+        lib.oracle_route_v.restype = _I
+        lib.oracle_route_v.argtypes = [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P]
+        lib.oracle_forward_v.restype = _I
+        lib.oracle_forward_v.argtypes = [_I, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                         _I, _P, _P, _P, _P, _I, _I, ctypes.c_longlong, _P, _P]
         lib.oracle_forward.restype = _I
         lib.oracle_forward.argtypes = [_I, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                        _I, _P, _P, _P, _P, _P]
@@ -70,10 +76,28 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
-def route(x, Wg, k: int, bias=None):
+#: Gate-weight rules: the method's softmax over the k selected logits, the
+#: softmax over all E logits without renormalisation ("Mixtral 8x7B模型架构解析"
+#: Router.forward), the sigmoid of each selected logit ("万亿 MoE" forward
+#: listing).
+W_SOFTMAX_TOPK, W_SOFTMAX_ALL, W_SIGMOID = 0, 1, 2
+#: Expert activations: SwiGLU silu(W1 x) * W3 x, and the "万亿 MoE" listing's
+#: sigmoid gate sigmoid(W1 x) * W3 x.
+ACT_SILU, ACT_SIGMOID = 0, 1
+
+
+def capacity_limit(capacity_factor: float, T: int, k: int, E: int) -> int:
+    """Per-expert capacity for a capacity factor: floor(cf * T * k / E), the
+    factor times the mean number of (token, slot) pairs per expert (computed
+    in double precision in exactly this order)."""
+    return int(math.floor(float(capacity_factor) * float(T * k) / float(E)))
+
+
+def route(x, Wg, k: int, bias=None, w_mode: int = W_SOFTMAX_TOPK):
     """Router of every token.  Returns dict with ``idx`` [T,k] int32, ``w``
     [T,k] f64, ``gap`` [T] f64 (k-th minus (k+1)-th logit, inf if k == E),
-    ``logits`` [T,E] f64 and ``counts`` [E] int64."""
+    ``logits`` [T,E] f64 and ``counts`` [E] int64.  ``w_mode`` picks the
+    gate-weight rule (the selected set does not depend on it)."""
     x, Wg = _bits(x), _bits(Wg)
     T, d = x.shape
     E = Wg.shape[0]
@@ -84,17 +108,23 @@ def route(x, Wg, k: int, bias=None):
     gap = np.empty((T,), np.float64)
     logits = np.empty((T, E), np.float64)
     counts = np.empty((E,), np.int64)
-    rc = _load().oracle_route(T, d, E, k, _ptr(x), _ptr(Wg), _ptr(b), _ptr(idx), _ptr(w),
-                              _ptr(gap), _ptr(logits), _ptr(counts))
+    rc = _load().oracle_route_v(T, d, E, k, _ptr(x), _ptr(Wg), _ptr(b), int(w_mode), _ptr(idx),
+                                _ptr(w), _ptr(gap), _ptr(logits), _ptr(counts))
     if rc != 0:
         raise ValueError("oracle_route rejected its arguments")
     return {"idx": idx, "w": w, "gap": gap, "logits": logits, "counts": counts}
 
 
-def forward(x, Wg, W1, W3, W2, k: int, bias=None, tokens=None, shared=None, forced=None):
+def forward(x, Wg, W1, W3, W2, k: int, bias=None, tokens=None, shared=None, forced=None,
+            w_mode: int = W_SOFTMAX_TOPK, act_mode: int = ACT_SILU, capacity=None,
+            route_all=None):
     """Layer output (f64) for ``tokens`` (default: all).  ``shared`` is an
     optional (Ws1, Ws3, Ws2) triple of the always-on expert; ``forced`` an
-    optional [n,k] int array of experts to use instead of the token's top-k."""
+    optional [n,k] int array of experts to use instead of the token's top-k.
+    Variants: ``w_mode`` / ``act_mode`` (see the constants above);
+    ``capacity`` (int, per-expert limit, None = dropless) keeps each expert's
+    first ``capacity`` (token, slot) pairs in token order, ranked by the
+    routing ``route_all`` [T,k] (default: the oracle's own)."""
     x, Wg, W1, W3, W2 = (_bits(a) for a in (x, Wg, W1, W3, W2))
     T, d = x.shape
     E, dff = W1.shape[0], W1.shape[1]
@@ -115,10 +145,16 @@ def forward(x, Wg, W1, W3, W2, k: int, bias=None, tokens=None, shared=None, forc
     f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
     if f is not None:
         assert f.shape == (n, k)
+    ra = None if route_all is None else np.ascontiguousarray(route_all, dtype=np.int32)
+    if ra is not None:
+        assert ra.shape == (T, k)
+    cap = -1 if capacity is None else int(capacity)
+    assert capacity is None or cap >= 0
     out = np.empty((n, d), np.float64)
-    rc = _load().oracle_forward(n, _ptr(tok), T, d, E, dff, k, _ptr(x), _ptr(Wg), _ptr(b),
-                                _ptr(W1), _ptr(W3), _ptr(W2), dffs, _ptr(Ws1), _ptr(Ws3),
-                                _ptr(Ws2), _ptr(f), _ptr(out))
+    rc = _load().oracle_forward_v(n, _ptr(tok), T, d, E, dff, k, _ptr(x), _ptr(Wg), _ptr(b),
+                                  _ptr(W1), _ptr(W3), _ptr(W2), dffs, _ptr(Ws1), _ptr(Ws3),
+                                  _ptr(Ws2), _ptr(f), int(w_mode), int(act_mode), cap, _ptr(ra),
+                                  _ptr(out))
     if rc != 0:
         raise ValueError("oracle_forward rejected its arguments")
     return out

@@ -34,6 +34,19 @@ MUTANTS = {
                              "if (!taken[e] && (next < 0 || l[e] < l[next])) next = e;"),
     "gap_skips_a_place": ("*gap = l[sel[k - 1]] - l[next];",
                           "*gap = (k > 1 ? l[sel[k - 2]] : l[sel[k - 1]]) - l[next];"),
+    "softmax_all_normalised_over_selected": (
+        "for (int e = 0; e < E; ++e) s += exp(l[e] - m);",
+        "for (int e = 0; e < k; ++e) s += exp(l[sel[e]] - m);"),
+    "sigmoid_weight_sign": ("for (int j = 0; j < k; ++j) w[j] = sigmoid(l[sel[j]]);",
+                            "for (int j = 0; j < k; ++j) w[j] = sigmoid(-l[sel[j]]);"),
+    "sigmoid_gate_uses_silu": ("if (act_mode == 1) h[f] = sigmoid(a) * b;",
+                               "if (act_mode == 1) h[f] = silu(a) * b;"),
+    "sigmoid_gate_on_w3": ("if (act_mode == 1) h[f] = sigmoid(a) * b;",
+                           "if (act_mode == 1) h[f] = a * sigmoid(b);"),
+    "capacity_off_by_one": ("keep[(size_t)t * k + j] = cnt[e] < cap;",
+                            "keep[(size_t)t * k + j] = cnt[e] <= cap;"),
+    "capacity_reverse_token_order": ("            for (int t = 0; t < T; ++t)\n                for (int j = 0; j < k; ++j) {\n                    int e = sel_all",
+                                     "            for (int t = T - 1; t >= 0; --t)\n                for (int j = 0; j < k; ++j) {\n                    int e = sel_all"),
     "logits_without_bias": ("if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);",
                             "if (logits) { memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);"
                             " if (bias) for (int e = 0; e < E; ++e) logits[(size_t)t * E + e] -= bias[e]; }"),

@@ -318,3 +318,122 @@ def test_logits_and_gap_match_library_formulation(case, ties, with_bias):
         twin = np.isin(np.argsort(-L, axis=1, kind="stable")[:, k - 1:k + 1], [2, 5, 7]).all(1)
         assert twin.any()
         assert (r["gap"][twin] == 0).all()
+
+
+# ---------------------------------------------------------------- variants
+# Routing and expert variants the pages print beside the method: the softmax
+# over all experts without renormalisation ("Mixtral 8x7B模型架构解析"
+# Router.forward), sigmoid gate weights and the sigmoid-gated expert a*sigmoid(g)
+# ("万亿 MoE" forward listing), and the per-expert capacity of "Mistral 8x7B
+# SMoE" sec. 2.4.  Each is pinned against a library formulation (torch fp64
+# softmax / sigmoid / matmuls) or brute force that shares nothing with the C
+# code.
+
+def test_softmax_all_weights_are_the_full_softmax_at_the_selected_experts():
+    wl, inp = _inputs(T=80, d=32, E=10, dff=8, k=3)
+    bias = np.linspace(-0.3, 0.5, 10)
+    r0 = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=3, bias=bias)
+    r1 = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=3, bias=bias, w_mode=oracle.W_SOFTMAX_ALL)
+    assert np.array_equal(r0["idx"], r1["idx"]) and np.array_equal(r0["gap"], r1["gap"])
+    L = (_f64(inp["x"]) @ _f64(inp["Wg"]).T + torch.from_numpy(bias)[None, :])
+    P = torch.softmax(L, dim=-1).numpy()
+    ref = np.take_along_axis(P, r1["idx"].astype(np.int64), 1)
+    assert np.allclose(r1["w"], ref, rtol=1e-12, atol=0)
+    assert (r1["w"].sum(1) < 1).all()            # not renormalised when k < E
+    rk = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=10, w_mode=oracle.W_SOFTMAX_ALL)
+    rk0 = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=10)
+    assert np.allclose(rk["w"], rk0["w"], rtol=1e-12, atol=0)   # k = E: the same weights
+
+
+def test_sigmoid_weights_are_the_logistic_of_each_selected_logit():
+    wl, inp = _inputs(T=60, d=32, E=7, dff=8, k=2)
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), k=2, w_mode=oracle.W_SIGMOID)
+    L = (_f64(inp["x"]) @ _f64(inp["Wg"]).T)
+    ref = torch.sigmoid(torch.gather(L, 1, torch.from_numpy(r["idx"].astype(np.int64)))).numpy()
+    assert np.allclose(r["w"], ref, rtol=1e-12, atol=0)
+
+
+def _sigmoid_glu_torch(x, W1, W3, W2):
+    """The "万亿 MoE" listing's expert: one concatenated up-projection [W3; W1]
+    whose first half a is linear and second half g the gate, h = a * sigmoid(g)."""
+    x, W1, W3, W2 = map(_f64, (x, W1, W3, W2))
+    dff = W1.shape[0]
+    hcat = x @ torch.cat([W3, W1], 0).T
+    a, g = hcat[:, :dff], hcat[:, dff:]
+    return (a * torch.sigmoid(g)) @ W2.T
+
+
+def test_sigmoid_gated_expert_is_the_concatenated_listing_form():
+    wl, inp = _inputs(T=7, d=24, E=1, dff=40, k=1)
+    out = oracle.forward(*(bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")), k=1,
+                         act_mode=oracle.ACT_SIGMOID)
+    ref = _sigmoid_glu_torch(inp["x"], inp["W1"][0], inp["W3"][0], inp["W2"][0]).numpy()
+    assert _rel(out, ref) < 1e-12
+    swi = oracle.forward(*(bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")), k=1)
+    assert _rel(out, swi) > 1e-2
+
+
+def _dense_mask_layer(inp, k, weight_rule, expert_fn, keep=None):
+    """Every expert on every token (torch fp64), kept through a [T, E] mask
+    of gate weights chosen by ``weight_rule`` over the logits."""
+    x, Wg = _f64(inp["x"]), _f64(inp["Wg"])
+    L = (x @ Wg.T).numpy()
+    T, E = L.shape
+    M = np.zeros((T, E))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -L[t]))[:k]
+        w = weight_rule(L[t], order)
+        for j, e in enumerate(order):
+            if keep is None or keep[t, j]:
+                M[t, e] = w[j]
+    Y = np.zeros((T, x.shape[1]))
+    for e in range(E):
+        Y += M[:, e:e + 1] * expert_fn(inp["x"], inp["W1"][e], inp["W3"][e], inp["W2"][e]).numpy()
+    return Y, L
+
+
+def test_listing_layer_sigmoid_weights_and_sigmoid_gate():
+    # The "万亿 MoE" forward listing as a whole: w = sigmoid(logit) of each
+    # selected expert, expert output a * sigmoid(g), weighted sum.
+    wl, inp = _inputs(T=9, d=16, E=5, dff=12, k=2, seed=4)
+    out = oracle.forward(*(bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")), k=2,
+                         w_mode=oracle.W_SIGMOID, act_mode=oracle.ACT_SIGMOID)
+    Y, _ = _dense_mask_layer(inp, 2, lambda l, o: 1 / (1 + np.exp(-l[o])), _sigmoid_glu_torch)
+    assert _rel(out, Y) < 1e-12
+
+
+def test_capacity_limit_closed_form():
+    # floor(cf * T * k / E): capacity factor 1.2 ("Mistral 8x7B SMoE" sec. 2.4)
+    # on the small layer and a few exact cases.
+    assert oracle.capacity_limit(1.2, 512, 2, 8) == 153
+    assert oracle.capacity_limit(1.25, 8, 2, 4) == 5
+    assert oracle.capacity_limit(1.0, 16, 2, 8) == 4
+    assert oracle.capacity_limit(0.0, 16, 2, 8) == 0
+
+
+@pytest.mark.parametrize("cap", [0, 1, 3, 5, 100])
+def test_capacity_keeps_each_experts_first_pairs_in_token_order(cap):
+    # Brute force: walk the tokens in order with a counter per expert; a pair
+    # beyond its expert's capacity drops out of the dense-mask formulation.
+    wl, inp = _inputs(T=24, d=16, E=4, dff=12, k=2, seed=9, dffs=8)
+    names = ("x", "Wg", "W1", "W3", "W2")
+    shared = (bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"]))
+    out = oracle.forward(*(bits(inp[n]) for n in names), k=2, capacity=cap, shared=shared)
+    L = (_f64(inp["x"]) @ _f64(inp["Wg"]).T).numpy()
+    keep = np.zeros((24, 2), bool)
+    seen = [0] * 4
+    for t in range(24):
+        order = np.lexsort((np.arange(4), -L[t]))[:2]
+        for j, e in enumerate(order):
+            keep[t, j] = seen[e] < cap
+            seen[e] += 1
+    softmax_sel = lambda l, o: np.exp(l[o] - l[o].max()) / np.exp(l[o] - l[o].max()).sum()
+    Y, _ = _dense_mask_layer(inp, 2, softmax_sel, _swiglu_torch, keep=keep)
+    Y += _swiglu_torch(inp["x"], inp["Ws1"], inp["Ws3"], inp["Ws2"]).numpy()
+    assert _rel(out, Y) < 1e-12
+    if cap >= 24:
+        full = oracle.forward(*(bits(inp[n]) for n in names), k=2, shared=shared)
+        assert np.array_equal(out, full)
+    if cap == 0:
+        assert np.allclose(out, _swiglu_torch(inp["x"], inp["Ws1"], inp["Ws3"],
+                                              inp["Ws2"]).numpy(), rtol=1e-12, atol=1e-14)
