@@ -12,6 +12,8 @@ from .oracle import (  # noqa: F401
     W_SOFTMAX_TOPK,
     build,
     capacity_limit,
+    e4m3_to_double,
+    forward_fp8,
     num_threads,
     route,
     forward,

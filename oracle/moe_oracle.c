@@ -375,6 +375,117 @@ int oracle_forward_v(int n, const int32_t *tokens, int T, int d, int E, int dff,
     return err ? -1 : 0;
 }
 
+/* ---------------------------------------------------------------- FP8 experts
+ * Expert weights stored as 8-bit floating point codes with one scale per
+ * weight row ("Mistral 8x7B SMoE" (jsqmd.com) deployment section:
+ * quantised experts, router kept in higher precision): the weight is
+ * W[e, r, i] = scale[e, r] * e4m3(code[e, r, i]).  e4m3 is the OCP 8-bit
+ * format E4M3 (no infinities): sign bit 7, exponent bits 6..3 with bias 7,
+ * mantissa bits 2..0; exponent 0 holds the subnormals 2^-6 * m/8; exponent
+ * 15 with mantissa 7 is NaN; the largest finite value is 448. */
+static double e4m3_to_double(uint8_t b)
+{
+    const int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = e == 0 ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+    return sgn ? -v : v;
+}
+
+double oracle_e4m3_to_double(int code) { return e4m3_to_double((uint8_t)code); }
+
+/* One SwiGLU expert on one token with FP8 weights: rows of W1/W3 [dff, d]
+ * and W2 [d, dff] as codes, s1/s3 [dff] and s2 [d] the row scales. */
+static void swiglu_one_fp8(int d, int dff, const uint8_t *q1, const double *s1,
+                           const uint8_t *q3, const double *s3, const uint8_t *q2,
+                           const double *s2, const double *xt, double *h, double *y)
+{
+    for (int f = 0; f < dff; ++f) {
+        const uint8_t *r1 = q1 + (size_t)f * d;
+        const uint8_t *r3 = q3 + (size_t)f * d;
+        double a = 0.0, b = 0.0;
+        for (int i = 0; i < d; ++i) a += s1[f] * e4m3_to_double(r1[i]) * xt[i];
+        for (int i = 0; i < d; ++i) b += s3[f] * e4m3_to_double(r3[i]) * xt[i];
+        h[f] = silu(a) * b;
+    }
+    for (int o = 0; o < d; ++o) {
+        const uint8_t *r2 = q2 + (size_t)o * dff;
+        double acc = 0.0;
+        for (int f = 0; f < dff; ++f) acc += s2[o] * e4m3_to_double(r2[f]) * h[f];
+        y[o] = acc;
+    }
+}
+
+/* Layer output for n selected tokens with FP8 experts: the method (router in
+ * bf16, top-k, softmax over the selected, weighted sum in slot order) with
+ * W1/W3/W2 given as codes q1/q3 [E,dff,d], q2 [E,d,dff] and row scales
+ * s1/s3 [E,dff], s2 [E,d].  tokens and forced as in oracle_forward. */
+int oracle_forward_fp8(int n, const int32_t *tokens, int T, int d, int E, int dff, int k,
+                       const uint16_t *x, const uint16_t *Wg, const double *bias,
+                       const uint8_t *q1, const double *s1, const uint8_t *q3, const double *s3,
+                       const uint8_t *q2, const double *s2, const int32_t *forced, double *out)
+{
+    if (n < 0 || T < 1 || d < 1 || E < 1 || dff < 1 || k < 1 || k > E) return -1;
+    if (!x || !Wg || !q1 || !s1 || !q3 || !s3 || !q2 || !s2 || !out) return -1;
+    for (int r = 0; r < n; ++r) {
+        int t = tokens ? tokens[r] : r;
+        if (t < 0 || t >= T) return -1;
+        if (forced)
+            for (int j = 0; j < k; ++j)
+                if (forced[(size_t)r * k + j] < 0 || forced[(size_t)r * k + j] >= E) return -1;
+    }
+    int err = 0;
+#pragma omp parallel
+    {
+        double *xt = (double *)malloc(sizeof(double) * (size_t)d);
+        double *l = (double *)malloc(sizeof(double) * (size_t)E);
+        double *h = (double *)malloc(sizeof(double) * (size_t)dff);
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
+        double *w = (double *)malloc(sizeof(double) * (size_t)k);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+        unsigned char *taken = (unsigned char *)malloc((size_t)E);
+        if (!xt || !l || !h || !y || !w || !sel || !taken) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int r = 0; r < n; ++r) {
+                int t = tokens ? tokens[r] : r;
+                for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)t * d + i]);
+                route_one(d, E, k, xt, Wg, bias, l, sel, w, NULL, taken);
+                if (forced) {
+                    double m = -INFINITY, s = 0.0;
+                    for (int j = 0; j < k; ++j) {
+                        sel[j] = forced[(size_t)r * k + j];
+                        if (l[sel[j]] > m) m = l[sel[j]];
+                    }
+                    for (int j = 0; j < k; ++j) {
+                        w[j] = exp(l[sel[j]] - m);
+                        s += w[j];
+                    }
+                    for (int j = 0; j < k; ++j) w[j] /= s;
+                }
+                double *o = out + (size_t)r * d;
+                for (int i = 0; i < d; ++i) o[i] = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    int e = sel[j];
+                    swiglu_one_fp8(d, dff, q1 + (size_t)e * dff * d, s1 + (size_t)e * dff,
+                                   q3 + (size_t)e * dff * d, s3 + (size_t)e * dff,
+                                   q2 + (size_t)e * d * dff, s2 + (size_t)e * d, xt, h, y);
+                    for (int i = 0; i < d; ++i) o[i] += w[j] * y[i];
+                }
+            }
+        }
+        free(xt);
+        free(l);
+        free(h);
+        free(y);
+        free(w);
+        free(sel);
+        free(taken);
+    }
+    return err ? -1 : 0;
+}
+
 /* One SwiGLU expert applied to n rows (no routing): out[r] = W2(silu(W1 x_r) * W3 x_r).
  * Used to check the expert FFN by itself. */
 int oracle_swiglu(int n, int d, int dff, const uint16_t *x, const uint16_t *W1,

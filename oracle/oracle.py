@@ -55,6 +55,11 @@ def _load():
         lib.oracle_forward.restype = _I
         lib.oracle_forward.argtypes = [_I, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                                        _I, _P, _P, _P, _P, _P]
+        lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_e4m3_to_double.argtypes = [_I]
+        lib.oracle_forward_fp8.restype = _I
+        lib.oracle_forward_fp8.argtypes = [_I, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                                           _P, _P, _P, _P, _P]
         lib.oracle_swiglu.restype = _I
         lib.oracle_swiglu.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P]
         _lib = lib
@@ -170,4 +175,34 @@ def swiglu(x, W1, W3, W2):
     rc = _load().oracle_swiglu(n, d, dff, _ptr(x), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(out))
     if rc != 0:
         raise ValueError("oracle_swiglu rejected its arguments")
+    return out
+
+
+def e4m3_to_double(code: int) -> float:
+    """Value of one e4m3 code (OCP E4M3, no infinities)."""
+    return float(_load().oracle_e4m3_to_double(int(code)))
+
+
+def forward_fp8(x, Wg, q1, s1, q3, s3, q2, s2, k: int, bias=None, tokens=None, forced=None):
+    """Layer output (f64) with FP8 experts: q1/q3 [E,dff,d] and q2 [E,d,dff]
+    e4m3 codes (numpy uint8), s1/s3 [E,dff] and s2 [E,d] row scales; the
+    router reads bf16 x and Wg as in ``forward``."""
+    x, Wg = _bits(x), _bits(Wg)
+    q1, q3, q2 = (np.ascontiguousarray(a, dtype=np.uint8) for a in (q1, q3, q2))
+    s1, s3, s2 = (np.ascontiguousarray(a, dtype=np.float64) for a in (s1, s3, s2))
+    T, d = x.shape
+    E, dff = q1.shape[0], q1.shape[1]
+    assert q1.shape == (E, dff, d) and q3.shape == (E, dff, d) and q2.shape == (E, d, dff)
+    assert s1.shape == (E, dff) and s3.shape == (E, dff) and s2.shape == (E, d)
+    assert Wg.shape == (E, d)
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    n = T if tok is None else tok.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+    f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
+    out = np.empty((n, d), np.float64)
+    rc = _load().oracle_forward_fp8(n, _ptr(tok), T, d, E, dff, k, _ptr(x), _ptr(Wg), _ptr(b),
+                                    _ptr(q1), _ptr(s1), _ptr(q3), _ptr(s3), _ptr(q2), _ptr(s2),
+                                    _ptr(f), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_forward_fp8 rejected its arguments")
     return out

@@ -146,3 +146,45 @@ def shard_tokens(T: int, rank: int, world: int) -> tuple[int, int]:
 def rank_seed(seed: int, rank: int) -> int:
     """Seed of rank ``rank``'s independent batch under weak scaling."""
     return seed + 1000003 * rank
+
+
+def make_fp8_experts(wl: Workload, seed: int = 42, device="cpu", pow2_scales: bool = False) -> dict:
+    """Seeded FP8 expert weights of ``wl``'s shapes: the bf16 recipe's normal
+    draws (W1, W3 with sigma 1/sqrt(d), W2 with 1/sqrt(d_ff), drawn after x
+    and Wg from the same seeded generator), each weight row stored as e4m3
+    codes (torch.float8_e4m3fn, round to nearest even) and one fp32 scale,
+    scale = max|row| / 448 (rounded up to a power of two when
+    ``pow2_scales``), so that no code overflows the format.  Returns x, Wg (bf16, as make_inputs), q1, q3 [E,d_ff,d]
+    and q2 [E,d,d_ff] as uint8 code tensors, s1, s3 [E,d_ff] and s2 [E,d]
+    fp32, and the router bias."""
+    device = torch.device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    T, d, E, f = wl.T, wl.d, wl.E, wl.d_ff
+    out = {
+        "x": _draw(g, (T, d), 1.0, device, _X_ROWS_PER_SLICE),
+        "Wg": _draw(g, (E, d), 1.0 / math.sqrt(d), device, E),
+    }
+    for name, shape, sigma in (("1", (E, f, d), 1.0 / math.sqrt(d)),
+                               ("3", (E, f, d), 1.0 / math.sqrt(d)),
+                               ("2", (E, d, f), 1.0 / math.sqrt(f))):
+        q = torch.empty(shape, dtype=torch.uint8, device=device)
+        sc = torch.empty(shape[:2], dtype=torch.float32, device=device)
+        for e in range(shape[0]):
+            w = torch.randn(shape[1:], generator=g, dtype=torch.float32, device=device) * sigma
+            s = w.abs().amax(dim=1).clamp_min(1e-30) / 448.0
+            if pow2_scales:
+                s = torch.exp2(torch.ceil(torch.log2(s)))
+            q[e] = (w / s[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+            sc[e] = s
+        out["q" + name] = q
+        out["s" + name] = sc
+    out["bias"] = router_bias(wl, device)
+    return out
+
+
+def fp8_dequant_bf16(q: torch.Tensor, s: torch.Tensor) -> torch.Tensor:
+    """bf16 tensor of scale * e4m3(code) (exact when the scales are powers of
+    two and the products in range), for checks only."""
+    v = q.view(torch.float8_e4m3fn).to(torch.float32) * s[..., None]
+    return v.to(torch.bfloat16)

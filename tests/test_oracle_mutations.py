@@ -47,6 +47,12 @@ MUTANTS = {
                             "keep[(size_t)t * k + j] = cnt[e] <= cap;"),
     "capacity_reverse_token_order": ("            for (int t = 0; t < T; ++t)\n                for (int j = 0; j < k; ++j) {\n                    int e = sel_all",
                                      "            for (int t = T - 1; t >= 0; --t)\n                for (int j = 0; j < k; ++j) {\n                    int e = sel_all"),
+    "e4m3_exponent_bias": ("ldexp(8.0 + m, e - 10)", "ldexp(8.0 + m, e - 11)"),
+    "e4m3_subnormal_scale": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
+    "fp8_scale_of_wrong_row": ("for (int i = 0; i < d; ++i) b += s3[f] * e4m3_to_double(r3[i]) * xt[i];",
+                               "for (int i = 0; i < d; ++i) b += s3[0] * e4m3_to_double(r3[i]) * xt[i];"),
+    "fp8_w2_scale_by_hidden_index": ("acc += s2[o] * e4m3_to_double(r2[f]) * h[f];",
+                                     "acc += s2[f % d] * e4m3_to_double(r2[f]) * h[f];"),
     "logits_without_bias": ("if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);",
                             "if (logits) { memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);"
                             " if (bias) for (int e = 0; e < E; ++e) logits[(size_t)t * E + e] -= bias[e]; }"),

@@ -437,3 +437,53 @@ def test_capacity_keeps_each_experts_first_pairs_in_token_order(cap):
     if cap == 0:
         assert np.allclose(out, _swiglu_torch(inp["x"], inp["Ws1"], inp["Ws3"],
                                               inp["Ws2"]).numpy(), rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- FP8 experts
+def test_e4m3_decoder_matches_the_format_and_torch():
+    # OCP E4M3: 1.0 = 0x38, largest finite 448 = 0x7E, smallest normal 2^-6 =
+    # 0x08, smallest subnormal 2^-9 = 0x01, NaN 0x7F / 0xFF, no infinities;
+    # every code against torch's float8_e4m3fn conversion (a library routine).
+    assert oracle.e4m3_to_double(0x38) == 1.0
+    assert oracle.e4m3_to_double(0x7E) == 448.0 and oracle.e4m3_to_double(0xFE) == -448.0
+    assert oracle.e4m3_to_double(0x08) == 2.0 ** -6 and oracle.e4m3_to_double(0x01) == 2.0 ** -9
+    assert math.isnan(oracle.e4m3_to_double(0x7F)) and math.isnan(oracle.e4m3_to_double(0xFF))
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    for c in range(256):
+        v = oracle.e4m3_to_double(c)
+        if math.isnan(ref[c].item()):
+            assert math.isnan(v)
+        else:
+            assert v == ref[c].item(), hex(c)
+
+
+def test_fp8_layer_with_power_of_two_scales_is_the_bf16_layer_exactly():
+    # With power-of-two row scales every dequantised weight s * e4m3(q) is a
+    # bf16 value; the FP8 layer must then equal the (pinned) bf16 layer on
+    # those weights bit for bit -- same fp64 arithmetic in the same order.
+    wl = Workload("fp8", 12, 32, 5, 24, 2)
+    inp = synth.make_fp8_experts(wl, seed=6, pow2_scales=True)
+    W = {n: synth.fp8_dequant_bf16(inp["q" + n], inp["s" + n]) for n in ("1", "3", "2")}
+    for n in ("1", "3", "2"):
+        back = W[n].to(torch.float64) / inp["s" + n].double()[..., None]
+        assert torch.equal(back, inp["q" + n].view(torch.float8_e4m3fn).to(torch.float64))
+    a = oracle.forward_fp8(bits(inp["x"]), bits(inp["Wg"]),
+                           *(t.numpy() for t in (inp["q1"], inp["s1"].double(), inp["q3"],
+                                                 inp["s3"].double(), inp["q2"], inp["s2"].double())),
+                           k=2)
+    b = oracle.forward(bits(inp["x"]), bits(inp["Wg"]), bits(W["1"]), bits(W["3"]), bits(W["2"]),
+                       k=2)
+    assert np.array_equal(a, b)
+    assert len(np.unique(inp["s1"].numpy())) > 1      # per-row scales really differ
+
+
+def test_fp8_layer_is_linear_in_the_w2_and_w3_scales():
+    wl = Workload("fp8", 8, 32, 4, 16, 2)
+    inp = synth.make_fp8_experts(wl, seed=2)
+    args = lambda s1, s3, s2: (bits(inp["x"]), bits(inp["Wg"]), inp["q1"].numpy(), s1,
+                                inp["q3"].numpy(), s3, inp["q2"].numpy(), s2)
+    s1, s3, s2 = (inp[n].double().numpy() for n in ("s1", "s3", "s2"))
+    base = oracle.forward_fp8(*args(s1, s3, s2), k=2)
+    assert np.array_equal(oracle.forward_fp8(*args(s1, s3, 2 * s2), k=2), 2 * base)
+    assert np.array_equal(oracle.forward_fp8(*args(s1, 2 * s3, s2), k=2), 2 * base)
+    assert _rel(oracle.forward_fp8(*args(2 * s1, s3, s2), k=2), base) > 1e-3
