@@ -5,16 +5,22 @@
 
 One JSON line on rank 0.  A *step* is one pass of the whole layer (routing,
 dispatch, both expert GEMMs, combine) over one batch of every layer of the
-workload.  The default workload is the fixed-total-parameter granularity
-sweep of the "万亿 MoE 只激活 4.9%" page: T = 512 tokens, d = 512,
-E * d_ff = 32768, (E, d_ff, k) in {(8,4096,1), (8,4096,2), (32,1024,1),
-(32,1024,2), (64,512,4), (128,256,8)} -- six layers, 604 MB of bf16 weights,
-more than the 126 MB L2, so every step streams its weights from HBM.
+workload.  The default workload is the largest configuration: the
+fine-grained layer with d = 7168, 256 routed experts of d_ff = 2048, top-8
+softmax routing and one always-on shared expert of d_ff = 2048, T = 8192
+tokens ("MoE" (theaiera.top) sec. 10.5, the "1 shared + 8 of 256" remark);
+22.6 GB of bf16 weights, far more than the 126 MB L2, so every step streams
+its weights from HBM.  ``--workload sweep`` runs the fixed-total-parameter
+granularity sweep of the "万亿 MoE 只激活 4.9%" page instead (T = 512, d = 512,
+E * d_ff = 32768, six layers), and the other names the Mixtral-shaped prefill
+and decode layers and the small layer.
 
 Metric: MoE-layer tokens/s (tokens x layers per second) and active TFLOP/s.
 Timing: K steps captured in one CUDA graph, bracketed by a barrier and device
 synchronisation, max over ranks; a second pass of the same K steps, captured
-with CUDA events at every kernel boundary, gives each kernel's duration.
+with CUDA events at every kernel boundary, gives each kernel's duration; a
+third pass replays a one-step graph K times between events for the median
+step time.
 Multi-GPU is weak scaling: every rank runs the same workload on its own seeded
 batch with its own weights (data parallel replicas, no collective on the data
 path).  ``--impl reference`` times the fp64 CPU oracle instead.
@@ -22,6 +28,7 @@ path).  ``--impl reference`` times the fp64 CPU oracle instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -44,6 +51,7 @@ METRIC = "MoE-layer tokens/s & active TFLOP/s, % of bf16 tensor / HBM roofline"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -57,11 +65,30 @@ def workload(name: str) -> list:
         rest = name[len("mixtral_prefill_T"):]
         skew = rest.endswith("_skewed")
         return [synth.mixtral_prefill(int(rest.replace("_skewed", "")), skew)]
+    if name.startswith("mixtral_decode_T") and name.endswith("_fp8"):
+        wl = synth.mixtral_decode(int(name[len("mixtral_decode_T"):-len("_fp8")]))
+        return [dataclasses.replace(wl, name=wl.name + "_fp8", extra={"fp8": True})]
     if name.startswith("mixtral_decode_T"):
         return [synth.mixtral_decode(int(name[len("mixtral_decode_T"):]))]
     if name.startswith("fine_grained_T"):
-        return [synth.fine_grained(int(name[len("fine_grained_T"):]))]
+        rest = name[len("fine_grained_T"):]
+        if "_E" in rest:
+            T, E = rest.split("_E")
+            return [synth.fine_grained(int(T), int(E))]
+        return [synth.fine_grained(int(rest))]
     raise SystemExit(f"unknown workload {name}")
+
+
+def is_fp8(wl) -> bool:
+    return bool(wl.extra.get("fp8"))
+
+
+def make_inputs(wl, seed, device):
+    """The workload's seeded inputs: bf16 experts, or e4m3 experts with row
+    scales for the FP8 workloads."""
+    if is_fp8(wl):
+        return synth.make_fp8_experts(wl, seed=seed, device=device)
+    return synth.make_inputs(wl, seed=seed, device=device)
 
 
 def describe(wls, name):
@@ -70,7 +97,9 @@ def describe(wls, name):
         "layers": [{"T": w.T, "d": w.d, "E": w.E, "d_ff": w.d_ff, "k": w.k,
                     **({"d_ff_shared": w.d_ff_shared} if w.d_ff_shared else {}),
                     **({"router_bias": f"+{synth.SKEW_BIAS} on expert {synth.SKEW_EXPERT}"}
-                       if w.skew else {})} for w in wls],
+                       if w.skew else {}),
+                    **({"experts": "e4m3 codes with fp32 row scales, bf16 router"}
+                       if is_fp8(w) else {})} for w in wls],
         "global_batch_tokens": sum(w.T for w in wls),
     }
 
@@ -182,42 +211,57 @@ def barrier(world):
 
 
 # ----------------------------------------------------------------------------- oracle arm
-def oracle_step_fn(wls, seed, tokens_per_layer):
-    """A bounded sample of one step on the host cores: the oracle's forward of
-    ``tokens_per_layer`` seeded tokens of every layer."""
-    import oracle
+def oracle_host_inputs(wls, inps):
+    """Raw bf16 bits (host numpy arrays) of every layer's inputs, copied once
+    from wherever the inputs live."""
     from sparse_mixture_experts_histogram_b200.synth import bits
     data = []
-    g = np.random.default_rng(seed)
-    for wl in wls:
-        inp = synth.make_inputs(wl, seed=seed, device="cpu")
-        b = None if inp["bias"] is None else inp["bias"].double().numpy()
+    for wl, inp in zip(wls, inps):
+        b = None if inp["bias"] is None else inp["bias"].double().cpu().numpy()
         shared = (bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"])) if wl.d_ff_shared else None
-        arrs = [bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")]
-        tok = np.sort(g.choice(wl.T, size=min(tokens_per_layer, wl.T), replace=False))
-        data.append((wl, arrs, b, shared, tok))
+        if is_fp8(wl):
+            arrs = [bits(inp["x"]), bits(inp["Wg"])] + [
+                inp[n].cpu().numpy() if n.startswith("q") else inp[n].double().cpu().numpy()
+                for n in ("q1", "s1", "q3", "s3", "q2", "s2")]
+        else:
+            arrs = [bits(inp[n]) for n in ("x", "Wg", "W1", "W3", "W2")]
+        data.append((wl, arrs, b, shared))
+    return data
+
+
+def oracle_step_fn(data, seed, tokens_per_layer):
+    """A bounded sample of one step on the host cores: the oracle's forward
+    (routing over all E experts, the k selected experts, the shared expert) of
+    ``tokens_per_layer`` seeded tokens of every layer."""
+    import oracle
+    g = np.random.default_rng(seed)
+    toks = [np.sort(g.choice(wl.T, size=min(tokens_per_layer, wl.T), replace=False))
+            for (wl, _, _, _) in data]
 
     def step():
         n = 0
-        for wl, arrs, b, shared, tok in data:
-            oracle.forward(*arrs, wl.k, bias=b, tokens=tok, shared=shared)
+        for (wl, arrs, b, shared), tok in zip(data, toks):
+            if is_fp8(wl):
+                oracle.forward_fp8(*arrs, wl.k, bias=b, tokens=tok)
+            else:
+                oracle.forward(*arrs, wl.k, bias=b, tokens=tok, shared=shared)
             n += len(tok)
         return n
     return step
 
 
-def run_oracle(wls, steps, warmup, target_s=2.0, seed=42):
+def run_oracle(data, steps, warmup, target_s=2.0, seed=42):
     """Times the oracle: calibrate a per-layer token sample that takes about
     ``target_s`` per step, then run ``warmup`` + ``steps`` steps."""
     import oracle
     oracle.build()
-    probe = oracle_step_fn(wls, seed, 4)
+    probe = oracle_step_fn(data, seed, oracle.num_threads())
     t0 = time.perf_counter()
     n = probe()
     dt = max(time.perf_counter() - t0, 1e-6)
     per_tok = dt / n
-    tpl = int(max(1, min(max(w.T for w in wls), target_s / per_tok / len(wls))))
-    step = oracle_step_fn(wls, seed, tpl)
+    tpl = int(max(1, min(max(d[0].T for d in data), target_s / per_tok / len(data))))
+    step = oracle_step_fn(data, seed, tpl)
     for _ in range(warmup):
         step()
     t0 = time.perf_counter()
@@ -235,7 +279,13 @@ def reference_arm(args):
     if rank != 0:
         return 0
     wls = workload(args.workload)
-    r = run_oracle(wls, args.steps, args.warmup, target_s=args.oracle_step_s)
+    # Inputs are drawn where the GPU arm draws them (the same bits); the
+    # oracle itself only ever runs on the host cores.
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inps = [make_inputs(wl, seed=42 + i, device=dev) for i, wl in enumerate(wls)]
+    data = oracle_host_inputs(wls, inps)
+    del inps
+    r = run_oracle(data, args.steps, args.warmup, target_s=args.oracle_step_s)
     sample = (f"{r['tokens_per_layer']} seeded tokens of each of the {len(wls)} layer(s) per step "
               f"(fp64 oracle, all routing and expert work of those tokens)")
     line = {
@@ -275,6 +325,34 @@ def traffic_record(kernel_key):
     return r
 
 
+def profile_arm(args):
+    """``--profile``: run every layer of the workload ``--steps`` times through
+    the public API (eager launches, nothing timed) and exit -- the program an
+    ncu capture wraps."""
+    import sparse_mixture_experts_histogram_b200 as moe
+    dev = torch.device("cuda", 0)
+    wls = workload(args.workload)
+    inps = [make_inputs(wl, seed=42 + i, device=dev) for i, wl in enumerate(wls)]
+    outs = [torch.empty(wl.T, wl.d, dtype=torch.float32, device=dev) for wl in wls]
+    ws = torch.empty(max(moe.moe_workspace_size_ex(w.T, w.d, w.E, w.d_ff, w.k, w.d_ff_shared)
+                         for w in wls), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    for _ in range(args.steps):
+        for wl, inp, out in zip(wls, inps, outs):
+            if is_fp8(wl):
+                moe.moe_forward_fp8(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"],
+                                    inp["bias"], inp["q1"], inp["s1"], inp["q3"], inp["s3"],
+                                    inp["q2"], inp["s2"], out, ws)
+            else:
+                moe.moe_forward_ex(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"],
+                                   inp["bias"], inp["W1"], inp["W3"], inp["W2"], wl.d_ff_shared,
+                                   inp.get("Ws1"), inp.get("Ws3"), inp.get("Ws2"), out, ws)
+    st, code = moe.moe_get_device_error(ws)
+    print(json.dumps({"profile_run": args.workload, "launch_rounds": args.steps,
+                      "status": st, "error_word": code}))
+    return 0 if st == 0 else 1
+
+
 def gpu_arm(args):
     import sparse_mixture_experts_histogram_b200 as moe
     rank, world, local = dist_init(nccl=True)
@@ -287,7 +365,7 @@ def gpu_arm(args):
     # ---- resident inputs and buffers
     inps, outs = [], []
     for i, wl in enumerate(wls):
-        inps.append(synth.make_inputs(wl, seed=seed + i, device=dev))
+        inps.append(make_inputs(wl, seed=seed + i, device=dev))
         outs.append(torch.empty(wl.T, wl.d, dtype=torch.float32, device=dev))
     ws_bytes = max(moe.moe_workspace_size_ex(w.T, w.d, w.E, w.d_ff, w.k, w.d_ff_shared)
                    for w in wls)
@@ -309,11 +387,21 @@ def gpu_arm(args):
             stream.synchronize()
             hit.append(int((cnt > 0).sum().item()))
 
-    def layer_call(i, events=None):
+    def layer_call(i, events=None, x=None, out=None):
         wl, inp = wls[i], inps[i]
-        a = (wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["bias"], inp["W1"],
+        x = inp["x"] if x is None else x
+        out = outs[i] if out is None else out
+        if is_fp8(wl):
+            a = (wl.T, wl.d, wl.E, wl.d_ff, wl.k, x, inp["Wg"], inp["bias"], inp["q1"],
+                 inp["s1"], inp["q3"], inp["s3"], inp["q2"], inp["s2"], out, ws)
+            if events is None:
+                moe.moe_forward_fp8(*a, stream=stream)
+            else:
+                moe.moe_forward_fp8_traced(*a, events, stream=stream)
+            return
+        a = (wl.T, wl.d, wl.E, wl.d_ff, wl.k, x, inp["Wg"], inp["bias"], inp["W1"],
              inp["W3"], inp["W2"], wl.d_ff_shared, inp.get("Ws1"), inp.get("Ws3"),
-             inp.get("Ws2"), outs[i], ws)
+             inp.get("Ws2"), out, ws)
         if events is None:
             moe.moe_forward_ex(*a, stream=stream)
         else:
@@ -389,6 +477,19 @@ def gpu_arm(args):
         ms, clocks = timed(gK_plain)
         clocks["remeasured"] = True
     ms_traced, _ = timed(gK, soak_s=0.2)
+
+    # Median step: the one-step graph replayed K more times, each replay
+    # between its own pair of events (the median over >= 20 replays).
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        step_ev[0].record(stream)
+        for i in range(args.steps):
+            g1.replay()
+            step_ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    step_ms = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
+    ms_median = dist_max(statistics.median(step_ms), world)
     st, code = moe.moe_get_device_error(ws, stream)
     if st != 0:
         raise SystemExit(f"device error word {code:#x} after the timed region")
@@ -418,13 +519,14 @@ def gpu_arm(args):
     # ---- throughput and roofline
     tokens_per_step = sum(w.T for w in wls)
     flops_per_step = sum(acc.active_flops(w.T, w.d, w.E, w.d_ff, w.k, w.d_ff_shared) for w in wls)
-    bytes_per_step = sum(acc.algorithmic_bytes(w.T, w.d, w.E, w.d_ff, w.k, h, w.d_ff_shared)
+    bytes_per_step = sum(acc.algorithmic_bytes(w.T, w.d, w.E, w.d_ff, w.k, h, w.d_ff_shared,
+                                               fp8=is_fp8(w))
                          for w, h in zip(wls, hit))
     sec = ms / 1e3
     value = weak_scaling_value(world, tokens_per_step, args.steps, ms)
     pk, pk_src = peaks()
     # dominant kernel: the expert feed-forward (both projections, one launch)
-    up_bytes = [acc.ffn_bytes(w.T, w.d, w.d_ff, w.k, h) for w, h in zip(wls, hit)]
+    up_bytes = [acc.ffn_bytes(w.T, w.d, w.d_ff, w.k, h, fp8=is_fp8(w)) for w, h in zip(wls, hit)]
     up_flops = [acc.ffn_flops(w.T, w.d, w.d_ff, w.k) for w in wls]
     up_time = [sum(t) / len(t) for t in per_layer_up]
     ai = sum(up_flops) / sum(up_bytes)
@@ -438,6 +540,13 @@ def gpu_arm(args):
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "peak_source": f"hbm_gbs ({pk_src})"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    if roof["bound"] == "tensor":
+        roof["frac_of_burst_peak"] = roof["achieved"] / pk["bf16_tflops"]
+    # The same against the B200's nominal figures (dense bf16 tensor peak,
+    # HBM3e bandwidth), on which the targets are stated.
+    spec_peak = SPEC_PEAKS["bf16_tflops"] if roof["bound"] == "tensor" else SPEC_PEAKS["hbm_gbs"]
+    roof["spec"] = {"peak": spec_peak, "frac": roof["achieved"] / spec_peak,
+                    "source": "B200 nominal: 2.25 PFLOP/s dense bf16, 8 TB/s HBM3e"}
     tr = traffic_record(f"expert_ffn:{args.workload}")
     roof["traffic"] = None if tr is None else tr["bytes_per_launch"]
     kinds = []
@@ -452,6 +561,8 @@ def gpu_arm(args):
     roof["launch_ms"] = sum(up_time) / len(up_time)
     step_roof = max(flops_per_step / (pk["bf16_tflops_sustained"] * 1e12),
                     bytes_per_step / (pk["hbm_gbs"] * 1e9))
+    step_roof_spec = max(flops_per_step / (SPEC_PEAKS["bf16_tflops"] * 1e12),
+                         bytes_per_step / (SPEC_PEAKS["hbm_gbs"] * 1e9))
 
     # ---- end to end through the public API with host buffers
     # Every step copies each layer's x in from pinned host memory and its out
@@ -487,10 +598,7 @@ def gpu_arm(args):
                 ev_in[b][i].record(s_in)
             stream.wait_event(ev_in[b][i])
             stream.wait_event(ev_out[b][i])           # the earlier o_dev[b][i] is copied out
-            moe.moe_forward_ex(wl.T, wl.d, wl.E, wl.d_ff, wl.k, x_dev[b][i], inp["Wg"],
-                               inp["bias"], inp["W1"], inp["W3"], inp["W2"], wl.d_ff_shared,
-                               inp.get("Ws1"), inp.get("Ws3"), inp.get("Ws2"), o_dev[b][i], ws,
-                               stream=stream)
+            layer_call(i, x=x_dev[b][i], out=o_dev[b][i])
             ev_cmp[b][i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_cmp[b][i])
@@ -524,7 +632,10 @@ def gpu_arm(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("fp16 MMA on e4m3 experts (bf16 router)" if any(is_fp8(w) for w in wls)
+                  else "bf16"),
+        "data": "synthetic",
         "config": {**describe(wls, args.workload), "parallelism": f"dp{world} (replicas)",
                    "l2": ("no flush: the step's working set "
                           f"({bytes_per_step / 1e6:.0f} MB of algorithmic bytes) exceeds the "
@@ -532,6 +643,9 @@ def gpu_arm(args):
                           "working set below L2 size: warm-L2 number")},
         "active_tflops": world * flops_per_step * args.steps / sec / 1e12,
         "step_roofline_frac": step_roof * args.steps / sec * 1.0,
+        "step_roofline_frac_spec": step_roof_spec * args.steps / sec * 1.0,
+        "ms_per_step_median": ms_median,
+        "median_replays": args.steps,
         "roofline": roof,
         "kernel_ms": kernel_ms,
         "kernel_share": kernel_share,
@@ -551,7 +665,8 @@ def gpu_arm(args):
     }
     del g1, gK, gK_plain
     if world == 1 and not args.no_cpu_baseline:
-        r = run_oracle(wls, steps=2, warmup=0, target_s=args.oracle_step_s)
+        r = run_oracle(oracle_host_inputs(wls, inps), steps=2, warmup=0,
+                       target_s=args.oracle_step_s)
         line["cpu_baseline"] = {
             "value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
             "sample": (f"{r['tokens_per_layer']} seeded tokens of each of the {len(wls)} layers, "
@@ -569,16 +684,23 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="sweep")
+    ap.add_argument("--workload", default="fine_grained_T8192",
+                    help="fine_grained_T8192 (default: the largest config, 256 experts top-8 "
+                         "plus a shared expert), sweep, small, mixtral_prefill_T{2048,8192}"
+                         "[_skewed], mixtral_decode_T{1,8,32,128}[_fp8]")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--oracle-step-s", type=float, default=5.0,
+    ap.add_argument("--oracle-step-s", type=float, default=4.0,
                     help="seconds of host work per oracle step (bounded sample)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run the layers --steps times untimed and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return reference_arm(args)
+    if args.profile:
+        return profile_arm(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

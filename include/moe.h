@@ -102,7 +102,8 @@ MOE_API size_t moe_workspace_size_ex(int T, int d, int E, int d_ff, int k, int d
  *     build skewed loads)
  *   idx [T,k] int32 out: experts of each token, by logit descending
  *   w [T,k] fp32 out: their softmax weights (sum to 1 per token)
- *   counts [E] int32 out: number of (token, slot) pairs routed to each expert
+ *   counts [E] int32 out, or NULL: number of (token, slot) pairs routed to
+ *     each expert
  * Passages: jsqmd.com sec. 3.2 (gate -> topk -> softmax over the selected
  * values); theaiera.top sec. 10.3 (weights sum to 1); torch.unique / per
  * expert token lists of sec. 10.4 become the histogram. */
@@ -172,29 +173,112 @@ MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const mo
                           const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
                           float *out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Layer variants the pages describe beside the method.  All fields zero is
+ * the method itself (moe_forward_ex).
+ *   weights: gate-weight rule of the k selected experts
+ *     MOE_WEIGHTS_SOFTMAX_TOPK  softmax over the k selected logits (the method)
+ *     MOE_WEIGHTS_SOFTMAX_ALL   softmax over all E logits; the selected keep
+ *                               their probabilities, not renormalised
+ *                               ("Mixtral 8x7B模型架构解析" (bjdmk.com.cn),
+ *                               Router.forward)
+ *     MOE_WEIGHTS_SIGMOID       the logistic sigmoid of each selected logit
+ *                               ("万亿 MoE" (m.xxqk.cn) forward listing)
+ *   activation: expert hidden units
+ *     MOE_ACT_SILU     silu(W1 x) * (W3 x), SwiGLU (the method)
+ *     MOE_ACT_SIGMOID  sigmoid(W1 x) * (W3 x), the listing's a * sigmoid(g)
+ *                      with its gate g the W1 rows and a the W3 rows
+ *   capacity_factor: 0 = dropless (the method); > 0: expert capacity
+ *     C = floor(capacity_factor * T * k / E) ("Mistral 8x7B SMoE" (jsqmd.com)
+ *     sec. 2.4, capacity factor 1.2): of the (token, slot) pairs routed to an
+ *     expert only the first C in token order are computed; a dropped pair
+ *     adds nothing to its token (the other slots keep their weights).
+ *     Negative or non-finite values are MOE_ERR_INVALID_ARG.
+ * Selection (top-k, ties to the lower index) is the same under every rule. */
+#define MOE_WEIGHTS_SOFTMAX_TOPK 0
+#define MOE_WEIGHTS_SOFTMAX_ALL 1
+#define MOE_WEIGHTS_SIGMOID 2
+#define MOE_ACT_SILU 0
+#define MOE_ACT_SIGMOID 1
+
+typedef struct {
+    int weights;
+    int activation;
+    double capacity_factor;
+} moe_variant;
+
+/* moe_forward_ex under a layer variant (variant NULL: the method).  Same
+ * workspace as moe_forward_ex. */
+MOE_API moe_status moe_forward_variant(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                                       const moe_bf16 *Wg, const float *router_bias,
+                                       const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2,
+                                       int d_ff_shared, const moe_bf16 *Ws1, const moe_bf16 *Ws3,
+                                       const moe_bf16 *Ws2, const moe_variant *variant, float *out,
+                                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_route with the gate-weight rule `weights` (MOE_WEIGHTS_*). */
+MOE_API moe_status moe_route_variant(int T, int d, int E, int k, const moe_bf16 *x,
+                                     const moe_bf16 *Wg, const float *router_bias, int weights,
+                                     int32_t *idx, float *w, int32_t *counts, void *ws,
+                                     size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer with FP8 expert weights ("Mistral 8x7B SMoE" (jsqmd.com)
+ * deployment section: quantised experts, the router kept in higher
+ * precision).  Each expert weight is an e4m3 code (OCP 8-bit floating point
+ * E4M3, no infinities; raw bytes) times an fp32 scale of its row:
+ *   W1[e,f,i] = s1[e,f] * e4m3(W1q[e,f,i])   W1q, W3q [E,d_ff,d], s1, s3 [E,d_ff]
+ *   W2[e,o,f] = s2[e,o] * e4m3(W2q[e,o,f])   W2q [E,d,d_ff], s2 [E,d]
+ * x, Wg and router_bias are those of moe_forward_ex (bf16 router).  Inside,
+ * the token rows given to the experts and the hidden activations H are fp16
+ * (every e4m3 value is exact in fp16; x and H must stay within +-65504).
+ * No shared expert.  Same workspace as moe_forward.  Streaming half the
+ * weight bytes of bf16 is what this path is for: decode-sized batches,
+ * where the layer is bound by HBM bandwidth. */
+MOE_API moe_status moe_forward_fp8(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                                   const moe_bf16 *Wg, const float *router_bias,
+                                   const uint8_t *W1q, const float *s1, const uint8_t *W3q,
+                                   const float *s3, const uint8_t *W2q, const float *s2,
+                                   float *out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* moe_expert_ffn for callers that cannot allocate device memory: the same
  * computation, arguments and results as moe_expert_ffn, minus the workspace.
  * The pages have no counterpart of this entry point; it exists for code that
  * may not call cudaMalloc (a plugin handed only its tensors by a host program
  * that owns all device memory, or a loop that must stay out of the
  * allocator), which still owns x_perm, offsets, the weights and y_perm.
- *   The intermediate H [S, d_ff] bf16 lives in a fixed 32 MiB device array
- *   inside the library (every GPU that loads the library keeps it until the
- *   process exits): S * d_ff * 2 must be at most 32 MiB - 256 bytes, larger
- *   sizes return MOE_ERR_WORKSPACE.  Nothing is allocated and no allocating
- *   routine is called.
+ *   Its scratch (an error word, the expert kernel's readiness counters and
+ *   the intermediate H [S, d_ff] bf16) lives in one fixed device array of
+ *   MOE_STATIC_SCRATCH_BYTES inside the library; every GPU that loads the
+ *   library keeps it until the process exits.  A call needs
+ *     256 + align256(4 * (ceil(S/32) + E) * d_ff/128) + 2 * S * d_ff
+ *   bytes of it (moe_expert_ffn_static_bytes); larger sizes return
+ *   MOE_ERR_WORKSPACE before anything is launched.  Nothing is allocated and
+ *   no allocating routine is called.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The lookup is repeated after the device's
+ *   context has changed (cudaDeviceReset).
  *   All calls share the one array: calls that may overlap on the GPU (other
  *   streams, other host threads) race on it and must be serialised by the
- *   caller.  The array keeps the last call's contents; the call clears its
- *   error word itself.  The device error word of this entry point is not
- *   readable through moe_get_device_error. */
+ *   caller.  The array keeps the last call's contents; every call clears the
+ *   error word and the counters itself.  The error word is read with
+ *   moe_expert_ffn_static_error. */
+#define MOE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
 MOE_API moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
                                          const int32_t *offsets, const moe_bf16 *W1,
                                          const moe_bf16 *W3, const moe_bf16 *W2, float *y_perm,
                                          moe_stream_t stream);
+
+/* Bytes of the fixed array a moe_expert_ffn_static call of these sizes needs
+ * (the formula above); 0 for sizes outside the supported range.  The pages
+ * have no counterpart. */
+MOE_API size_t moe_expert_ffn_static_bytes(int S, int E, int d_ff);
+
+/* Waits for `stream`, then reads the error word of the fixed array of the
+ * current device (what the last moe_expert_ffn_static call on it left) into
+ * *code (may be NULL).  Returns like moe_get_device_error.  Allocates
+ * nothing.  The pages have no counterpart. */
+MOE_API moe_status moe_expert_ffn_static_error(uint32_t *code, moe_stream_t stream);
 
 /* Number of events moe_forward_traced records. */
 #define MOE_TRACE_EVENTS 6
@@ -215,6 +299,17 @@ MOE_API moe_status moe_forward_traced(int T, int d, int E, int d_ff, int k, cons
                                       int d_ff_shared, const moe_bf16 *Ws1, const moe_bf16 *Ws3,
                                       const moe_bf16 *Ws2, float *out, void *ws, size_t ws_bytes,
                                       moe_stream_t stream, void *const *events, int n_events);
+
+/* moe_forward_fp8 with caller-created CUDA events recorded at the kernel
+ * boundaries, with the meaning of moe_forward_traced's events (events[3] and
+ * events[4] mark the same point: there is no shared expert). */
+MOE_API moe_status moe_forward_fp8_traced(int T, int d, int E, int d_ff, int k,
+                                          const moe_bf16 *x, const moe_bf16 *Wg,
+                                          const float *router_bias, const uint8_t *W1q,
+                                          const float *s1, const uint8_t *W3q, const float *s3,
+                                          const uint8_t *W2q, const float *s2, float *out,
+                                          void *ws, size_t ws_bytes, moe_stream_t stream,
+                                          void *const *events, int n_events);
 
 /* Waits for `stream`, then reads the device error word of workspace `ws`
  * into *code (may be NULL).  Returns MOE_OK if it is zero, MOE_ERR_TIMEOUT

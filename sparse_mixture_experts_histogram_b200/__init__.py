@@ -7,17 +7,29 @@ FLOP/byte/parameter closed forms used for throughput and roofline numbers.
 """
 from .binding import (  # noqa: F401
     ABI_FUNCTIONS,
+    ACT_SIGMOID,
+    ACT_SILU,
+    WEIGHTS_SIGMOID,
+    WEIGHTS_SOFTMAX_ALL,
+    WEIGHTS_SOFTMAX_TOPK,
     MoEError,
+    MoEVariant,
     load_library,
     moe_combine,
     moe_expert_ffn,
     moe_expert_ffn_static,
+    moe_expert_ffn_static_bytes,
+    moe_expert_ffn_static_error,
     moe_forward,
     moe_forward_ex,
+    moe_forward_fp8,
+    moe_forward_fp8_traced,
     moe_forward_traced,
+    moe_forward_variant,
     moe_get_device_error,
     moe_permute,
     moe_route,
+    moe_route_variant,
     moe_status_string,
     moe_workspace_size,
     moe_workspace_size_ex,

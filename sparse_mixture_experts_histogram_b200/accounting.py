@@ -55,22 +55,33 @@ def active_flops(T: int, d: int, E: int, d_ff: int, k: int, d_ff_shared: int = 0
     return 2 * 3 * d * d_ff * k * T + 2 * T * d * E + 2 * 3 * d * d_ff_shared * T
 
 
+def fp8_scale_bytes(d: int, d_ff: int) -> int:
+    """fp32 row scales of one FP8 expert: W1 and W3 rows (d_ff each), W2 rows (d)."""
+    return 4 * (2 * d_ff + d)
+
+
 def algorithmic_bytes(T: int, d: int, E: int, d_ff: int, k: int, experts_hit: int,
-                      d_ff_shared: int = 0) -> int:
-    """Minimum HBM bytes of one layer call: hit experts' bf16 weights, bf16 Wg,
-    bf16 x read, fp32 out written (+ the shared expert's bf16 weights)."""
-    return (2 * experts_hit * expert_params(d, d_ff) + 2 * d * E + 2 * T * d + 4 * T * d
-            + 2 * expert_params(d, d_ff_shared))
+                      d_ff_shared: int = 0, fp8: bool = False) -> int:
+    """Minimum HBM bytes of one layer call: hit experts' weights (bf16, or e4m3
+    codes plus their fp32 row scales), bf16 Wg, bf16 x read, fp32 out written
+    (+ the shared expert's bf16 weights)."""
+    wb = (experts_hit * (expert_params(d, d_ff) + fp8_scale_bytes(d, d_ff)) if fp8
+          else 2 * experts_hit * expert_params(d, d_ff))
+    return (wb + 2 * d * E + 2 * T * d + 4 * T * d + 2 * expert_params(d, d_ff_shared))
 
 
-def ffn_bytes(T: int, d: int, d_ff: int, k: int, experts_hit: int, d_ff_shared: int = 0) -> int:
-    """Algorithmic bytes of the expert feed-forward kernel (both projections):
-    bf16 W1, W3, W2 of the hit experts + the permuted bf16 rows read (S = T*k
-    rows of d) + the fp32 expert outputs written (S rows of d).  The hidden
-    activations H are an intermediate and are not counted.  A shared expert
-    is its own launch over the T token rows with its own weights."""
-    S = T * k
-    return 2 * 3 * experts_hit * d * d_ff + 2 * S * d + 4 * S * d
+def ffn_bytes(T: int, d: int, d_ff: int, k: int, experts_hit: int, d_ff_shared: int = 0,
+              fp8: bool = False) -> int:
+    """Algorithmic bytes of the routed experts' feed-forward (both
+    projections): bf16 W1, W3, W2 of the hit experts, the bf16 token rows
+    read once (T rows of d) and the fp32 layer output written once (T rows of
+    d).  The k routed copies of each row, the hidden activations H and the
+    per-slot expert outputs are implementation bytes and are not counted.  A
+    shared expert is its own launch over the T token rows with its own
+    weights."""
+    if fp8:
+        return experts_hit * (3 * d * d_ff + fp8_scale_bytes(d, d_ff)) + 2 * T * d + 4 * T * d
+    return 2 * 3 * experts_hit * d * d_ff + 2 * T * d + 4 * T * d
 
 
 def ffn_flops(T: int, d: int, d_ff: int, k: int) -> int:

@@ -27,10 +27,23 @@ DEVERR_BITS = {0x1: "TIMEOUT_TMA", 0x2: "TIMEOUT_MMA", 0x4: "TIMEOUT_EPI", 0x8: 
 ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "moe_permute",
                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_ex",
                  "moe_forward_traced", "moe_get_device_error", "moe_status_string",
-                 "moe_expert_ffn_static")
+                 "moe_expert_ffn_static", "moe_expert_ffn_static_bytes",
+                 "moe_expert_ffn_static_error", "moe_forward_variant", "moe_route_variant",
+                 "moe_forward_fp8", "moe_forward_fp8_traced")
 TRACE_EVENTS = 6
 #: What each of moe_forward_traced's events marks (event i = start of stage i).
 TRACE_STAGES = ("route", "scatter", "expert_ffn", "shared_ffn", "combine")
+
+
+#: Gate-weight rules and expert activations of ``moe_variant`` (include/moe.h).
+WEIGHTS_SOFTMAX_TOPK, WEIGHTS_SOFTMAX_ALL, WEIGHTS_SIGMOID = 0, 1, 2
+ACT_SILU, ACT_SIGMOID = 0, 1
+
+
+class MoEVariant(ctypes.Structure):
+    """``moe_variant``: gate-weight rule, expert activation, capacity factor."""
+    _fields_ = [("weights", ctypes.c_int), ("activation", ctypes.c_int),
+                ("capacity_factor", ctypes.c_double)]
 
 
 class MoEError(RuntimeError):
@@ -67,8 +80,15 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
             "moe_forward": (_I, [_I] * 5 + [_P] * 7 + [_SZ, _P]),
             "moe_forward_ex": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P]),
             "moe_forward_traced": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 5 + [_SZ, _P, _P, _I]),
+            "moe_forward_variant": (_I, [_I] * 5 + [_P] * 6 + [_I] + [_P] * 3 + [_P, _P, _P, _SZ,
+                                                                               _P]),
+            "moe_route_variant": (_I, [_I] * 4 + [_P] * 3 + [_I] + [_P] * 4 + [_SZ, _P]),
+            "moe_forward_fp8": (_I, [_I] * 5 + [_P] * 11 + [_SZ, _P]),
+            "moe_forward_fp8_traced": (_I, [_I] * 5 + [_P] * 11 + [_SZ, _P, _P, _I]),
             "moe_get_device_error": (_I, [_P, _P, _P]),
             "moe_expert_ffn_static": (_I, [_I] * 4 + [_P] * 6 + [_P]),
+            "moe_expert_ffn_static_bytes": (_SZ, [_I] * 3),
+            "moe_expert_ffn_static_error": (_I, [_P, _P]),
             "moe_status_string": (ctypes.c_char_p, [_I]),
         }
         for name, (res, args) in sig.items():
@@ -146,10 +166,24 @@ def moe_expert_ffn(S, d, E, d_ff, x_perm, offsets, W1, W3, W2, y_perm, ws, strea
 def moe_expert_ffn_static(S, d, E, d_ff, x_perm, offsets, W1, W3, W2, y_perm, stream=None):
     """moe_expert_ffn without a workspace argument, for callers that cannot
     allocate device memory: the intermediate lives in a fixed 32 MiB array
-    inside the library (see include/moe.h for its limit and sharing rules)."""
+    inside the library (see include/moe.h for its limit and sharing rules;
+    moe_expert_ffn_static_bytes gives a call's need)."""
     _check(load_library().moe_expert_ffn_static(S, d, E, d_ff, _ptr(x_perm), _ptr(offsets),
                                                 _ptr(W1), _ptr(W3), _ptr(W2), _ptr(y_perm),
                                                 _stream(stream)), "moe_expert_ffn_static")
+
+
+def moe_expert_ffn_static_bytes(S, E, d_ff) -> int:
+    """Bytes of the fixed array a moe_expert_ffn_static call needs (0: unsupported)."""
+    return int(load_library().moe_expert_ffn_static_bytes(S, E, d_ff))
+
+
+def moe_expert_ffn_static_error(stream=None) -> tuple[int, int]:
+    """(status, error word) the last moe_expert_ffn_static call on the current
+    device left in the fixed array."""
+    code = ctypes.c_uint32(0)
+    st = load_library().moe_expert_ffn_static_error(ctypes.byref(code), _stream(stream))
+    return int(st), int(code.value)
 
 
 def moe_combine(T, d, k, y_perm, row_of_slot, w, shared_y, out, stream=None):
@@ -169,6 +203,50 @@ def moe_forward_ex(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared
                                          _ptr(W1), _ptr(W3), _ptr(W2), d_ff_shared, _ptr(Ws1),
                                          _ptr(Ws3), _ptr(Ws2), _ptr(out), _ptr(ws),
                                          _ws_bytes(ws), _stream(stream)), "moe_forward_ex")
+
+
+def moe_forward_variant(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,
+                        Ws2, variant, out, ws, stream=None):
+    """``variant``: a MoEVariant, a (weights, activation, capacity_factor)
+    tuple, or None for the method."""
+    if variant is not None and not isinstance(variant, MoEVariant):
+        variant = MoEVariant(*variant)
+    vp = None if variant is None else ctypes.cast(ctypes.pointer(variant), ctypes.c_void_p)
+    _check(load_library().moe_forward_variant(T, d, E, d_ff, k, _ptr(x), _ptr(Wg),
+                                              _ptr(router_bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                                              d_ff_shared, _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), vp,
+                                              _ptr(out), _ptr(ws), _ws_bytes(ws),
+                                              _stream(stream)), "moe_forward_variant")
+
+
+def moe_route_variant(T, d, E, k, x, Wg, router_bias, weights, idx, w, counts, ws, stream=None):
+    _check(load_library().moe_route_variant(T, d, E, k, _ptr(x), _ptr(Wg), _ptr(router_bias),
+                                            int(weights), _ptr(idx), _ptr(w), _ptr(counts),
+                                            _ptr(ws), _ws_bytes(ws), _stream(stream)),
+           "moe_route_variant")
+
+
+def moe_forward_fp8(T, d, E, d_ff, k, x, Wg, router_bias, W1q, s1, W3q, s3, W2q, s2, out, ws,
+                    stream=None):
+    """FP8 experts: W*q uint8 e4m3 codes, s* fp32 row scales (include/moe.h)."""
+    _check(load_library().moe_forward_fp8(T, d, E, d_ff, k, _ptr(x), _ptr(Wg), _ptr(router_bias),
+                                          _ptr(W1q), _ptr(s1), _ptr(W3q), _ptr(s3), _ptr(W2q),
+                                          _ptr(s2), _ptr(out), _ptr(ws), _ws_bytes(ws),
+                                          _stream(stream)), "moe_forward_fp8")
+
+
+def moe_forward_fp8_traced(T, d, E, d_ff, k, x, Wg, router_bias, W1q, s1, W3q, s3, W2q, s2, out,
+                           ws, events, stream=None):
+    if len(events) != TRACE_EVENTS:
+        raise ValueError(f"need {TRACE_EVENTS} events")
+    arr = (ctypes.c_void_p * TRACE_EVENTS)(
+        *[e if isinstance(e, int) else e.cuda_event for e in events])
+    _check(load_library().moe_forward_fp8_traced(T, d, E, d_ff, k, _ptr(x), _ptr(Wg),
+                                                 _ptr(router_bias), _ptr(W1q), _ptr(s1),
+                                                 _ptr(W3q), _ptr(s3), _ptr(W2q), _ptr(s2),
+                                                 _ptr(out), _ptr(ws), _ws_bytes(ws),
+                                                 _stream(stream), arr, TRACE_EVENTS),
+           "moe_forward_fp8_traced")
 
 
 def moe_forward_traced(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,

@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -19,7 +20,9 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, ranks counter @8,
-                                      // partial outputs per row of the expert kernel @12
+                                      // partial outputs per row of the expert kernel @12,
+                                      // work counters of the routed @16 and shared @20
+                                      // expert kernels
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -134,6 +137,37 @@ cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, ui
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_tmap_e4m3(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols)
+{
+    std::call_once(g_encode_once, load_encode);
+    if (g_encode == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_f16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows)
+{
+    std::call_once(g_encode_once, load_encode);
+    if (g_encode == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 int device_sm_count()
 {
     int dev = 0;
@@ -180,9 +214,11 @@ const char *moe_status_string(moe_status s)
 static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
                              const float *bias, int32_t *idx, float *w, int32_t *counts,
                              int32_t *offsets, uint8_t *ws, const Layout &L, cudaStream_t s,
-                             bool slots = false)
+                             bool slots = false, int wmode = 0, int cap = -1)
 {
     RouteLaunch a{};
+    a.wmode = wmode;
+    a.cap = cap;
     a.T = T;
     a.d = d;
     a.E = E;
@@ -209,15 +245,29 @@ static moe_status route_impl(int T, int d, int E, int k, const moe_bf16 *x, cons
     return from_cuda(launch_route(a, s));
 }
 
+moe_status moe_route_variant(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
+                             const float *router_bias, int weights, int32_t *idx, float *w,
+                             int32_t *counts, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 moe_status moe_route(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
                      const float *router_bias, int32_t *idx, float *w, int32_t *counts, void *ws,
                      size_t ws_bytes, moe_stream_t stream)
 {
+    return moe_route_variant(T, d, E, k, x, Wg, router_bias, MOE_WEIGHTS_SOFTMAX_TOPK, idx, w,
+                             counts, ws, ws_bytes, stream);
+}
+
+moe_status moe_route_variant(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf16 *Wg,
+                             const float *router_bias, int weights, int32_t *idx, float *w,
+                             int32_t *counts, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (weights < 0 || weights > 2) return MOE_ERR_INVALID_ARG;
     moe_status st = check_shapes(T, d, E, 128, k, 0);
     if (st != MOE_OK) return st;
-    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(idx) || !ok_ptr(w) || !ok_ptr(counts) || !ok_ptr(ws))
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(idx) || !ok_ptr(w) || !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
     if (router_bias != nullptr && !aligned16(router_bias)) return MOE_ERR_INVALID_ARG;
+    if (counts != nullptr && !aligned16(counts)) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_workspace_size(T, d, E, 128, k)) return MOE_ERR_WORKSPACE;
     const Layout L = forward_layout(T, d, E, 128, k, 0);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -225,7 +275,7 @@ moe_status moe_route(int T, int d, int E, int k, const moe_bf16 *x, const moe_bf
     st = from_cuda(cudaMemsetAsync(wsb, 0, L.zero_bytes, s));
     if (st != MOE_OK) return st;
     return route_impl(T, d, E, k, x, Wg, router_bias, idx, w, counts,
-                      reinterpret_cast<int32_t *>(wsb + L.offsets), wsb, L, s);
+                      reinterpret_cast<int32_t *>(wsb + L.offsets), wsb, L, s, false, weights);
 }
 
 moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int32_t *idx,
@@ -257,6 +307,7 @@ moe_status moe_permute(int T, int d, int E, int k, const moe_bf16 *x, const int3
     st = from_cuda(launch_ranks(r, s));
     if (st != MOE_OK) return st;
     ScatterLaunch c{};
+    c.cap = -1;
     c.T = T;
     c.d = d;
     c.E = E;
@@ -277,9 +328,11 @@ static moe_status mark(void *const *events, int i, cudaStream_t s);
 static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const moe_bf16 *x,
                            const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
                            const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *h_ready,
-                           uint32_t *err, cudaStream_t s, bool pdl, int ksplit)
+                           uint32_t *sched, uint32_t *err, cudaStream_t s, bool pdl, int ksplit,
+                           int act = 0)
 {
     FfnLaunch f{};
+    f.act = act;
     f.E = E;
     f.d = d;
     f.d_ff = d_ff;
@@ -294,6 +347,7 @@ static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const mo
     f.H = H;
     f.Y = y;
     f.h_ready = h_ready;
+    f.sched = sched;
     f.err = err;
     f.pdl = pdl;
     return from_cuda(launch_ffn(f, s));
@@ -319,7 +373,8 @@ moe_status moe_expert_ffn(int S, int d, int E, int d_ff, const moe_bf16 *x_perm,
     return ffn_impl(S, d, E, d_ff, S, x_perm, offsets, W1, W3, W2,
                     reinterpret_cast<moe_bf16 *>(wsb + kHeaderBytes + ctr), y_perm,
                     reinterpret_cast<uint32_t *>(wsb + kHeaderBytes),
-                    reinterpret_cast<uint32_t *>(wsb), s, false, 1);
+                    reinterpret_cast<uint32_t *>(wsb + 16), reinterpret_cast<uint32_t *>(wsb), s,
+                    false, 1);
 }
 
 moe_status moe_combine(int T, int d, int k, const float *y_perm, const int32_t *row_of_slot,
@@ -362,10 +417,23 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
                                const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
                                const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
                                float *out, void *ws, size_t ws_bytes, moe_stream_t stream,
-                               void *const *events)
+                               void *const *events, const moe_variant *variant = nullptr)
 {
     moe_status st = check_shapes(T, d, E, d_ff, k, d_ff_shared);
     if (st != MOE_OK) return st;
+    const int wmode = variant ? variant->weights : MOE_WEIGHTS_SOFTMAX_TOPK;
+    const int act = variant ? variant->activation : MOE_ACT_SILU;
+    const double cf = variant ? variant->capacity_factor : 0.0;
+    if (wmode < 0 || wmode > 2 || act < 0 || act > 1 || !(cf >= 0.0) || cf > 1e9)
+        return MOE_ERR_INVALID_ARG;
+    // Per-expert capacity floor(cf * T * k / E); no expert ever receives more
+    // than T pairs, so a capacity of T or more drops nothing.
+    int cap = -1;
+    if (cf > 0.0) {
+        const double c = std::floor(cf * static_cast<double>(static_cast<long long>(T) * k) /
+                                    static_cast<double>(E));
+        if (c < static_cast<double>(T)) cap = static_cast<int>(c);
+    }
     if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) || !ok_ptr(out) ||
         !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
@@ -394,18 +462,23 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     // token list and its total, and the expert kernel derives the segment
     // starts and gathers the rows of x itself, so there is no permuted copy
     // of x and no scatter launch in between.
-    const bool narrow = ffn_small_supported(d);
+    // Dropping by capacity needs the token order of each expert's pairs,
+    // which only the token-ordered dispatch (ranks, scatter) keeps.
+    const bool narrow = ffn_small_supported(d) && cap < 0;
     // Overlapping launches pay off for small layers; for large ones they only
     // take SM slots early (measured: neutral to slightly negative).
     const bool pdl = events == nullptr && S <= 4096;
     if ((st = mark(events, 0, s)) != MOE_OK) return st;
     st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
-                    reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s, narrow);
+                    reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s, narrow, wmode,
+                    cap);
     if (st != MOE_OK) return st;
 
     if ((st = mark(events, 1, s)) != MOE_OK) return st;
     if (!narrow) {
         ScatterLaunch c{};
+        c.cap = cap;
+        c.offsets = offsets;
         c.T = T;
         c.d = d;
         c.E = E;
@@ -423,10 +496,13 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     }
 
     // A token never picks one expert twice, so no segment exceeds T rows.
-    const int ksplit = ffn_splits(S, E, d, d_ff);
+    // (The capacity path of a narrow layer runs the general expert kernel on
+    // the permuted copy, without a K split.)
+    const int ksplit = (cap >= 0 && ffn_small_supported(d)) ? 1 : ffn_splits(S, E, d, d_ff);
     if ((st = mark(events, 2, s)) != MOE_OK) return st;
     if (narrow) {
         FfnLaunch f{};
+        f.act = act;
         f.E = E;
         f.d = d;
         f.d_ff = d_ff;
@@ -451,7 +527,8 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         st = from_cuda(launch_ffn_small(f, ksplit, reinterpret_cast<int *>(wsb + 12), s));
     } else {
         st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
-                      reinterpret_cast<uint32_t *>(wsb + L.hready), err, s, pdl, ksplit);
+                      reinterpret_cast<uint32_t *>(wsb + L.hready),
+                      reinterpret_cast<uint32_t *>(wsb + 16), err, s, pdl, ksplit, act);
     }
     if (st != MOE_OK) return st;
 
@@ -461,7 +538,8 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
         float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
         st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys,
-                      reinterpret_cast<uint32_t *>(wsb + L.hready_s), err, s, false, 1);
+                      reinterpret_cast<uint32_t *>(wsb + L.hready_s),
+                      reinterpret_cast<uint32_t *>(wsb + 20), err, s, false, 1, act);
         if (st != MOE_OK) return st;
         shared_y = Ys;
     }
@@ -498,6 +576,133 @@ moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *
 {
     return forward_impl(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,
                         Ws2, out, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_variant(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                               const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
+                               const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
+                               const moe_bf16 *Ws1, const moe_bf16 *Ws3, const moe_bf16 *Ws2,
+                               const moe_variant *variant, float *out, void *ws, size_t ws_bytes,
+                               moe_stream_t stream)
+{
+    return forward_impl(T, d, E, d_ff, k, x, Wg, router_bias, W1, W3, W2, d_ff_shared, Ws1, Ws3,
+                        Ws2, out, ws, ws_bytes, stream, nullptr, variant);
+}
+
+static moe_status fp8_impl(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                           const moe_bf16 *Wg, const float *router_bias, const uint8_t *W1q,
+                           const float *s1, const uint8_t *W3q, const float *s3,
+                           const uint8_t *W2q, const float *s2, float *out, void *ws,
+                           size_t ws_bytes, moe_stream_t stream, void *const *events)
+{
+    moe_status st = check_shapes(T, d, E, d_ff, k, 0);
+    if (st != MOE_OK) return st;
+    if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(W1q) || !ok_ptr(W3q) || !ok_ptr(W2q) ||
+        !ok_ptr(s1) || !ok_ptr(s3) || !ok_ptr(s2) || !ok_ptr(out) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (router_bias != nullptr && !aligned16(router_bias)) return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_INVALID_ARG;
+    const Layout L = forward_layout(T, d, E, d_ff, k, 0);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    uint32_t *err = reinterpret_cast<uint32_t *>(wsb);
+    const int S = T * k;
+    int32_t *idx = reinterpret_cast<int32_t *>(wsb + L.idx);
+    float *w = reinterpret_cast<float *>(wsb + L.w);
+    int32_t *offsets = reinterpret_cast<int32_t *>(wsb + L.offsets);
+    int32_t *row = reinterpret_cast<int32_t *>(wsb + L.row);
+    float *Y = reinterpret_cast<float *>(wsb + L.Y);
+    st = from_cuda(cudaMemsetAsync(wsb, 0, L.zero_bytes, s));
+    if (st != MOE_OK) return st;
+    const bool pdl = events == nullptr && S <= 4096;
+    // Router in bf16 (unchanged), token-ordered dispatch with the rows
+    // converted to fp16, the FP8 expert kernel, the combine.
+    if ((st = mark(events, 0, s)) != MOE_OK) return st;
+    st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
+                    reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s);
+    if (st != MOE_OK) return st;
+    if ((st = mark(events, 1, s)) != MOE_OK) return st;
+    ScatterLaunch c{};
+    c.cap = -1;
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.k = k;
+    c.x = x;
+    c.idx = idx;
+    c.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
+    c.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
+    c.x_perm = reinterpret_cast<uint16_t *>(wsb + L.xperm);
+    c.row_of_slot = row;
+    c.err = err;
+    c.pdl = pdl;
+    c.to_f16 = true;
+    st = from_cuda(launch_scatter(c, s));
+    if (st != MOE_OK) return st;
+    // The workspace holds ffn_splits(...) partial outputs per row.
+    const int ksplit = std::min(down_ksplit(S, E, d, d_ff), ffn_splits(S, E, d, d_ff));
+    FfnFp8Launch f{};
+    f.f.E = E;
+    f.f.d = d;
+    f.f.d_ff = d_ff;
+    f.f.S = S;
+    f.f.max_rows = T;
+    f.f.ksplit = ksplit;
+    f.f.offsets = offsets;
+    f.f.x = reinterpret_cast<const uint16_t *>(wsb + L.xperm);
+    f.f.H = reinterpret_cast<uint16_t *>(wsb + L.H);
+    f.f.Y = Y;
+    f.f.h_ready = reinterpret_cast<uint32_t *>(wsb + L.hready);
+    f.f.err = err;
+    f.f.pdl = pdl;
+    f.q1 = W1q;
+    f.q3 = W3q;
+    f.q2 = W2q;
+    f.s1 = s1;
+    f.s3 = s3;
+    f.s2 = s2;
+    if ((st = mark(events, 2, s)) != MOE_OK) return st;
+    st = from_cuda(launch_ffn_fp8(f, s));
+    if (st != MOE_OK) return st;
+    if ((st = mark(events, 3, s)) != MOE_OK) return st;
+    if ((st = mark(events, 4, s)) != MOE_OK) return st;
+    CombineLaunch cb{};
+    cb.T = T;
+    cb.d = d;
+    cb.k = k;
+    cb.ksplit = ksplit;
+    cb.y = Y;
+    cb.row_of_slot = row;
+    cb.w = w;
+    cb.out = out;
+    cb.pdl = false;
+    st = from_cuda(launch_combine(cb, s));
+    if (st != MOE_OK) return st;
+    return mark(events, 5, s);
+}
+
+moe_status moe_forward_fp8(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                           const moe_bf16 *Wg, const float *router_bias, const uint8_t *W1q,
+                           const float *s1, const uint8_t *W3q, const float *s3,
+                           const uint8_t *W2q, const float *s2, float *out, void *ws,
+                           size_t ws_bytes, moe_stream_t stream)
+{
+    return fp8_impl(T, d, E, d_ff, k, x, Wg, router_bias, W1q, s1, W3q, s3, W2q, s2, out, ws,
+                    ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_fp8_traced(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
+                                  const moe_bf16 *Wg, const float *router_bias,
+                                  const uint8_t *W1q, const float *s1, const uint8_t *W3q,
+                                  const float *s3, const uint8_t *W2q, const float *s2,
+                                  float *out, void *ws, size_t ws_bytes, moe_stream_t stream,
+                                  void *const *events, int n_events)
+{
+    if (events == nullptr || n_events != MOE_TRACE_EVENTS) return MOE_ERR_INVALID_ARG;
+    return fp8_impl(T, d, E, d_ff, k, x, Wg, router_bias, W1q, s1, W3q, s3, W2q, s2, out, ws,
+                    ws_bytes, stream, events);
 }
 
 moe_status moe_forward_traced(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,

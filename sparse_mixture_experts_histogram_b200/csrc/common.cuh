@@ -76,6 +76,7 @@ struct DispatchOut {
     int32_t *counts;     // [E] per-expert pair counts, or nullptr
     uint32_t *done;      // tile completion counter (zero at kernel start)
     int ntiles;
+    int cap;             // per-expert capacity (segments hold min(count, cap) rows), or -1
 };
 
 // Called by the 128 threads of one routing tile after they filled sm.sel.
@@ -169,6 +170,12 @@ __device__ __forceinline__ void dispatch_tile(DispatchSmem &sm, int row, int til
     if (q == 0) {
         const int per = (E + 31) >> 5;
         const int base = lane * per;
+        // With a capacity an expert's segment holds only its first `cap`
+        // pairs in token order.
+        if (o.cap >= 0)
+            for (int i = 0; i < per; ++i)
+                if (base + i < E) sm.tot[base + i] = min(sm.tot[base + i], o.cap);
+        __syncwarp();
         int local = 0;
         for (int i = 0; i < per; ++i)
             if (base + i < E) local += sm.tot[base + i];

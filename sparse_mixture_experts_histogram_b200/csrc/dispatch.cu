@@ -9,6 +9,7 @@
 // Method: "MoE" (theaiera.top, LLMs-from-scratch ch.10) sec. 10.4 gathers,
 // per expert, the tokens that selected it (mask / nonzero / index_select);
 // here every expert's tokens become one contiguous, token-ordered segment.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -50,12 +51,15 @@ __global__ void __launch_bounds__(kTileTokens) ranks_kernel(const RanksParams p)
 
 struct ScatterParams {
     int T, d, E, k;
+    int cap;             // per-expert capacity, or -1 (dropless)
+    const int32_t *offsets;  // [E+1] segment starts (read when cap >= 0)
     const uint4 *x;
     const int32_t *idx, *rank, *tilebase;
     uint4 *x_perm;
     int32_t *row_of_slot;
     uint32_t *err;
     int S;
+    int to_f16;  // convert the rows to fp16 on the way
     int chunks;  // 16-byte-vector chunks of kScatterVec*32 per row
 };
 
@@ -80,12 +84,16 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
         const size_t s = static_cast<size_t>(t) * p.k + lane;
         const int e = p.idx[s];
         const int r = p.rank[s];
+        bool dropped = false;
         if (e >= 0 && e < p.E && r >= 0) {
             const int row = p.tilebase[static_cast<size_t>(t / kTileTokens) * p.E + e] + r;
-            if (row >= 0 && row < p.S) my_row = row;
+            // With a capacity, a pair ranked at or beyond it in its expert's
+            // token order is dropped: no row, nothing added for this slot.
+            if (p.cap >= 0 && row - p.offsets[e] >= p.cap) dropped = true;
+            else if (row >= 0 && row < p.S) my_row = row;
         }
         if (c == 0) {
-            if (my_row < 0) atomicOr(p.err, kErrIndex);
+            if (my_row < 0 && !dropped) atomicOr(p.err, kErrIndex);
             p.row_of_slot[s] = my_row;
         }
     }
@@ -99,6 +107,19 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
     for (int u = 0; u < kScatterVec; ++u) {
         const int v = (c * kScatterVec + u) * 32 + lane;
         if (v < nv) val[u] = __ldg(src + v);
+    }
+    if (p.to_f16) {
+#pragma unroll
+        for (int u = 0; u < kScatterVec; ++u) {
+            uint32_t *w = reinterpret_cast<uint32_t *>(&val[u]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float lo = __uint_as_float(w[i] << 16);
+                const float hi = __uint_as_float(w[i] & 0xffff0000u);
+                const __half2 h = __floats2half2_rn(lo, hi);
+                w[i] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+        }
     }
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
@@ -130,6 +151,7 @@ cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s)
     p.dout.counts = nullptr;
     p.dout.done = a.done;
     p.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
+    p.dout.cap = -1;
     ranks_kernel<<<p.dout.ntiles, kTileTokens, 0, s>>>(p);
     return cudaGetLastError();
 }
@@ -141,6 +163,8 @@ cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s)
     p.d = a.d;
     p.E = a.E;
     p.k = a.k;
+    p.cap = a.cap;
+    p.offsets = a.offsets;
     p.x = reinterpret_cast<const uint4 *>(a.x);
     p.idx = a.idx;
     p.rank = a.rank;
@@ -149,6 +173,7 @@ cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s)
     p.row_of_slot = a.row_of_slot;
     p.err = a.err;
     p.S = a.T * a.k;
+    p.to_f16 = a.to_f16 ? 1 : 0;
     const int nv = a.d / 8;
     p.chunks = (nv + 32 * kScatterVec - 1) / (32 * kScatterVec);
     const long long warps = static_cast<long long>(a.T) * p.chunks;

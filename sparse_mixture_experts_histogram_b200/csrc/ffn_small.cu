@@ -97,6 +97,7 @@ struct SmallParams {
     int x_rows;
     float *Y;               // [nsplit, S, d]
     uint32_t *err;
+    int act;                // expert activation: 0 silu(g) * b, 1 sigmoid(g) * b
 };
 
 struct Item {
@@ -548,7 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int jt = 0; jt < 8; ++jt) {
                         if (c0 + jt < it.valid) {
                             const float gv = __uint_as_float(a[jt]);
-                            const float h = __fdividef(gv * __uint_as_float(b[jt]), 1.0f + __expf(-gv));
+                            const float bv = __uint_as_float(b[jt]);
+                            const float h = __fdividef(p.act ? bv : gv * bv, 1.0f + __expf(-gv));
                             // row c0+jt (c0 is a multiple of 8, so the row's swizzle
                             // phase is jt), column f, 128-byte-swizzled layout
                             *reinterpret_cast<__nv_bfloat16 *>(hrow + jt * 128 + ((hchunk ^ jt) << 4)) =
@@ -619,6 +621,7 @@ cudaError_t launch_small_cfg(const FfnLaunch &a, int nsplit_max, int *nsplit_out
                              static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return e;
     SmallParams p{};
+    p.act = a.act;
     p.E = a.E;
     p.d = a.d;
     p.d_ff = a.d_ff;

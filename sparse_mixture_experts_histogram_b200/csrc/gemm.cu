@@ -79,6 +79,7 @@ struct FfnParams {
     uint32_t *h_ready;      // [tiles, d_ff/128]: epilogue warps done with (token tile, H block)
     uint32_t *err;
     int stream_weights;     // each weight block feeds one token tile: L2 evict-first
+    int act;                // expert activation: 0 silu(g) * b, 1 sigmoid(g) * b
 };
 
 struct Unit {
@@ -417,7 +418,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                     for (int j = 0; j < 32; ++j) {
                         if (c0 + j < w.valid) {
                             const float g = __uint_as_float(a[j]);
-                            const float h = __fdividef(g * __uint_as_float(b[j]), 1.0f + __expf(-g));
+                            const float bv = __uint_as_float(b[j]);
+                            const float h = __fdividef(p.act ? bv : g * bv, 1.0f + __expf(-g));
                             p.H[static_cast<size_t>(w.r0 + c0 + j) * p.d_ff + f] =
                                 __float2bfloat16_rn(h);
                         }
@@ -490,6 +492,7 @@ cudaError_t launch_ffn_cfg(const FfnLaunch &a, cudaStream_t s)
     p.h_ready = a.h_ready;
     p.err = a.err;
     p.stream_weights = a.max_rows <= BN ? 1 : 0;
+    p.act = a.act;
     // Upper bound of the work units: every segment rounds up to whole tiles.
     const long long tiles = (static_cast<long long>(a.S) + BN - 1) / BN + E;
     const long long units = tiles * (a.d_ff / 128) + tiles * ((a.d + 255) / 256) * p.ksplit;
@@ -548,6 +551,8 @@ int down_ksplit(int S, int E_seg, int d, int d_ff)
 
 cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s)
 {
+    if (a.sched != nullptr && ffn_pair_eligible(a.S, a.offsets ? a.E : 1, a.ksplit))
+        return launch_ffn_pair(a, a.sched, s);
     switch (ffn_token_tile(a.S, a.offsets ? a.E : 1)) {
     case 32: return launch_ffn_cfg<32, 6>(a, s);
     case 64: return launch_ffn_cfg<64, 5>(a, s);

@@ -1,0 +1,617 @@
+// gemm_fp8.cu -- the experts' feed-forward with FP8 weights: e4m3 codes with
+// one fp32 scale per weight row, W = scale[row] * e4m3(code).  One
+// persistent kernel on the 5th-generation tensor cores.
+//
+// The unit structure is that of the bf16 expert kernel (gemm.cu): up units
+// (expert, 128 W1 and W3 rows, token tile) then down units (expert, two
+// 128-row W2 blocks, token tile, K range), weights on the MMA's M side and
+// the segment's rows on N.  What differs is the operand path:
+//   * TMA brings each 128 x 64 weight tile as e4m3 bytes (8 KB, 64-byte
+//     swizzle) -- half the bytes of bf16, the point of FP8 where the layer
+//     streams its weights from HBM (decode);
+//   * four converter warps widen the tiles to fp16 (exact: every e4m3 value is
+//     an fp16 value) straight into the 128-byte-swizzled K-major layout the
+//     MMA reads, then release the raw stage and mark the operand stage full;
+//   * the MMA is kind::f16 with fp16 A and B (the token rows x_perm and the
+//     hidden activations H are fp16 in this path) and fp32 accumulators;
+//   * the epilogue multiplies each accumulator row by its weight row's scale
+//     before the activation (up units) or before the fp32 output (down units).
+//
+// Pipelines: a deep ring of input stages (the two e4m3 weight tiles of a K
+// step, the step's fp16 token rows) keeps enough bytes in flight to stream
+// HBM; the converters fill a ring of two fp16 operand stages from it.  An
+// input stage is free once the converters have read its tiles and the MMAs
+// its token rows.
+//
+// Roles: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warps 6..9 converters.
+//
+// Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
+// architecture" (jsqmd.com) sec. 3.1 FeedForward) with quantised expert
+// weights and the router kept in higher precision (the same page's
+// deployment section on quantisation).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "launch.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kF8Threads = 320;
+constexpr int kF8MaxStages = 8;
+constexpr int kF8OpStages = 2;
+constexpr uint32_t kRawTile = 128 * 64;   // 128 weight rows x 64 e4m3 codes (8 KB)
+constexpr uint32_t kW16Tile = 128 * 128;  // 128 weight rows x 64 fp16 (16 KB)
+constexpr size_t kF8Fixed = 1024 /* alignment slack */ +
+                            (2 * kF8MaxStages + 2 * kF8OpStages + 5) * 8 + 16 +
+                            4 * (kMaxE + 1) * sizeof(int32_t) + 64;
+
+// Two rings: a deep one of input stages (the e4m3 weight tiles of a K step
+// and its token rows, fp16), which keeps enough bytes in flight to stream
+// HBM, and a shallow one of converted fp16 weight operands.
+template <int BN>
+struct F8Cfg {
+    static constexpr uint32_t kInStage = 2 * kRawTile + BN * 128u;
+    static constexpr uint32_t kOpStage = 2 * kW16Tile;
+    static constexpr int kFit = static_cast<int>(
+        (227 * 1024 - kF8Fixed - kF8OpStages * kOpStage) / kInStage);
+    static constexpr int ST = kFit < kF8MaxStages ? kFit : kF8MaxStages;
+    static constexpr int kAccCols = 2 * BN;
+    static constexpr uint32_t kTmemCols = 2u * kAccCols;
+    static constexpr size_t kSmem =
+        kF8Fixed + static_cast<size_t>(ST) * kInStage + kF8OpStages * kOpStage;
+    static_assert(ST >= 4, "pipeline depth");
+    static_assert(kTmemCols >= 32 && kTmemCols <= 512, "tensor memory");
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+    static_assert(kSmem > 227 * 1024 / 2, "one CTA per SM");
+};
+
+struct F8Params {
+    int E, d, d_ff, S, ksplit;
+    size_t part_stride;
+    const int32_t *offsets;
+    const float *s1, *s3, *s2;  // row scales [E, d_ff], [E, d_ff], [E, d]
+    __half *H;                  // [S, d_ff]
+    float *Y;                   // [ksplit, S, d]
+    uint32_t *h_ready;
+    uint32_t *err;
+    int act;
+};
+
+struct F8Unit {
+    bool up;
+    int e, blk, r0, valid, tile, k_beg, k_end, ks;
+};
+
+template <int BN>
+__device__ __forceinline__ F8Unit decode_f8(int u, int u_up, const int32_t *s_off,
+                                            const int32_t *s_pu, const int32_t *s_pd,
+                                            const int32_t *s_tb, int E, int ksplit, int ksu, int ksd)
+{
+    F8Unit w;
+    w.up = u < u_up;
+    const int32_t *pre = w.up ? s_pu : s_pd;
+    const int x = w.up ? u : u - u_up;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= x) lo = mid;
+        else hi = mid - 1;
+    }
+    w.e = lo;
+    int local = x - pre[lo];
+    const int cnt = s_off[lo + 1] - s_off[lo];
+    const int ntb = (cnt + BN - 1) / BN;
+    if (w.up) {
+        w.ks = 0;
+        w.k_beg = 0;
+        w.k_end = ksu;
+    } else {
+        w.ks = local % ksplit;
+        local /= ksplit;
+        w.k_beg = w.ks * ksd / ksplit;
+        w.k_end = (w.ks + 1) * ksd / ksplit;
+    }
+    w.blk = local / ntb;
+    const int tb = local - w.blk * ntb;
+    w.r0 = s_off[lo] + tb * BN;
+    const int rem = cnt - tb * BN;
+    w.valid = rem < BN ? rem : BN;
+    w.tile = s_tb[lo] + tb;
+    return w;
+}
+
+__device__ __forceinline__ void f8_drain_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer() - t0 > 100000000ull) break;  // 100 ms
+    }
+}
+
+__device__ __forceinline__ uint32_t f8_ld_acquire(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void f8_fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void f8_fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ bool f8_wait_counter(const uint32_t *ctr, uint32_t target,
+                                                volatile uint32_t *abort_flag, uint32_t *gerr)
+{
+    if (f8_ld_acquire(ctr) >= target) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (f8_ld_acquire(ctr) >= target) return true;
+        if (*abort_flag) return false;
+        if ((it & 15u) == 0 && ptx::globaltimer() - t0 > kWaitTimeoutNs) {
+            *abort_flag = 1u;
+            if (gerr) atomicOr(gerr, kErrTimeoutEpi);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ int f8_scan(int v, int lane)
+{
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+    }
+    return v;
+}
+
+// Two e4m3 codes (low byte first) to two fp16 values (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two)
+{
+    const __half2_raw h =
+        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// Instruction descriptor of kind::f16 with fp16 A/B, fp32 D, both K-major.
+__device__ __forceinline__ uint32_t idesc_f16_f32(int M, int N)
+{
+    return (1u << 4)                                 // D format fp32
+           | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8   (A, B format fp16 = 0)
+           | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kF8Threads, 1)
+    ffn_fp8_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW3,
+                   const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmX,
+                   const __grid_constant__ CUtensorMap tmH, const F8Params p)
+{
+    using C = F8Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    constexpr int ST = C::ST;
+    uint8_t *ops = smem;                                       // [2] fp16 weight operands
+    uint8_t *ins = smem + kF8OpStages * C::kOpStage;          // [ST] e4m3 tiles + token rows
+    uint64_t *in_full = reinterpret_cast<uint64_t *>(ins + ST * C::kInStage);
+    uint64_t *in_empty = in_full + kF8MaxStages;
+    uint64_t *op_full = in_empty + kF8MaxStages;
+    uint64_t *op_empty = op_full + kF8OpStages;
+    uint64_t *tfull = op_empty + kF8OpStages;  // [2]
+    uint64_t *tempty = tfull + 2;             // [2]
+    uint64_t *drain = tempty + 2;             // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    int32_t *s_off = reinterpret_cast<int32_t *>(tmem_slot + 4);
+    int32_t *s_pu = s_off + (kMaxE + 1);
+    int32_t *s_pd = s_pu + (kMaxE + 1);
+    int32_t *s_tb = s_pd + (kMaxE + 1);
+
+    const int E = p.offsets ? p.E : 1;
+    const int MBU = p.d_ff / 128;
+    const int MBD = (p.d + 255) / 256;
+    const int KSU = p.d / 64;
+    const int KSD = p.d_ff / 64;
+    const int KSPLIT = p.ksplit;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            ptx::mbar_init(&in_full[s], 1);
+            ptx::mbar_init(&in_empty[s], 4 + 1);  // converter warps (e4m3 read) + MMA (rows read)
+        }
+        for (int s = 0; s < kF8OpStages; ++s) {
+            ptx::mbar_init(&op_full[s], 4);       // the four converter warps
+            ptx::mbar_init(&op_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], 4);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        ptx::fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        ptx::prefetch_tensormap(&tmW1);
+        ptx::prefetch_tensormap(&tmW3);
+        ptx::prefetch_tensormap(&tmW2);
+        ptx::prefetch_tensormap(&tmX);
+        ptx::prefetch_tensormap(&tmH);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::grid_dep_wait();
+    if (warp == 2) {
+        const int per = (E + 31) >> 5;
+        const int base = lane * per;
+        bool bad = false;
+        int nu = 0, nd = 0, nt = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = base + i;
+            if (e < E) {
+                const int o0 = p.offsets ? p.offsets[e] : 0;
+                const int o1 = p.offsets ? p.offsets[e + 1] : p.S;
+                s_off[e] = o0;
+                if (e == E - 1) s_off[E] = o1;
+                const int c = o1 - o0;
+                if (o0 < 0 || c < 0 || o1 > p.S) {
+                    bad = true;
+                } else {
+                    const int ntb = (c + BN - 1) / BN;
+                    nt += ntb;
+                    nu += ntb * MBU;
+                    nd += ntb * MBD * KSPLIT;
+                }
+            }
+        }
+        __syncwarp();
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad) {
+            nu = nd = nt = 0;
+            if (lane == 0) atomicOr(p.err, kErrOffsets);
+        }
+        const int iu = f8_scan(nu, lane);
+        const int id = f8_scan(nd, lane);
+        const int it = f8_scan(nt, lane);
+        int ru = iu - nu, rd = id - nd, rt = it - nt;
+        for (int i = 0; i < per; ++i) {
+            const int e = base + i;
+            if (e < E) {
+                s_pu[e] = ru;
+                s_pd[e] = rd;
+                s_tb[e] = rt;
+                if (!bad) {
+                    const int ntb = (s_off[e + 1] - s_off[e] + BN - 1) / BN;
+                    ru += ntb * MBU;
+                    rd += ntb * MBD * KSPLIT;
+                    rt += ntb;
+                }
+            }
+        }
+        if (lane == 31) {
+            s_pu[E] = iu;
+            s_pd[E] = id;
+            s_tb[E] = it;
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int u_up = s_pu[E];
+    const int total = u_up + s_pd[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, issued = 0;
+            uint32_t last_parity[kF8MaxStages];
+#pragma unroll
+            for (int s = 0; s < kF8MaxStages; ++s) last_parity[s] = 0;
+            const uint64_t pol_w = ptx::policy_evict_first();
+            bool stop = false;
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+                const CUtensorMap *ta0 = w.up ? &tmW1 : &tmW2;
+                const CUtensorMap *ta1 = w.up ? &tmW3 : &tmW2;
+                const CUtensorMap *tb = w.up ? &tmX : &tmH;
+                const int arow0 = w.up ? w.e * p.d_ff + w.blk * 128 : w.e * p.d + w.blk * 256;
+                const int arow1 = w.up ? arow0 : arow0 + 128;
+                int ready_blk = -1;
+                for (int ks = w.k_beg; ks < w.k_end; ++ks) {
+                    if (!bounded_wait(&in_empty[stage], phase ^ 1u, abort_flag, p.err,
+                                      kErrTimeoutEpi)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *in = ins + stage * C::kInStage;
+                    ptx::mbar_arrive_expect_tx(&in_full[stage], C::kInStage);
+                    ptx::tma_load_2d_hint(in, ta0, &in_full[stage], ks * 64, arow0, pol_w);
+                    ptx::tma_load_2d_hint(in + kRawTile, ta1, &in_full[stage], ks * 64, arow1,
+                                          pol_w);
+                    issued |= 1u << stage;
+                    last_parity[stage] = phase;
+                    if (!w.up && (ks >> 1) != ready_blk) {
+                        ready_blk = ks >> 1;
+                        if (!f8_wait_counter(&p.h_ready[w.tile * MBU + ready_blk], 4u, abort_flag,
+                                             p.err)) {
+                            stop = true;
+                            break;
+                        }
+                        f8_fence_proxy_async_global();
+                    }
+                    ptx::tma_load_2d(in + 2 * kRawTile, tb, &in_full[stage], ks * 64, w.r0);
+                    if (++stage == static_cast<uint32_t>(ST)) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < ST; ++s)
+                if (issued & (1u << s)) f8_drain_wait(&in_full[s], last_parity[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;    // input ring
+            uint32_t ost = 0, ophase = 0;     // operand ring
+            int i = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x, ++i) {
+                const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+                const int n = ((w.valid + 15) >> 4) << 4;
+                const uint32_t idesc = idesc_f16_f32(128, n);
+                const int buf = i & 1;
+                const uint32_t use = static_cast<uint32_t>(i >> 1);
+                if (!bounded_wait(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.err,
+                                  kErrTimeoutEpi))
+                    break;
+                ptx::tc_fence_after();
+                const uint32_t d0 = tmem + static_cast<uint32_t>(buf * C::kAccCols);
+                for (int ks = w.k_beg; ks < w.k_end; ++ks) {
+                    // The token rows came with the input stage; the weights
+                    // were converted into the operand stage.
+                    if (!bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma) ||
+                        !bounded_wait(&op_full[ost], ophase, abort_flag, p.err, kErrTimeoutTma)) {
+                        stop = true;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
+                    const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage + 2 * kRawTile);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
+                        const uint32_t acc = ((ks - w.k_beg) | kk) ? 1u : 0u;
+                        ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc, idesc,
+                                         acc);
+                        ptx::tc_mma_bf16(d0 + BN, ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
+                                         bdesc, idesc, acc);
+                    }
+                    ptx::tc_commit(&op_empty[ost]);
+                    ptx::tc_commit(&in_empty[stage]);
+                    if (++stage == static_cast<uint32_t>(ST)) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++ost == static_cast<uint32_t>(kF8OpStages)) {
+                        ost = 0;
+                        ophase ^= 1u;
+                    }
+                }
+                if (!stop) ptx::tc_commit(&tfull[buf]);
+            }
+            ptx::tc_commit(drain);
+            f8_drain_wait(drain, 0u);
+        }
+    } else if (warp >= 6) {
+        // Converters: thread r widens weight row r of both tiles of a step.
+        const int r = threadIdx.x - 192;  // 0..127
+        uint32_t stage = 0, phase = 0;    // input ring
+        uint32_t ost = 0, ophase = 0;     // operand ring
+        bool stop = false;
+        for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+            const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+            for (int ks = w.k_beg; ks < w.k_end; ++ks) {
+                const bool ok =
+                    bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma) &&
+                    bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag, p.err, kErrTimeoutMma);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    *abort_flag = 1u;
+                    stop = true;
+                    break;
+                }
+                const uint8_t *ra = ins + stage * C::kInStage;
+                uint8_t *op = ops + ost * C::kOpStage;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    // Raw row r: 64 bytes, 16-byte chunk j stored at chunk
+                    // j ^ ((r >> 1) & 3) (64-byte swizzle).
+                    const uint8_t *src = ra + t * kRawTile + r * 64;
+                    uint8_t *dst = op + t * kW16Tile + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(
+                            src + ((j ^ ((r >> 1) & 3)) << 4));
+                        // 16 codes = columns 16j..16j+15 -> two 16-byte fp16
+                        // chunks 2j and 2j+1 of the 128-byte-swizzled row.
+                        uint4 lo, hi;
+                        lo.x = e4m3x2_to_f16x2(v.x);
+                        lo.y = e4m3x2_to_f16x2(v.x >> 16);
+                        lo.z = e4m3x2_to_f16x2(v.y);
+                        lo.w = e4m3x2_to_f16x2(v.y >> 16);
+                        hi.x = e4m3x2_to_f16x2(v.z);
+                        hi.y = e4m3x2_to_f16x2(v.z >> 16);
+                        hi.z = e4m3x2_to_f16x2(v.w);
+                        hi.w = e4m3x2_to_f16x2(v.w >> 16);
+                        *reinterpret_cast<uint4 *>(dst + (((2 * j) ^ (r & 7)) << 4)) = lo;
+                        *reinterpret_cast<uint4 *>(dst + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+                    }
+                }
+                // The MMA reads the operand through the async proxy.
+                f8_fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(&in_empty[stage]);
+                    ptx::mbar_arrive(&op_full[ost]);
+                }
+                if (++stage == static_cast<uint32_t>(ST)) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++ost == static_cast<uint32_t>(kF8OpStages)) {
+                    ost = 0;
+                    ophase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // Epilogue: warps 2..5, one TMEM lane quarter each.
+        const int q = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        int i = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x, ++i) {
+            const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+            const int buf = i & 1;
+            const uint32_t use = static_cast<uint32_t>(i >> 1);
+            if (!bounded_wait_warp(&tfull[buf], use & 1u, abort_flag, p.err, kErrTimeoutMma))
+                break;
+            ptx::tc_fence_after();
+            const uint32_t tb = tmem + lane_base + static_cast<uint32_t>(buf * C::kAccCols);
+            const int row_in_blk = 32 * q + lane;
+            float sa, sb;
+            if (w.up) {
+                const int f = w.blk * 128 + row_in_blk;
+                sa = p.s1[static_cast<size_t>(w.e) * p.d_ff + f];
+                sb = p.s3[static_cast<size_t>(w.e) * p.d_ff + f];
+            } else {
+                const int o0 = w.blk * 256 + row_in_blk;
+                sa = o0 < p.d ? p.s2[static_cast<size_t>(w.e) * p.d + o0] : 0.0f;
+                sb = o0 + 128 < p.d ? p.s2[static_cast<size_t>(w.e) * p.d + o0 + 128] : 0.0f;
+            }
+            for (int c0 = 0; c0 < w.valid; c0 += 32) {
+                uint32_t a[32], b[32];
+                ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), a);
+                ptx::tmem_ld32(tb + static_cast<uint32_t>(BN + c0), b);
+                ptx::tc_wait_ld();
+                if (w.up) {
+                    const int f = w.blk * 128 + row_in_blk;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < w.valid) {
+                            const float g = sa * __uint_as_float(a[j]);
+                            const float bv = sb * __uint_as_float(b[j]);
+                            const float h = __fdividef(p.act ? bv : g * bv, 1.0f + __expf(-g));
+                            p.H[static_cast<size_t>(w.r0 + c0 + j) * p.d_ff + f] = __float2half_rn(h);
+                        }
+                    }
+                } else {
+                    const int o0 = w.blk * 256 + row_in_blk;
+                    const bool has0 = o0 < p.d;
+                    const bool has1 = o0 + 128 < p.d;
+                    float *Y = p.Y + w.ks * p.part_stride;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < w.valid) {
+                            float *yr = Y + static_cast<size_t>(w.r0 + c0 + j) * p.d;
+                            if (has0) yr[o0] = sa * __uint_as_float(a[j]);
+                            if (has1) yr[o0 + 128] = sb * __uint_as_float(b[j]);
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            if (w.up) {
+                // Publish this warp's slice of the H block to the down units
+                // (which read it through TMA, the async proxy).
+                f8_fence_proxy_async_global();
+                __threadfence();
+            }
+            __syncwarp();
+            if (lane == 0) {
+                if (w.up) atomicAdd(&p.h_ready[w.tile * MBU + w.blk], 1u);
+                ptx::mbar_arrive(&tempty[buf]);
+            }
+        }
+    }
+
+    ptx::grid_dep_launch();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int BN>
+cudaError_t launch_fp8_cfg(const FfnFp8Launch &a, cudaStream_t s)
+{
+    using C = F8Cfg<BN>;
+    const int E = a.f.offsets ? a.f.E : 1;
+    CUtensorMap tW1, tW3, tW2, tX, tH;
+    cudaError_t e = make_tmap_e4m3(&tW1, a.q1, static_cast<uint64_t>(E) * a.f.d_ff, a.f.d);
+    if (e == cudaSuccess) e = make_tmap_e4m3(&tW3, a.q3, static_cast<uint64_t>(E) * a.f.d_ff, a.f.d);
+    if (e == cudaSuccess) e = make_tmap_e4m3(&tW2, a.q2, static_cast<uint64_t>(E) * a.f.d, a.f.d_ff);
+    if (e == cudaSuccess) e = make_tmap_f16(&tX, a.f.x, a.f.S, a.f.d, BN);
+    if (e == cudaSuccess) e = make_tmap_f16(&tH, a.f.H, a.f.S, a.f.d_ff, BN);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ffn_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::kSmem));
+    if (e != cudaSuccess) return e;
+    F8Params p{};
+    p.E = E;
+    p.d = a.f.d;
+    p.d_ff = a.f.d_ff;
+    p.S = a.f.S;
+    p.ksplit = a.f.ksplit < 1 ? 1 : a.f.ksplit;
+    p.part_stride = static_cast<size_t>(a.f.S) * a.f.d;
+    p.offsets = a.f.offsets;
+    p.s1 = a.s1;
+    p.s3 = a.s3;
+    p.s2 = a.s2;
+    p.H = reinterpret_cast<__half *>(a.f.H);
+    p.Y = a.f.Y;
+    p.h_ready = a.f.h_ready;
+    p.err = a.f.err;
+    p.act = a.f.act;
+    const long long tiles = (static_cast<long long>(a.f.S) + BN - 1) / BN + E;
+    const long long units =
+        tiles * (a.f.d_ff / 128) + tiles * ((a.f.d + 255) / 256) * p.ksplit;
+    long long grid = device_sm_count();
+    if (units < grid) grid = units;
+    if (grid < 1) grid = 1;
+    return launch_pdl(ffn_fp8_kernel<BN>, dim3(static_cast<unsigned>(grid)), dim3(kF8Threads),
+                      C::kSmem, s, a.f.pdl, tW1, tW3, tW2, tX, tH, p);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_fp8(const FfnFp8Launch &a, cudaStream_t s)
+{
+    switch (ffn_token_tile(a.f.S, a.f.offsets ? a.f.E : 1)) {
+    case 32: return launch_fp8_cfg<32>(a, s);
+    case 64: return launch_fp8_cfg<64>(a, s);
+    default: return launch_fp8_cfg<128>(a, s);
+    }
+}
+
+}  // namespace moe

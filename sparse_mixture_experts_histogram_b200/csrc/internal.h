@@ -9,6 +9,7 @@ namespace moe {
 
 struct RouteLaunch {
     int T, d, E, k;
+    int wmode;           // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid
     const uint16_t *x;   // [T,d] bf16
     const uint16_t *Wg;  // [E,d] bf16
     const float *bias;   // [E] or nullptr
@@ -30,6 +31,7 @@ struct RouteLaunch {
     int32_t *perm;       // [E, perm_stride]
     int32_t *gcnt;       // [E] zero before the launch (left zero)
     int perm_stride;
+    int cap;             // per-expert capacity of the token-ordered dispatch, or -1
 };
 
 struct RanksLaunch {
@@ -41,12 +43,15 @@ struct RanksLaunch {
 
 struct ScatterLaunch {
     int T, d, E, k;
+    int cap;                  // per-expert capacity, or -1 (dropless)
+    const int32_t *offsets;   // [E+1] segment starts, needed when cap >= 0
     const uint16_t *x;
     const int32_t *idx, *rank, *tilebase;
     uint16_t *x_perm;
     int32_t *row_of_slot;
     uint32_t *err;
     bool pdl;  // launched right after another kernel of this library
+    bool to_f16;  // write x_perm as fp16 (the FP8 expert path) instead of bf16
 };
 
 struct FfnLaunch {
@@ -63,8 +68,12 @@ struct FfnLaunch {
     uint16_t *H;              // [S, d_ff] intermediate
     float *Y;                 // [ksplit, S, d]
     uint32_t *h_ready;        // ffn_ready_counters(S, E, d_ff) counters, zero before the launch
+    uint32_t *sched;          // work counter, zero before the launch; when set, large
+                              // batches run the CTA-pair kernel (launch_ffn_pair)
     uint32_t *err;
     bool pdl;                 // launched right after another kernel of this library
+    int act;                  // expert activation: 0 silu(W1 x) * W3 x (SwiGLU),
+                              // 1 sigmoid(W1 x) * W3 x
     // Narrow kernel only: when set, the rows of segment e are gathered from x
     // ([x_rows, d]) through the token list perm[e * perm_stride + position]
     // instead of being read from a permuted copy.
@@ -93,6 +102,10 @@ cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s);
 cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s);
 cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s);
 cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s);
+// The same computation by CTA pairs sharing 256-row MMAs, for segments of
+// about 128 rows or more and no K split (called by launch_ffn).
+bool ffn_pair_eligible(int S, int E_seg, int ksplit);
+cudaError_t launch_ffn_pair(const FfnLaunch &a, uint32_t *sched, cudaStream_t s);
 // Narrow layers (d <= 1024): every CTA runs whole hidden chunks (up, H in
 // shared memory, down) and writes `nsplit` partial outputs [nsplit, S, d].
 cudaError_t launch_ffn_small(const FfnLaunch &a, int nsplit_max, int *nsplit_out,
@@ -103,6 +116,23 @@ int ffn_token_tile(int S, int E_seg);
 size_t ffn_ready_counters(int S, int E_seg, int d_ff);
 int down_ksplit(int S, int E_seg, int d, int d_ff);
 cudaError_t launch_combine(const CombineLaunch &a, cudaStream_t s);
+
+// Expert FFN with FP8 weights (gemm_fp8.cu): e4m3 codes and per-row fp32
+// scales; f.x (the permuted token rows) and f.H are fp16 in this path.
+struct FfnFp8Launch {
+    FfnLaunch f;
+    const uint8_t *q1, *q3;   // [E, d_ff, d] e4m3
+    const uint8_t *q2;        // [E, d, d_ff] e4m3
+    const float *s1, *s3;     // [E, d_ff]
+    const float *s2;          // [E, d]
+};
+cudaError_t launch_ffn_fp8(const FfnFp8Launch &a, cudaStream_t s);
+
+// 2-D e4m3 (byte) matrix read in boxes of 64 columns (64-byte swizzle) by
+// 128 rows, and 2-D fp16 matrix read like make_tmap_bf16.
+cudaError_t make_tmap_e4m3(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols);
+cudaError_t make_tmap_f16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows);
 
 // Tensor maps (tensormap.cpp side, implemented in api.cu).
 // 2-D bf16 row-major matrix [rows, cols] read in boxes of 64 columns (128 B,

@@ -12,10 +12,13 @@
 // The scratch is a file-scope __device__ array, so every GPU that loads the
 // library holds kStaticScratchBytes of it until the process exits.  In host
 // code the array's name is only a host-side stand-in: its device address is
-// looked up once per device with cudaGetSymbolAddress (with that device
-// current) on the first call made on that device, and that address is what
-// the kernels receive.
+// looked up with cudaGetSymbolAddress (with the device current) on the first
+// call made on that device, and that address is what the kernels receive.
+// The lookup is repeated when the device's context has changed since (after
+// a cudaDeviceReset the array lives at a new address).
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <mutex>
@@ -27,7 +30,7 @@ namespace moe {
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr size_t kStaticScratchBytes = MOE_STATIC_SCRATCH_BYTES;  // 32 MiB
 constexpr size_t kStaticHeaderBytes = 256;                // device error word, then H
 constexpr int kStaticMaxDevices = 64;
 
@@ -35,18 +38,59 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 std::mutex g_static_mutex;
 void *g_static_ptr[kStaticMaxDevices] = {};
+unsigned long long g_static_ctx[kStaticMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device (looked up once
-// per device).  Returns nullptr if the lookup failed.
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+void load_ctx_fns()
+{
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+}
+
+// Unique id of the context current on this thread, or 0 if there is none
+// (yet) or it cannot be asked for.
+unsigned long long current_ctx_id()
+{
+    std::call_once(g_ctx_once, load_ctx_fns);
+    if (g_ctx_current == nullptr || g_ctx_id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    unsigned long long id = 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_static_scratch on device `dev` (the current device).
+// Returns nullptr if the lookup failed.
 void *static_scratch_address(int dev)
 {
     std::lock_guard<std::mutex> lock(g_static_mutex);
-    if (g_static_ptr[dev] == nullptr) {
+    const unsigned long long id = current_ctx_id();
+    if (g_static_ptr[dev] == nullptr || id == 0 || id != g_static_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
         g_static_ptr[dev] = p;
+        g_static_ctx[dev] = current_ctx_id();
     }
     return g_static_ptr[dev];
+}
+
+// Bytes of the fixed scratch a call of these sizes needs: the header (error
+// word), the readiness counters of the expert kernel and H [S, d_ff] bf16.
+size_t static_need(int S, int E, int d_ff)
+{
+    const size_t ctr_bytes = (ffn_ready_counters(S, E, d_ff) * 4 + 255) / 256 * 256;
+    return kStaticHeaderBytes + ctr_bytes + static_cast<size_t>(S) * d_ff * 2;
 }
 
 }  // namespace
@@ -71,9 +115,8 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
         if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
     // The tile counters and H [S, d_ff] bf16 must fit in the fixed scratch
     // behind the header.
+    if (static_need(S, E, d_ff) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
     const size_t ctr_bytes = (ffn_ready_counters(S, E, d_ff) * 4 + 255) / 256 * 256;
-    const size_t h_bytes = static_cast<size_t>(S) * d_ff * 2;
-    if (ctr_bytes + h_bytes > kStaticScratchBytes - kStaticHeaderBytes) return MOE_ERR_WORKSPACE;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStaticMaxDevices)
@@ -105,4 +148,30 @@ extern "C" moe_status moe_expert_ffn_static(int S, int d, int E, int d_ff,
     f.pdl = false;
     if (launch_ffn(f, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+extern "C" moe_status moe_expert_ffn_static_error(uint32_t *code, moe_stream_t stream)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStaticMaxDevices)
+        return MOE_ERR_CUDA;
+    const uint8_t *scratch = static_cast<const uint8_t *>(static_scratch_address(dev));
+    if (scratch == nullptr) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (code) *code = word;
+    if (word == 0) return MOE_OK;
+    if (word & (MOE_DEVERR_TIMEOUT_TMA | MOE_DEVERR_TIMEOUT_MMA | MOE_DEVERR_TIMEOUT_EPI))
+        return MOE_ERR_TIMEOUT;
+    return MOE_ERR_DEVICE;
+}
+
+extern "C" size_t moe_expert_ffn_static_bytes(int S, int E, int d_ff)
+{
+    if (S < 1 || E < 1 || E > 256 || d_ff < 128 || d_ff % 128 || d_ff > 65536 || S > (1 << 24))
+        return 0;
+    return static_need(S, E, d_ff);
 }

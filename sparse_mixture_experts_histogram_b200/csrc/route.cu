@@ -30,6 +30,7 @@ constexpr uint32_t kRouteABytes = 128 * 128;   // 128 token rows x 64 bf16
 
 struct RouteParams {
     int T, d, E, Npad, stages, ntiles;
+    int wmode;      // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid
     uint32_t tmem_cols;
     const float *bias;
     int32_t *idx;
@@ -77,6 +78,34 @@ __device__ __forceinline__ void topk_insert(float (&tv)[K], int (&ti)[K], float 
             tv[0] = v;
             ti[0] = e;
         }
+    }
+}
+
+// Gate weights of the k selected logits tv[0..K) (descending):
+//   wmode 0: softmax over the selected logits (the method)
+//   wmode 1: softmax over all E logits, given their maximum m_all and
+//            sum_all = sum_e exp(l_e - m_all); not renormalised over the
+//            selected ("Mixtral 8x7B模型架构解析" Router.forward)
+//   wmode 2: the sigmoid of each selected logit ("万亿 MoE" forward listing)
+template <int K>
+__device__ __forceinline__ void gate_weights(const float (&tv)[K], int wmode, float m_all,
+                                             float sum_all, float (&w)[K])
+{
+    if (wmode == 1) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) w[j] = expf(tv[j] - m_all) / sum_all;
+    } else if (wmode == 2) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) w[j] = 1.0f / (1.0f + expf(-tv[j]));
+    } else {
+        float s = 0.0f;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            w[j] = expf(tv[j] - tv[0]);
+            s += w[j];
+        }
+#pragma unroll
+        for (int j = 0; j < K; ++j) w[j] = w[j] / s;
     }
 }
 
@@ -206,6 +235,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
             tv[j] = -CUDART_INF_F;
             ti[j] = -1;
         }
+        // Running maximum and sum of exp(l - max) over all E logits (for the
+        // softmax over all experts).
+        float run_m = -CUDART_INF_F, run_s = 0.0f;
         if (ok) {
             const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
             for (int c0 = 0; c0 < p.Npad; c0 += 16) {
@@ -215,7 +247,39 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int e = c0 + jj;
-                    if (e < p.E) topk_insert<K>(tv, ti, __uint_as_float(r[jj]) + bias_s[e], e);
+                    // A NaN logit (only from non-finite inputs) ranks like -inf.
+                    const float l0 = __uint_as_float(r[jj]) + bias_s[e];
+                    const float l = (l0 == l0) ? l0 : -CUDART_INF_F;
+                    if (e < p.E) {
+                        topk_insert<K>(tv, ti, l, e);
+                        if (p.wmode == 1 && l > -CUDART_INF_F) {
+                            if (l > run_m) {
+                                run_s = run_s * expf(run_m - l) + 1.0f;
+                                run_m = l;
+                            } else {
+                                run_s += expf(l - run_m);
+                            }
+                        }
+                    }
+                }
+            }
+            // Logits equal to -inf (or NaN) are never inserted; the slots they
+            // leave empty all hold -inf, so -- ties going to the lower index --
+            // they take the lowest experts not yet selected, in order.  Every
+            // slot then holds a distinct expert in [0, E) (k <= E), the same
+            // choice the CUDA-core router makes.
+            int cand = 0;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                if (ti[j] < 0) {
+                    bool used = true;
+                    while (used) {
+                        used = false;
+#pragma unroll
+                        for (int jj = 0; jj < K; ++jj) used |= (ti[jj] == cand);
+                        if (used) ++cand;
+                    }
+                    ti[j] = cand++;
                 }
             }
         }
@@ -223,18 +287,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
         const bool valid = ok && (t < p.T);
         if (valid) {
-            const float m = tv[0];
-            float ex[K];
-            float s = 0.0f;
-#pragma unroll
-            for (int j = 0; j < K; ++j) {
-                ex[j] = expf(tv[j] - m);
-                s += ex[j];
-            }
+            float wv[K];
+            gate_weights<K>(tv, p.wmode, run_m, run_s, wv);
 #pragma unroll
             for (int j = 0; j < K; ++j) {
                 p.idx[static_cast<size_t>(t) * K + j] = ti[j];
-                p.w[static_cast<size_t>(t) * K + j] = ex[j] / s;
+                p.w[static_cast<size_t>(t) * K + j] = wv[j];
             }
         }
 #pragma unroll
@@ -269,6 +327,7 @@ constexpr int kSmallThreads = 256;
 
 struct SmallRouteParams {
     int T, d, E;
+    int wmode;      // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid
     const uint4 *x;
     const uint4 *Wg;
     const float *bias;
@@ -431,18 +490,24 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
             for (int i = 0; i < kMaxE / 32; ++i)
                 if (lane + 32 * i == be) taken |= 1u << i;
         }
-        if (lane == 0) {
-            float ex[K];
-            float s = 0.0f;
+        // Sum of exp(l - max) over all E logits (the softmax over all
+        // experts); tv[0] is the maximum.
+        float sum_all = 0.0f;
+        if (p.wmode == 1) {
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                ex[j] = expf(tv[j] - tv[0]);
-                s += ex[j];
-            }
+            for (int i = 0; i < kMaxE / 32; ++i)
+                if (lane + 32 * i < p.E && v[i] > -CUDART_INF_F) sum_all += expf(v[i] - tv[0]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                sum_all += __shfl_xor_sync(0xffffffffu, sum_all, off);
+        }
+        if (lane == 0) {
+            float wv[K];
+            gate_weights<K>(tv, p.wmode, tv[0], sum_all, wv);
 #pragma unroll
             for (int j = 0; j < K; ++j) {
                 p.idx[static_cast<size_t>(t) * K + j] = ti[j];
-                p.w[static_cast<size_t>(t) * K + j] = ex[j] / s;
+                p.w[static_cast<size_t>(t) * K + j] = wv[j];
                 ds.sel[warp][j] = ti[j];
             }
         }
@@ -488,6 +553,7 @@ cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
     p.T = a.T;
     p.d = a.d;
     p.E = a.E;
+    p.wmode = a.wmode;
     p.x = reinterpret_cast<const uint4 *>(a.x);
     p.Wg = reinterpret_cast<const uint4 *>(a.Wg);
     p.bias = a.bias;
@@ -500,6 +566,7 @@ cudaError_t launch_route_small_cfg(const RouteLaunch &a, cudaStream_t s)
     p.dout.offsets = a.offsets;
     p.dout.counts = a.counts;
     p.dout.done = a.done;
+    p.dout.cap = a.cap;
     p.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
     const int blocks = (a.T + kSmallTok - 1) / kSmallTok;
     fill_slots(a, &p.slots, &p.sout);
@@ -546,6 +613,7 @@ cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
     p.d = a.d;
     p.E = a.E;
     p.Npad = Npad;
+    p.wmode = a.wmode;
     p.stages = stages;
     p.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
     p.tmem_cols = cols;
@@ -559,6 +627,7 @@ cudaError_t launch_route_k(const RouteLaunch &a, cudaStream_t s)
     p.dout.offsets = a.offsets;
     p.dout.counts = a.counts;
     p.dout.done = a.done;
+    p.dout.cap = a.cap;
     p.dout.ntiles = p.ntiles;
     fill_slots(a, &p.slots, &p.sout);
     route_kernel<K><<<p.ntiles, kRouteThreads, smem, s>>>(tmX, tmWg, p);

@@ -81,8 +81,12 @@ def mixtral_decode(T: int) -> Workload:
     return Workload(f"mixtral_decode_T{T}", T, 4096, 8, 14336, 2)
 
 
-def fine_grained(T: int = 8192) -> Workload:
-    return Workload(f"fine_grained_T{T}_E256_k8_shared", T, 7168, 256, 2048, 8, d_ff_shared=2048)
+def fine_grained(T: int = 8192, E: int = 256) -> Workload:
+    """d = 7168, E routed experts of d_ff = 2048, top-8, one shared expert of
+    d_ff = 2048.  E = 256 is the configuration; fewer experts with T scaled by
+    E/256 keep its rows per expert (for profiling captures that must stay
+    small)."""
+    return Workload(f"fine_grained_T{T}_E{E}_k8_shared", T, 7168, E, 2048, 8, d_ff_shared=2048)
 
 
 def router_bias(wl: Workload, device="cpu") -> torch.Tensor | None:

@@ -150,3 +150,37 @@ def sample_tokens(T, n, idx=None, near=None, seed=0):
             if not any(e in idx[t] for t in chosen):
                 chosen.add(int(np.nonzero((idx == e).any(1))[0][0]))
     return np.array(sorted(chosen))
+
+
+def gpu_forward_variant(wl, inp, variant, ws=None):
+    dev = inp["x"].device
+    out = torch.empty(wl.T, wl.d, dtype=torch.float32, device=dev)
+    ws = workspace(wl) if ws is None else ws
+    moe.moe_forward_variant(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["bias"],
+                            inp["W1"], inp["W3"], inp["W2"], wl.d_ff_shared, inp.get("Ws1"),
+                            inp.get("Ws3"), inp.get("Ws2"), variant, out, ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 0, f"device error word {code:#x}"
+    return out
+
+
+def check_forward_variant(wl, inp, variant, tokens=None):
+    """Whole layer under a variant (weights, activation, capacity_factor) vs
+    the oracle with the same variant.  Routing is checked as for the method;
+    the oracle takes the GPU's selection for the compared tokens (identical
+    outside near ties) and, for the capacity ranks, for all tokens."""
+    weights, act, cf = variant
+    idx, r, near = check_routing(wl, inp)
+    out = gpu_forward_variant(wl, inp, variant).cpu().numpy().astype(np.float64)
+    tok = np.arange(wl.T) if tokens is None else np.asarray(tokens)
+    shared = None
+    if wl.d_ff_shared:
+        shared = (bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"]))
+    bias = None if inp["bias"] is None else inp["bias"].double().cpu().numpy()
+    cap = oracle.capacity_limit(cf, wl.T, wl.k, wl.E) if cf > 0 else None
+    ref = oracle.forward(bits(inp["x"]), bits(inp["Wg"]), bits(inp["W1"]), bits(inp["W3"]),
+                         bits(inp["W2"]), wl.k, bias=bias, tokens=tok, shared=shared,
+                         forced=idx[tok], w_mode=weights, act_mode=act, capacity=cap,
+                         route_all=idx if cap is not None else None)
+    mx, mean = assert_close(out[tok], ref, f"{wl.name} variant {variant}")
+    return {"max_rel": mx, "mean_rel": mean, "near_ties": int(near.sum()), "cap": cap}

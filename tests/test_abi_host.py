@@ -113,3 +113,47 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     with pytest.raises(RuntimeError, match="missing"):
         binding.load_library(str(tmp_path / "nope.so"))
     monkeypatch.setattr(binding, "_lib", None)
+
+
+def _static_need(S, E, d_ff):
+    ctr = 4 * (-(-S // 32) + E) * (d_ff // 128)
+    return 256 + -(-ctr // 256) * 256 + 2 * S * d_ff
+
+
+def test_static_scratch_limit_matches_its_documented_formula(lib):
+    cap = 32 << 20
+    assert "#define MOE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)" in open(
+        os.path.join(ROOT, "include", "moe.h")).read()
+    for S, E, d_ff in [(1, 1, 128), (37, 6, 640), (4096, 8, 4096), (131000, 1, 128)]:
+        assert moe.moe_expert_ffn_static_bytes(S, E, d_ff) == _static_need(S, E, d_ff)
+    assert moe.moe_expert_ffn_static_bytes(10, 1, 100) == 0
+    # The largest S that fits for (E=1, d_ff=128), and one row more: the
+    # larger call is refused on the host before anything is launched.
+    S = max(s for s in range(130000, 132000) if _static_need(s, 1, 128) <= cap)
+    assert _static_need(S + 1, 1, 128) > cap
+    assert lib.moe_expert_ffn_static(S + 1, 128, 1, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     None) == 3
+    # 4096 rows x 4096 hidden x 2 bytes alone fill the array: refused too.
+    assert lib.moe_expert_ffn_static(4096, 512, 8, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     None) == 3
+    assert lib.moe_expert_ffn_static(S, 128, 1, 128, FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     None) == 1
+
+
+def test_variant_arguments_are_checked_on_the_host(lib):
+    V = binding.MoEVariant
+    ws = 1 << 40
+    for bad in (V(3, 0, 0.0), V(-1, 0, 0.0), V(0, 2, 0.0), V(0, 0, -1.0), V(0, 0, float("nan")),
+                V(0, 0, float("inf"))):
+        st = lib.moe_forward_variant(16, 512, 8, 1024, 2, FAKE, FAKE, None, FAKE, FAKE, FAKE, 0,
+                                     None, None, None, ctypes.addressof(bad), FAKE, FAKE, ws, None)
+        assert st == 1, (bad.weights, bad.activation, bad.capacity_factor)
+    assert lib.moe_route_variant(16, 512, 8, 2, FAKE, FAKE, None, 3, FAKE, FAKE, None, FAKE, ws,
+                                 None) == 1
+    assert lib.moe_route_variant(16, 512, 8, 9, FAKE, FAKE, None, 1, FAKE, FAKE, None, FAKE, ws,
+                                 None) == 1
+    h = open(os.path.join(ROOT, "include", "moe.h")).read()
+    for name, v in (("MOE_WEIGHTS_SOFTMAX_TOPK", 0), ("MOE_WEIGHTS_SOFTMAX_ALL", 1),
+                    ("MOE_WEIGHTS_SIGMOID", 2), ("MOE_ACT_SILU", 0), ("MOE_ACT_SIGMOID", 1)):
+        assert f"#define {name} {v}" in h
+    assert ctypes.sizeof(V) == 16

@@ -65,7 +65,18 @@ def test_flops_and_bytes_closed_forms():
         assert acc.ffn_flops(T, d, f, k) + acc.ffn_flops(T, d, fs, 1) == \
             acc.active_flops(T, d, 1, f, k, fs) - 2 * T * d
     # the FFN kernel's bytes: all hit experts' weights once, rows in, fp32 rows out
-    assert acc.ffn_bytes(512, 512, 4096, 2, 8) == 2 * 3 * 8 * 512 * 4096 + 6 * 1024 * 512
+    assert acc.ffn_bytes(512, 512, 4096, 2, 8) == 2 * 3 * 8 * 512 * 4096 + 6 * 512 * 512
     # decode T=1 streams the two hit experts: 0.70 GB
     b = acc.algorithmic_bytes(1, 4096, 8, 14336, 2, experts_hit=2)
     assert abs(b / 1e9 - 0.705) < 0.001
+
+
+def test_fp8_bytes_count_one_byte_per_weight_and_the_row_scales():
+    # e4m3 experts: one byte per weight plus an fp32 scale per W1, W3 and W2
+    # row; everything else as in the bf16 layer.
+    d, f, E, T, k = 4096, 14336, 8, 8, 2
+    assert acc.fp8_scale_bytes(d, f) == 4 * (2 * f + d)
+    b16 = acc.algorithmic_bytes(T, d, E, f, k, experts_hit=8)
+    b8 = acc.algorithmic_bytes(T, d, E, f, k, experts_hit=8, fp8=True)
+    assert b16 - b8 == 8 * (3 * d * f - acc.fp8_scale_bytes(d, f))
+    assert acc.ffn_bytes(T, d, f, k, 8, fp8=True) == 8 * (3 * d * f + 4 * (2 * f + d)) + 6 * T * d

@@ -9,8 +9,8 @@ import sparse_mixture_experts_histogram_b200 as moe
 from sparse_mixture_experts_histogram_b200 import synth
 from sparse_mixture_experts_histogram_b200.synth import Workload, bits
 
-from gpu_util import (assert_close, check_forward, check_routing, gpu_forward, gpu_route,
-                      sample_tokens, workspace)
+from gpu_util import (assert_close, check_forward, check_forward_variant, check_routing,
+                      gpu_forward, gpu_route, sample_tokens, workspace)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +42,27 @@ ROUTE_CASES = [
 @pytest.mark.parametrize("wl", ROUTE_CASES, ids=lambda w: w.name)
 def test_route_matches_oracle(wl):
     check_routing(wl, _inputs(wl))
+
+
+# Shapes with T*E*d above 2^30 take the tensor-core router (tcgen05 MMA,
+# top-k and softmax in its epilogue): ragged T, k in {1, 2, 4, 8}, E not a
+# multiple of 16, with and without a router bias.
+TC_ROUTE_CASES = [
+    Workload("tc_T1153_d7168_E256_k8", 1153, 7168, 256, 128, 8),
+    Workload("tc_T1000_d7168_E200_k1", 1000, 7168, 200, 128, 1),
+    Workload("tc_T1153_d4096_E256_k2", 1153, 4096, 256, 128, 2),
+    Workload("tc_T1200_d7168_E136_k4", 1200, 7168, 136, 128, 4),
+]
+
+
+@pytest.mark.parametrize("with_bias", [False, True], ids=["nobias", "bias"])
+@pytest.mark.parametrize("wl", TC_ROUTE_CASES, ids=lambda w: w.name)
+def test_tensor_core_route_matches_oracle(wl, with_bias):
+    assert wl.T * wl.E * wl.d > 2 ** 30
+    inp = synth.make_inputs(wl, device=DEV)
+    if with_bias:
+        inp["bias"] = torch.linspace(-0.5, 0.5, wl.E, dtype=torch.float32, device=DEV)
+    check_routing(wl, inp)
 
 
 def test_route_equal_logits_pick_lowest_indices():
@@ -281,14 +302,17 @@ def test_forward_narrow_repeatable_whatever_the_slot_order(wl):
 
 
 @pytest.mark.parametrize("wl", [Workload("nonfinite_narrow", 64, 256, 8, 256, 2),
-                                Workload("nonfinite_wide", 40, 1152, 8, 256, 3)],
+                                Workload("nonfinite_wide", 40, 1152, 8, 256, 3),
+                                Workload("nonfinite_tensor_core_router", 700, 7168, 256, 128, 8)],
                          ids=lambda w: w.name)
 def test_nonfinite_rows_route_in_bounds(wl):
     # Inputs are finite by construction everywhere else; a NaN or Inf row must
     # still give every slot of its token a distinct expert in [0, E) (NaN ranks
     # like -inf, ties go to the lower index), raise no device error, and leave
-    # the other tokens' outputs as they were.
-    inp = _inputs(wl, seed=5)
+    # the other tokens' outputs as they were.  The first two shapes take the
+    # CUDA-core router, the last (T*E*d > 2^30) the tensor-core router.
+    big = wl.T * wl.E * wl.d > 2 ** 30
+    inp = synth.make_inputs(wl, seed=5, device=DEV) if big else _inputs(wl, seed=5)
     bad = inp["x"].clone()
     bad[3] = float("nan")
     bad[17] = float("inf")
@@ -323,8 +347,132 @@ def test_forward_mixtral_prefill(T, skew):
 
 
 def test_forward_fine_grained_shared():
+    # Sampled output check: 8 seeded tokens, every near-tie token and one
+    # token of every hit expert, so each of the 256 experts' segments is
+    # compared element by element at least once.
     wl = synth.fine_grained(8192)
     inp = synth.make_inputs(wl, device=DEV)
     idx, r, near = check_routing(wl, inp)
-    tok = sample_tokens(wl.T, 8, None, near)
+    tok = sample_tokens(wl.T, 8, idx, near)
+    assert set(np.unique(idx[tok])) == set(np.unique(idx))
     check_forward(wl, inp, tokens=tok, r=r)
+
+
+# ------------------------------------------------------------------ variants
+# Gate-weight rules, the sigmoid-gated expert and the expert capacity (the
+# variants the pages print beside the method), against the oracle with the
+# same variant.  Narrow layers (d <= 1024) and wide ones, both routers.
+VARIANT_ROUTE_CASES = [
+    Workload("var_T300_E16_k4", 300, 256, 16, 128, 4),
+    Workload("var_tc_T1153_d7168_E200_k8", 1153, 7168, 200, 128, 8),
+]
+
+
+@pytest.mark.parametrize("weights", [moe.WEIGHTS_SOFTMAX_ALL, moe.WEIGHTS_SIGMOID])
+@pytest.mark.parametrize("wl", VARIANT_ROUTE_CASES, ids=lambda w: w.name)
+def test_route_variant_weights_match_oracle(wl, weights):
+    big = wl.T * wl.E * wl.d > 2 ** 30
+    inp = synth.make_inputs(wl, device=DEV) if big else _inputs(wl)
+    inp["bias"] = torch.linspace(-0.4, 0.4, wl.E, dtype=torch.float32, device=DEV)
+    bias = inp["bias"].double().cpu().numpy()
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), wl.k, bias=bias, w_mode=weights)
+    idx = torch.empty(wl.T, wl.k, dtype=torch.int32, device=DEV)
+    w = torch.empty(wl.T, wl.k, dtype=torch.float32, device=DEV)
+    ws = workspace(wl)
+    moe.moe_route_variant(wl.T, wl.d, wl.E, wl.k, inp["x"], inp["Wg"], inp["bias"], weights, idx,
+                          w, None, ws)
+    assert moe.moe_get_device_error(ws)[0] == 0
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    far = r["gap"] >= 1e-3
+    assert np.array_equal(np.sort(idx, 1)[far], np.sort(r["idx"], 1)[far])
+    wg = np.take_along_axis(w, np.argsort(idx, 1), 1)
+    wo = np.take_along_axis(r["w"], np.argsort(r["idx"], 1), 1)
+    assert np.max(np.abs(wg[far] - wo[far])) < 2e-4
+
+
+VARIANT_FORWARD_CASES = [
+    (Workload("var_narrow_T300_d256_E16_k2", 300, 256, 16, 384, 2), (1, 0, 0.0)),
+    (Workload("var_narrow_T300_d256_E16_k2", 300, 256, 16, 384, 2), (2, 1, 0.0)),
+    (Workload("var_narrow_T300_d256_E16_k2_shared", 300, 256, 16, 384, 2, d_ff_shared=256),
+     (2, 1, 0.0)),
+    (Workload("var_wide_T200_d1152_E8_k2", 200, 1152, 8, 384, 2), (1, 1, 0.0)),
+    (Workload("var_wide_T1100_d1152_E8_k2", 1100, 1152, 8, 512, 2), (2, 1, 0.0)),
+    # capacity: skewed router bias so that some experts overflow
+    (Workload("cap_narrow_T300_d256_E8_k2", 300, 256, 8, 384, 2, skew=True), (0, 0, 1.0)),
+    (Workload("cap_narrow_T300_d256_E8_k2_b", 300, 256, 8, 384, 2, skew=True), (2, 1, 1.25)),
+    (Workload("cap_wide_T700_d1152_E8_k2", 700, 1152, 8, 512, 2, skew=True), (0, 0, 1.2)),
+    (Workload("cap_wide_T2000_d1152_E16_k4", 2000, 1152, 16, 256, 4, skew=True), (1, 0, 0.8)),
+]
+
+
+@pytest.mark.parametrize("wl,variant", VARIANT_FORWARD_CASES,
+                         ids=[f"{w.name}-{v}" for w, v in VARIANT_FORWARD_CASES])
+def test_forward_variant_matches_oracle(wl, variant):
+    inp = _inputs(wl)
+    if wl.skew:
+        inp["bias"] = torch.zeros(wl.E, dtype=torch.float32, device=DEV)
+        inp["bias"][1] = 1.5
+        inp["bias"][2] = 1.0
+    res = check_forward_variant(wl, inp, variant)
+    if variant[2] > 0:
+        # the capacity does drop pairs on these inputs
+        idx, _, counts = gpu_route(wl, inp)
+        assert counts.max() > res["cap"]
+
+
+def test_forward_variant_none_is_the_method():
+    wl = Workload("var_none", 200, 256, 8, 256, 2)
+    inp = _inputs(wl)
+    from gpu_util import gpu_forward_variant
+    a = gpu_forward(wl, inp)
+    b = gpu_forward_variant(wl, inp, None)
+    c = gpu_forward_variant(wl, inp, (0, 0, 0.0))
+    assert torch.equal(a, b) and torch.equal(a, c)
+
+
+# ------------------------------------------------------------------ FP8 experts
+FP8_CASES = [
+    Workload("fp8_T8_d512_E8_k2", 8, 512, 8, 1024, 2),
+    Workload("fp8_T129_d384_E16_k4", 129, 384, 16, 640, 4),
+    Workload("fp8_T300_d1152_E8_k2", 300, 1152, 8, 512, 2),
+    Workload("fp8_T1000_d256_E8_k2", 1000, 256, 8, 256, 2),
+]
+
+
+def _fp8_forward(wl, inp):
+    out = torch.empty(wl.T, wl.d, dtype=torch.float32, device=DEV)
+    ws = workspace(wl)
+    moe.moe_forward_fp8(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["bias"],
+                        inp["q1"], inp["s1"], inp["q3"], inp["s3"], inp["q2"], inp["s2"], out, ws)
+    st, code = moe.moe_get_device_error(ws)
+    assert st == 0, f"device error word {code:#x}"
+    return out.cpu().numpy().astype(np.float64)
+
+
+def _fp8_check(wl, inp, tokens=None):
+    idx, r, near = check_routing(wl, inp)
+    out = _fp8_forward(wl, inp)
+    tok = np.arange(wl.T) if tokens is None else np.asarray(tokens)
+    bias = None if inp["bias"] is None else inp["bias"].double().cpu().numpy()
+    ref = oracle.forward_fp8(bits(inp["x"]), bits(inp["Wg"]), inp["q1"].cpu().numpy(),
+                             inp["s1"].double().cpu().numpy(), inp["q3"].cpu().numpy(),
+                             inp["s3"].double().cpu().numpy(), inp["q2"].cpu().numpy(),
+                             inp["s2"].double().cpu().numpy(), wl.k, bias=bias, tokens=tok,
+                             forced=idx[tok])
+    return assert_close(out[tok], ref, wl.name)
+
+
+@pytest.mark.parametrize("wl", FP8_CASES, ids=lambda w: w.name)
+def test_forward_fp8_matches_oracle(wl):
+    inp = {k: (None if v is None else v.to(DEV)) for k, v in
+           synth.make_fp8_experts(wl, seed=7, device="cpu").items()}
+    _fp8_check(wl, inp)
+
+
+@pytest.mark.parametrize("T", [1, 8, 128])
+def test_forward_fp8_mixtral_decode(T):
+    wl = synth.mixtral_decode(T)
+    inp = synth.make_fp8_experts(wl, seed=7, device=DEV)
+    idx, _, counts = gpu_route(wl, inp)
+    tok = sample_tokens(T, 8, idx)
+    _fp8_check(wl, inp, tokens=tok)
