@@ -42,6 +42,14 @@
  *   moe_get_device_error.  Buffers must stay valid until the stream has
  *   finished the work.  Calls sharing a workspace must be ordered on one
  *   stream.
+ * Co-residency: the expert kernels run one CTA (or CTA pair) per SM.  The
+ *   large-batch kernel hands out its work through a global counter, so it
+ *   finishes whatever number of its CTAs is resident at a time.  The
+ *   small-batch (decode) kernels assign work to CTAs statically; a CTA that
+ *   waits on another CTA's results spins (bounded) on the assumption that
+ *   all CTAs of the launch are resident, which holds when the layer has the
+ *   GPU to itself.  If other work keeps SMs occupied for longer than the
+ *   bound (2 s), the wait gives up with MOE_DEVERR_TIMEOUT_EPI.
  * Errors: arguments are checked on the host before anything is launched;
  *   the first failed check is returned and nothing is enqueued.  A failed
  *   launch returns MOE_ERR_CUDA.  Problems only the GPU can see (an

@@ -6,10 +6,10 @@
 // (expert, 128 W1 and W3 rows, token tile) then down units (expert, two
 // 128-row W2 blocks, token tile, K range), weights on the MMA's M side and
 // the segment's rows on N.  What differs is the operand path:
-//   * TMA brings each 128 x 64 weight tile as e4m3 bytes (8 KB, 64-byte
-//     swizzle) -- half the bytes of bf16, the point of FP8 where the layer
-//     streams its weights from HBM (decode);
-//   * four converter warps widen the tiles to fp16 (exact: every e4m3 value is
+//   * TMA brings each 128 x 128 weight tile (a 128-column K step) as e4m3
+//     bytes (16 KB, 128-byte swizzle) -- half the bytes of bf16, the point of
+//     FP8 where the layer streams its weights from HBM (decode);
+//   * eight converter warps widen the tiles to fp16 (exact: every e4m3 value is
 //     an fp16 value) straight into the 128-byte-swizzled K-major layout the
 //     MMA reads, then release the raw stage and mark the operand stage full;
 //   * the MMA is kind::f16 with fp16 A and B (the token rows x_perm and the
@@ -23,7 +23,8 @@
 // input stage is free once the converters have read its tiles and the MMAs
 // its token rows.
 //
-// Roles: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warps 6..9 converters.
+// Roles: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warps 6..13 converters
+// (one weight row of one tile per thread).
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward) with quantised expert
@@ -44,10 +45,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kF8Threads = 320;
+constexpr int kF8Threads = 448;   // warp 0 TMA, 1 MMA, 2..5 epilogue, 6..13 converters
+constexpr int kF8ConvWarps = 8;
 constexpr int kF8MaxStages = 8;
 constexpr int kF8OpStages = 2;
-constexpr uint32_t kRawTile = 128 * 64;   // 128 weight rows x 64 e4m3 codes (8 KB)
+constexpr uint32_t kRawTile = 128 * 128;  // 128 weight rows x 128 e4m3 codes (16 KB)
 constexpr uint32_t kW16Tile = 128 * 128;  // 128 weight rows x 64 fp16 (16 KB)
 constexpr size_t kF8Fixed = 1024 /* alignment slack */ +
                             (2 * kF8MaxStages + 2 * kF8OpStages + 5) * 8 + 16 +
@@ -58,7 +60,10 @@ constexpr size_t kF8Fixed = 1024 /* alignment slack */ +
 // HBM, and a shallow one of converted fp16 weight operands.
 template <int BN>
 struct F8Cfg {
-    static constexpr uint32_t kInStage = 2 * kRawTile + BN * 128u;
+    // One input stage covers a 128-column K step: two e4m3 weight tiles and
+    // the step's token rows as two 64-column fp16 atoms; an operand stage is
+    // one 64-column half of the step, widened.
+    static constexpr uint32_t kInStage = 2 * kRawTile + 2 * BN * 128u;
     static constexpr uint32_t kOpStage = 2 * kW16Tile;
     static constexpr int kFit = static_cast<int>(
         (227 * 1024 - kF8Fixed - kF8OpStages * kOpStage) / kInStage);
@@ -67,7 +72,7 @@ struct F8Cfg {
     static constexpr uint32_t kTmemCols = 2u * kAccCols;
     static constexpr size_t kSmem =
         kF8Fixed + static_cast<size_t>(ST) * kInStage + kF8OpStages * kOpStage;
-    static_assert(ST >= 4, "pipeline depth");
+    static_assert(ST >= 2, "pipeline depth");
     static_assert(kTmemCols >= 32 && kTmemCols <= 512, "tensor memory");
     static_assert(kSmem <= 227 * 1024, "shared memory");
     static_assert(kSmem > 227 * 1024 / 2, "one CTA per SM");
@@ -229,17 +234,17 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     const int E = p.offsets ? p.E : 1;
     const int MBU = p.d_ff / 128;
     const int MBD = (p.d + 255) / 256;
-    const int KSU = p.d / 64;
-    const int KSD = p.d_ff / 64;
+    const int KSU = p.d / 128;       // 128-column K steps
+    const int KSD = p.d_ff / 128;
     const int KSPLIT = p.ksplit;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             ptx::mbar_init(&in_full[s], 1);
-            ptx::mbar_init(&in_empty[s], 4 + 1);  // converter warps (e4m3 read) + MMA (rows read)
+            ptx::mbar_init(&in_empty[s], kF8ConvWarps + 1);  // converters (e4m3 read) + MMA (rows read)
         }
         for (int s = 0; s < kF8OpStages; ++s) {
-            ptx::mbar_init(&op_full[s], 4);       // the four converter warps
+            ptx::mbar_init(&op_full[s], kF8ConvWarps);
             ptx::mbar_init(&op_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -337,7 +342,6 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                 const CUtensorMap *tb = w.up ? &tmX : &tmH;
                 const int arow0 = w.up ? w.e * p.d_ff + w.blk * 128 : w.e * p.d + w.blk * 256;
                 const int arow1 = w.up ? arow0 : arow0 + 128;
-                int ready_blk = -1;
                 for (int ks = w.k_beg; ks < w.k_end; ++ks) {
                     if (!bounded_wait(&in_empty[stage], phase ^ 1u, abort_flag, p.err,
                                       kErrTimeoutEpi)) {
@@ -346,21 +350,21 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                     }
                     uint8_t *in = ins + stage * C::kInStage;
                     ptx::mbar_arrive_expect_tx(&in_full[stage], C::kInStage);
-                    ptx::tma_load_2d_hint(in, ta0, &in_full[stage], ks * 64, arow0, pol_w);
-                    ptx::tma_load_2d_hint(in + kRawTile, ta1, &in_full[stage], ks * 64, arow1,
+                    ptx::tma_load_2d_hint(in, ta0, &in_full[stage], ks * 128, arow0, pol_w);
+                    ptx::tma_load_2d_hint(in + kRawTile, ta1, &in_full[stage], ks * 128, arow1,
                                           pol_w);
                     issued |= 1u << stage;
                     last_parity[stage] = phase;
-                    if (!w.up && (ks >> 1) != ready_blk) {
-                        ready_blk = ks >> 1;
-                        if (!f8_wait_counter(&p.h_ready[w.tile * MBU + ready_blk], 4u, abort_flag,
+                    if (!w.up) {
+                        // The step's 128 columns of H are block ks.
+                        if (!f8_wait_counter(&p.h_ready[w.tile * MBU + ks], 4u, abort_flag,
                                              p.err)) {
                             stop = true;
                             break;
                         }
                         f8_fence_proxy_async_global();
                     }
-                    ptx::tma_load_2d(in + 2 * kRawTile, tb, &in_full[stage], ks * 64, w.r0);
+                    ptx::tma_load_3d(in + 2 * kRawTile, tb, &in_full[stage], 0, w.r0, ks * 2);
                     if (++stage == static_cast<uint32_t>(ST)) {
                         stage = 0;
                         phase ^= 1u;
@@ -387,35 +391,45 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                     break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem + static_cast<uint32_t>(buf * C::kAccCols);
-                for (int ks = w.k_beg; ks < w.k_end; ++ks) {
+                for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
                     // The token rows came with the input stage; the weights
-                    // were converted into the operand stage.
-                    if (!bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma) ||
-                        !bounded_wait(&op_full[ost], ophase, abort_flag, p.err, kErrTimeoutTma)) {
+                    // were converted, one 64-column half at a time, into the
+                    // operand stages.
+                    if (!bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma)) {
                         stop = true;
                         break;
                     }
-                    ptx::tc_fence_after();
-                    const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
-                    const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage + 2 * kRawTile);
+                    for (int hf = 0; hf < 2; ++hf) {
+                        if (!bounded_wait(&op_full[ost], ophase, abort_flag, p.err,
+                                          kErrTimeoutTma)) {
+                            stop = true;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
+                        const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage +
+                                                           2 * kRawTile + hf * BN * 128);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
-                        const uint32_t acc = ((ks - w.k_beg) | kk) ? 1u : 0u;
-                        ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc, idesc,
-                                         acc);
-                        ptx::tc_mma_bf16(d0 + BN, ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
-                                         bdesc, idesc, acc);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
+                            const uint32_t acc = ((ks - w.k_beg) | hf | kk) ? 1u : 0u;
+                            ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc,
+                                             idesc, acc);
+                            ptx::tc_mma_bf16(d0 + BN,
+                                             ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
+                                             bdesc, idesc, acc);
+                        }
+                        ptx::tc_commit(&op_empty[ost]);
+                        if (++ost == static_cast<uint32_t>(kF8OpStages)) {
+                            ost = 0;
+                            ophase ^= 1u;
+                        }
                     }
-                    ptx::tc_commit(&op_empty[ost]);
+                    if (stop) break;
                     ptx::tc_commit(&in_empty[stage]);
                     if (++stage == static_cast<uint32_t>(ST)) {
                         stage = 0;
                         phase ^= 1u;
-                    }
-                    if (++ost == static_cast<uint32_t>(kF8OpStages)) {
-                        ost = 0;
-                        ophase ^= 1u;
                     }
                 }
                 if (!stop) ptx::tc_commit(&tfull[buf]);
@@ -424,36 +438,43 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             f8_drain_wait(drain, 0u);
         }
     } else if (warp >= 6) {
-        // Converters: thread r widens weight row r of both tiles of a step.
-        const int r = threadIdx.x - 192;  // 0..127
+        // Converters: thread (t, r) widens row r of weight tile t of a step.
+        const int t = (threadIdx.x - 192) >> 7;  // 0, 1
+        const int r = (threadIdx.x - 192) & 127;
         uint32_t stage = 0, phase = 0;    // input ring
         uint32_t ost = 0, ophase = 0;     // operand ring
         bool stop = false;
         for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
             const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
-            for (int ks = w.k_beg; ks < w.k_end; ++ks) {
+            for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
                 const bool ok =
-                    bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma) &&
-                    bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag, p.err, kErrTimeoutMma);
+                    bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma);
                 if (!__all_sync(0xffffffffu, ok)) {
                     *abort_flag = 1u;
                     stop = true;
                     break;
                 }
                 const uint8_t *ra = ins + stage * C::kInStage;
-                uint8_t *op = ops + ost * C::kOpStage;
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    // Raw row r: 64 bytes, 16-byte chunk j stored at chunk
-                    // j ^ ((r >> 1) & 3) (64-byte swizzle).
-                    const uint8_t *src = ra + t * kRawTile + r * 64;
+                for (int hf = 0; hf < 2; ++hf) {
+                    const bool oke =
+                        bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag, p.err, kErrTimeoutMma);
+                    if (!__all_sync(0xffffffffu, oke)) {
+                        *abort_flag = 1u;
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *op = ops + ost * C::kOpStage;
+                    // Raw row r: 128 bytes, 16-byte chunk j stored at chunk
+                    // j ^ (r & 7) (128-byte swizzle); this half is chunks
+                    // 4hf..4hf+3, i.e. columns 64hf..64hf+63.
+                    const uint8_t *src = ra + t * kRawTile + r * 128;
                     uint8_t *dst = op + t * kW16Tile + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint4 v = *reinterpret_cast<const uint4 *>(
-                            src + ((j ^ ((r >> 1) & 3)) << 4));
-                        // 16 codes = columns 16j..16j+15 -> two 16-byte fp16
-                        // chunks 2j and 2j+1 of the 128-byte-swizzled row.
+                            src + (((4 * hf + j) ^ (r & 7)) << 4));
+                        // 16 codes = columns 16j..16j+15 of the half -> two
+                        // 16-byte fp16 chunks 2j and 2j+1 of the operand row.
                         uint4 lo, hi;
                         lo.x = e4m3x2_to_f16x2(v.x);
                         lo.y = e4m3x2_to_f16x2(v.x >> 16);
@@ -466,21 +487,21 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                         *reinterpret_cast<uint4 *>(dst + (((2 * j) ^ (r & 7)) << 4)) = lo;
                         *reinterpret_cast<uint4 *>(dst + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
                     }
+                    // The MMA reads the operand through the async proxy.
+                    f8_fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&op_full[ost]);
+                    if (++ost == static_cast<uint32_t>(kF8OpStages)) {
+                        ost = 0;
+                        ophase ^= 1u;
+                    }
                 }
-                // The MMA reads the operand through the async proxy.
-                f8_fence_proxy_async_shared();
+                if (stop) break;
                 __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(&in_empty[stage]);
-                    ptx::mbar_arrive(&op_full[ost]);
-                }
+                if (lane == 0) ptx::mbar_arrive(&in_empty[stage]);
                 if (++stage == static_cast<uint32_t>(ST)) {
                     stage = 0;
                     phase ^= 1u;
-                }
-                if (++ost == static_cast<uint32_t>(kF8OpStages)) {
-                    ost = 0;
-                    ophase ^= 1u;
                 }
             }
         }
@@ -571,8 +592,8 @@ cudaError_t launch_fp8_cfg(const FfnFp8Launch &a, cudaStream_t s)
     cudaError_t e = make_tmap_e4m3(&tW1, a.q1, static_cast<uint64_t>(E) * a.f.d_ff, a.f.d);
     if (e == cudaSuccess) e = make_tmap_e4m3(&tW3, a.q3, static_cast<uint64_t>(E) * a.f.d_ff, a.f.d);
     if (e == cudaSuccess) e = make_tmap_e4m3(&tW2, a.q2, static_cast<uint64_t>(E) * a.f.d, a.f.d_ff);
-    if (e == cudaSuccess) e = make_tmap_f16(&tX, a.f.x, a.f.S, a.f.d, BN);
-    if (e == cudaSuccess) e = make_tmap_f16(&tH, a.f.H, a.f.S, a.f.d_ff, BN);
+    if (e == cudaSuccess) e = make_tmap_f16_atoms(&tX, a.f.x, a.f.S, a.f.d, BN, 2);
+    if (e == cudaSuccess) e = make_tmap_f16_atoms(&tH, a.f.H, a.f.S, a.f.d_ff, BN, 2);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(ffn_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem));

@@ -15,9 +15,9 @@
 //       Y[r, o] = (A H^T)[o, r]                  -- fp32
 // The weights are the MMA's A operand (M = 256 over the pair), the tile's
 // rows its B operand (N = rows rounded up to 16; each CTA holds N/2 of them),
-// so a ragged segment costs only the MMA columns it needs.  Per CTA and 64-wide
-// K step one stage holds 128 weight rows and 128 token rows (of which the MMA
-// reads N/2); per 256 x N x 16
+// so a ragged segment costs only the MMA columns it needs.  Per CTA and
+// 128-wide K step one stage holds 128 weight rows and 128 token rows (of which
+// the MMA reads N/2), each as two 64-column atoms; per 256 x N x 16
 // MMA each SM reads half of A and half of B from its shared memory, half what
 // two 128-row MMAs sharing one B tile would read.
 //
@@ -57,13 +57,14 @@ namespace {
 
 constexpr int kPThreads = 320;           // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int kPEpiWarps = 8;
-constexpr int kPStages = 6;
+constexpr int kPStages = 3;
 constexpr int kPMaxN = 256;              // token rows per tile (MMA N)
 constexpr uint32_t kPATile = 128 * 128;  // 128 weight rows x 64 bf16 (16 KB)
 constexpr uint32_t kPBTile = 128 * 128;  // 128 token rows x 64 bf16 (16 KB): a CTA copies
                                          // 128 rows whatever its N/2 (fewer, larger copies
                                          // measured faster than copies of just the rows used)
-constexpr uint32_t kPStage = kPATile + kPBTile;
+constexpr int kPAtoms = 2;               // 64-column atoms per K step (128 columns)
+constexpr uint32_t kPStage = kPAtoms * (kPATile + kPBTile);  // [A atoms][B atoms], 64 KB
 constexpr int kPSlots = 4;               // unit-number ring
 constexpr uint32_t kPTmemCols = 512;     // two accumulators of 256 columns
 constexpr uint32_t kPAccCols = 256;
@@ -204,9 +205,9 @@ __device__ __forceinline__ float gate_mul(float g, float b, int act)
 __global__ void __launch_bounds__(kPThreads, 1)
     ffn_pair_kernel(const __grid_constant__ CUtensorMap tmW1,   // 64-row boxes
                     const __grid_constant__ CUtensorMap tmW3,   // 64-row boxes
-                    const __grid_constant__ CUtensorMap tmW2,   // 128-row boxes
-                    const __grid_constant__ CUtensorMap tmX,    // 128-row boxes
-                    const __grid_constant__ CUtensorMap tmH,    // 128-row boxes
+                    const __grid_constant__ CUtensorMap tmW2,   // 128 rows x 2 atoms
+                    const __grid_constant__ CUtensorMap tmX,    // 128 rows x 2 atoms
+                    const __grid_constant__ CUtensorMap tmH,    // 128 rows x 2 atoms
                     const PairParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -237,8 +238,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int E = p.offsets ? p.E : 1;
     const int MBU = p.d_ff / 128;        // up blocks per expert (128 columns of H)
     const int MBD = (p.d + 255) / 256;   // down blocks per expert (256 output columns)
-    const int KSU = p.d / 64;
-    const int KSD = p.d_ff / 64;
+    const int KSU = p.d / 128;       // 128-column K steps
+    const int KSD = p.d_ff / 128;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; ++s) {
@@ -376,12 +377,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const PUnit w = decode_punit(static_cast<int>(u), u_up, s_off, s_pu, s_pd, s_tb, E);
                 const int ksteps = w.up ? KSU : KSD;
                 const int half = w.n >> 1;               // B rows this CTA holds
-                const uint32_t tx = 2u * (kPATile + kPBTile);
+                const uint32_t tx = 2u * kPStage;
                 const int arow = w.up ? w.e * p.d_ff + w.blk * 128 + static_cast<int>(cta) * 64
                                       : w.e * p.d + w.blk * 256 + static_cast<int>(cta) * 128;
                 const CUtensorMap *tb = w.up ? &tmX : &tmH;
                 const int brow = w.r0 + static_cast<int>(cta) * half;
-                int ready_blk = -1;
                 for (int ks = 0; ks < ksteps; ++ks) {
                     if (!wait_cl(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
                         stop = true;
@@ -391,26 +391,32 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     const uint32_t fb = full0 + 8 * stage;
                     if (leader) ptx::mbar_arrive_expect_tx(&full[stage], tx);
                     if (w.up) {
-                        ptx::tma_load_2d_pair(sa, &tmW1, fb, ks * 64, arow, pol);
-                        ptx::tma_load_2d_pair(sa + kPATile / 2, &tmW3, fb, ks * 64, arow, pol);
+                        // A atom a = [64 W1 rows; the same 64 W3 rows]
+#pragma unroll
+                        for (int a = 0; a < kPAtoms; ++a) {
+                            const int c = ks * 128 + a * 64;
+                            ptx::tma_load_2d_pair(sa + a * kPATile, &tmW1, fb, c, arow, pol);
+                            ptx::tma_load_2d_pair(sa + a * kPATile + kPATile / 2, &tmW3, fb, c,
+                                                  arow, pol);
+                        }
                     } else {
-                        ptx::tma_load_2d_pair(sa, &tmW2, fb, ks * 64, arow, pol);
+                        ptx::tma_load_3d_pair(sa, &tmW2, fb, 0, arow, ks * kPAtoms, pol);
                     }
                     issued |= 1u << stage;
                     last_parity[stage] = phase;
-                    if (!w.up && (ks >> 1) != ready_blk) {
-                        // These 64 columns of H belong to 128-column block
-                        // ks/2: wait until every epilogue warp of both CTAs
-                        // of its up unit stored its part.
-                        ready_blk = ks >> 1;
-                        if (!wait_ready(&p.h_ready[w.tile * MBU + ready_blk], kPReadyTarget,
-                                        abort_flag, p.err)) {
+                    if (!w.up) {
+                        // These 128 columns of H are block ks: wait until
+                        // every epilogue warp of both CTAs of its up unit
+                        // stored its part.
+                        if (!wait_ready(&p.h_ready[w.tile * MBU + ks], kPReadyTarget, abort_flag,
+                                        p.err)) {
                             stop = true;
                             break;
                         }
                         fence_proxy_async_global();
                     }
-                    ptx::tma_load_2d_pair(sa + kPATile, tb, fb, ks * 64, brow, pol);
+                    ptx::tma_load_3d_pair(sa + kPAtoms * kPATile, tb, fb, 0, brow, ks * kPAtoms,
+                                          pol);
                     if (++stage == static_cast<uint32_t>(kPStages)) {
                         stage = 0;
                         phase ^= 1u;
@@ -452,12 +458,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     }
                     ptx::tc_fence_after();
                     const uint32_t sa = ptx::smem_addr(smem + stage * kPStage);
-                    const uint32_t sb = sa + kPATile;
+                    const uint32_t sb = sa + kPAtoms * kPATile;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        ptx::tc_mma_bf16_pair(dacc, ptx::sw128_kmajor_desc(sa + kk * 32),
-                                              ptx::sw128_kmajor_desc(sb + kk * 32), idesc,
-                                              (ks | kk) ? 1u : 0u);
+                    for (int a = 0; a < kPAtoms; ++a)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            ptx::tc_mma_bf16_pair(
+                                dacc, ptx::sw128_kmajor_desc(sa + a * kPATile + kk * 32),
+                                ptx::sw128_kmajor_desc(sb + a * kPBTile + kk * 32), idesc,
+                                (ks | a | kk) ? 1u : 0u);
                     ptx::tc_commit_pair(&empty[stage], 0x3);
                     if (++stage == static_cast<uint32_t>(kPStages)) {
                         stage = 0;
@@ -624,9 +633,10 @@ cudaError_t launch_ffn_pair(const FfnLaunch &a, uint32_t *sched, cudaStream_t s)
     CUtensorMap tW1, tW3, tW2, tX, tH;
     cudaError_t e = make_tmap_bf16(&tW1, a.W1, static_cast<uint64_t>(E) * a.d_ff, a.d, 64);
     if (e == cudaSuccess) e = make_tmap_bf16(&tW3, a.W3, static_cast<uint64_t>(E) * a.d_ff, a.d, 64);
-    if (e == cudaSuccess) e = make_tmap_bf16(&tW2, a.W2, static_cast<uint64_t>(E) * a.d, a.d_ff, 128);
-    if (e == cudaSuccess) e = make_tmap_bf16(&tX, a.x, a.S, a.d, 128);
-    if (e == cudaSuccess) e = make_tmap_bf16(&tH, a.H, a.S, a.d_ff, 128);
+    if (e == cudaSuccess)
+        e = make_tmap_bf16_atoms(&tW2, a.W2, static_cast<uint64_t>(E) * a.d, a.d_ff, 128, 2);
+    if (e == cudaSuccess) e = make_tmap_bf16_atoms(&tX, a.x, a.S, a.d, 128, 2);
+    if (e == cudaSuccess) e = make_tmap_bf16_atoms(&tH, a.H, a.S, a.d_ff, 128, 2);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kPSmem));

@@ -128,11 +128,19 @@ struct FfnFp8Launch {
 };
 cudaError_t launch_ffn_fp8(const FfnFp8Launch &a, cudaStream_t s);
 
-// 2-D e4m3 (byte) matrix read in boxes of 64 columns (64-byte swizzle) by
-// 128 rows, and 2-D fp16 matrix read like make_tmap_bf16.
+// A bf16 matrix [rows, cols] viewed as (64-column atoms) so that one box
+// brings `atoms` consecutive 64-column tiles of box_rows rows (128-byte
+// swizzle), each tile at the next multiple of box_rows * 128 bytes.
+cudaError_t make_tmap_bf16_atoms(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                                 uint32_t box_rows, uint32_t atoms);
+
+// 2-D e4m3 (byte) matrix read in boxes of 128 columns (128-byte swizzle) by
+// 128 rows; fp16 matrices read like make_tmap_bf16 / make_tmap_bf16_atoms.
 cudaError_t make_tmap_e4m3(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols);
 cudaError_t make_tmap_f16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                           uint32_t box_rows);
+cudaError_t make_tmap_f16_atoms(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                                uint32_t box_rows, uint32_t atoms);
 
 // Tensor maps (tensormap.cpp side, implemented in api.cu).
 // 2-D bf16 row-major matrix [rows, cols] read in boxes of 64 columns (128 B,
