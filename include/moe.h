@@ -164,7 +164,13 @@ MOE_API moe_status moe_combine(int T, int d, int k, const float *y_perm, const i
  * the router gives every expert its token list and the expert kernel reads
  * the rows of x through it; the rows of an expert are then not in token
  * order inside the workspace, which does not change out (each row's expert
- * output does not depend on its position; slots are summed in order). */
+ * output does not depend on its position; slots are summed in order).  For
+ * d > 1024 with k <= 2, no shared expert and segments large enough for the
+ * CTA-pair expert kernel (prefill), the combine runs inside that kernel: its
+ * down units add w[t,j] * y into out[t], which the dispatch zeroed first.
+ * At most two terms reach an element and two terms added onto zero give the
+ * same sum in either order, so out is still the same from run to run (it
+ * may differ in the last bit from moe_combine's fused multiply-add). */
 MOE_API moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
                        const moe_bf16 *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
                        const moe_bf16 *W2, float *out, void *ws, size_t ws_bytes,
@@ -298,7 +304,8 @@ MOE_API moe_status moe_expert_ffn_static_error(uint32_t *code, moe_stream_t stre
  *   events[1] before the dispatch scatter   events[4] before the combine
  *   events[2] before the expert FFN kernel  events[5] after the combine
  * (events[3] and events[4] mark the same point when there is no shared
- * expert).  n_events must be MOE_TRACE_EVENTS.  While `stream` is being
+ * expert, events[4] and events[5] when the expert kernel did the combine,
+ * see moe_forward).  n_events must be MOE_TRACE_EVENTS.  While `stream` is being
  * captured into a CUDA graph the events are recorded as graph event nodes.
  * The layer's work and results are those of moe_forward_ex. */
 MOE_API moe_status moe_forward_traced(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,

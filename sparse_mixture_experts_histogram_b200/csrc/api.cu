@@ -29,8 +29,8 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
     size_t tilectr, hready, hready_s, gcnt;
     size_t zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
-    size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, slotpos, perm, xperm, H, Y, Hs,
-        Ys, total;
+    size_t tilecnt, tilebase, rank, offsets, counts, idx, w, row, slotpos, slotrow, perm, xperm, H,
+        Y, Hs, Ys, total;
 };
 
 // Token lists of the slot mode: one row of perm_stride entries per expert.
@@ -70,6 +70,7 @@ Layout forward_layout(int T, int d, int E, int d_ff, int k, int d_ffs)
     L.w = take(S * 4);
     L.row = take(S * 4);
     L.slotpos = take(S * 4);
+    L.slotrow = take(S * 4);
     L.perm = take(static_cast<size_t>(E) * perm_stride(T) * 4);
     L.xperm = take(S * d * 2);
     L.H = take(S * d_ff * 2);
@@ -364,10 +365,15 @@ static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const mo
                            const int32_t *offsets, const moe_bf16 *W1, const moe_bf16 *W3,
                            const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *h_ready,
                            uint32_t *sched, uint32_t *err, cudaStream_t s, bool pdl, int ksplit,
-                           int act = 0)
+                           int act = 0, float *out = nullptr, const int32_t *slot_of_row = nullptr,
+                           const float *gate_w = nullptr, int k = 1)
 {
     FfnLaunch f{};
     f.act = act;
+    f.out = out;
+    f.slot_of_row = slot_of_row;
+    f.gate_w = gate_w;
+    f.k = k;
     f.E = E;
     f.d = d;
     f.d_ff = d_ff;
@@ -503,6 +509,18 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     // Overlapping launches pay off for small layers; for large ones they only
     // take SM slots early (measured: neutral to slightly negative).
     const bool pdl = events == nullptr && S <= 4096;
+    // A token never picks one expert twice, so no segment exceeds T rows.
+    // (The capacity path of a narrow layer runs the general expert kernel on
+    // the permuted copy, without a K split.)
+    const int ksplit = (cap >= 0 && ffn_small_supported(d)) ? 1 : ffn_splits(S, E, d, d_ff);
+    // With k <= 2, no shared expert and the CTA-pair expert kernel (which
+    // never splits K), the down units write the gate-weighted sum into out
+    // themselves: at most two terms reach each element, and two terms added
+    // onto zero give one result in either order.  No Y round trip and no
+    // combine launch then.
+    const bool fused_out =
+        !narrow && k <= 2 && d_ff_shared == 0 && ffn_pair_eligible(S, E, ksplit);
+    int32_t *slotrow = reinterpret_cast<int32_t *>(wsb + L.slotrow);
     if ((st = mark(events, 0, s)) != MOE_OK) return st;
     st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
                     reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s, narrow, wmode,
@@ -524,16 +542,14 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         c.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
         c.x_perm = xperm;
         c.row_of_slot = row;
+        c.slot_of_row = fused_out ? slotrow : nullptr;
+        c.out_zero = fused_out ? out : nullptr;
         c.err = err;
         c.pdl = pdl;
         st = from_cuda(launch_scatter(c, s));
         if (st != MOE_OK) return st;
     }
 
-    // A token never picks one expert twice, so no segment exceeds T rows.
-    // (The capacity path of a narrow layer runs the general expert kernel on
-    // the permuted copy, without a K split.)
-    const int ksplit = (cap >= 0 && ffn_small_supported(d)) ? 1 : ffn_splits(S, E, d, d_ff);
     if ((st = mark(events, 2, s)) != MOE_OK) return st;
     if (narrow) {
         FfnLaunch f{};
@@ -563,7 +579,8 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     } else {
         st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
                       reinterpret_cast<uint32_t *>(wsb + L.hready),
-                      reinterpret_cast<uint32_t *>(wsb + 16), err, s, pdl, ksplit, act);
+                      reinterpret_cast<uint32_t *>(wsb + 16), err, s, pdl, ksplit, act,
+                      fused_out ? out : nullptr, slotrow, w, k);
     }
     if (st != MOE_OK) return st;
 
@@ -579,6 +596,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         shared_y = Ys;
     }
     if ((st = mark(events, 4, s)) != MOE_OK) return st;
+    if (fused_out) return mark(events, 5, s);
 
     CombineLaunch cb{};
     cb.T = T;

@@ -57,6 +57,8 @@ struct ScatterParams {
     const int32_t *idx, *rank, *tilebase;
     uint4 *x_perm;
     int32_t *row_of_slot;
+    int32_t *slot_of_row;  // or nullptr
+    float4 *out_zero;      // or nullptr
     uint32_t *err;
     int S;
     int to_f16;  // convert the rows to fp16 on the way
@@ -95,6 +97,7 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
         if (c == 0) {
             if (my_row < 0 && !dropped) atomicOr(p.err, kErrIndex);
             p.row_of_slot[s] = my_row;
+            if (p.slot_of_row != nullptr && my_row >= 0) p.slot_of_row[my_row] = static_cast<int>(s);
         }
     }
     int rows[kMaxK];
@@ -118,6 +121,18 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
                 const float hi = __uint_as_float(w[i] & 0xffff0000u);
                 const __half2 h = __floats2half2_rn(lo, hi);
                 w[i] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+        }
+    }
+    if (p.out_zero != nullptr) {
+        // The same columns of out (fp32: two 16-byte vectors per bf16 one).
+        float4 *o = p.out_zero + static_cast<size_t>(t) * (2 * nv);
+#pragma unroll
+        for (int u = 0; u < kScatterVec; ++u) {
+            const int v = (c * kScatterVec + u) * 32 + lane;
+            if (v < nv) {
+                o[2 * v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                o[2 * v + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
     }
@@ -171,6 +186,8 @@ cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s)
     p.tilebase = a.tilebase;
     p.x_perm = reinterpret_cast<uint4 *>(a.x_perm);
     p.row_of_slot = a.row_of_slot;
+    p.slot_of_row = a.slot_of_row;
+    p.out_zero = reinterpret_cast<float4 *>(a.out_zero);
     p.err = a.err;
     p.S = a.T * a.k;
     p.to_f16 = a.to_f16 ? 1 : 0;

@@ -9,9 +9,15 @@
 //   * TMA brings each 128 x 128 weight tile (a 128-column K step) as e4m3
 //     bytes (16 KB, 128-byte swizzle) -- half the bytes of bf16, the point of
 //     FP8 where the layer streams its weights from HBM (decode);
-//   * eight converter warps widen the tiles to fp16 (exact: every e4m3 value is
-//     an fp16 value) straight into the 128-byte-swizzled K-major layout the
-//     MMA reads, then release the raw stage and mark the operand stage full;
+//   * eight converter warps widen the tiles to fp16 by bit moves (exact: every
+//     e4m3 value times 2^-8 is an fp16 value; the 2^8 goes into the row
+//     scale), then release the raw stage and mark the operand stage full.  With token tiles of up to 64 rows (decode) the widened weights go
+//     to tensor memory, one weight row per lane, and the MMA reads its A
+//     operand from there: the shared-memory traffic per weight code is then
+//     the TMA write and one converter read, which leaves the converters and
+//     the memory system, not shared-memory bandwidth, as the limit.  With
+//     128-row token tiles the accumulators fill tensor memory, and the
+//     operands go to shared memory in the 128-byte-swizzled K-major layout;
 //   * the MMA is kind::f16 with fp16 A and B (the token rows x_perm and the
 //     hidden activations H are fp16 in this path) and fp32 accumulators;
 //   * the epilogue multiplies each accumulator row by its weight row's scale
@@ -32,7 +38,6 @@
 // deployment section on quantisation).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -48,30 +53,39 @@ namespace {
 constexpr int kF8Threads = 448;   // warp 0 TMA, 1 MMA, 2..5 epilogue, 6..13 converters
 constexpr int kF8ConvWarps = 8;
 constexpr int kF8MaxStages = 8;
-constexpr int kF8OpStages = 2;
+constexpr int kF8MaxOps = 6;     // operand ring depth, tensor-memory operands
+constexpr int kF8OpStages = 2;   // operand ring depth, shared-memory operands
 constexpr uint32_t kRawTile = 128 * 128;  // 128 weight rows x 128 e4m3 codes (16 KB)
 constexpr uint32_t kW16Tile = 128 * 128;  // 128 weight rows x 64 fp16 (16 KB)
 constexpr size_t kF8Fixed = 1024 /* alignment slack */ +
-                            (2 * kF8MaxStages + 2 * kF8OpStages + 5) * 8 + 16 +
+                            (2 * kF8MaxStages + 2 * kF8MaxOps + 5) * 8 + 16 +
                             4 * (kMaxE + 1) * sizeof(int32_t) + 64;
 
 // Two rings: a deep one of input stages (the e4m3 weight tiles of a K step
 // and its token rows, fp16), which keeps enough bytes in flight to stream
-// HBM, and a shallow one of converted fp16 weight operands.
+// HBM, and one of converted fp16 weight operands.
 template <int BN>
 struct F8Cfg {
+    // Operands in tensor memory when the double-buffered accumulators
+    // (2 x 2 x BN columns) leave room for at least four operand stages.
+    static constexpr bool kTA = BN <= 64;
     // One input stage covers a 128-column K step: two e4m3 weight tiles and
     // the step's token rows as two 64-column fp16 atoms; an operand stage is
-    // one 64-column half of the step, widened.
+    // one 64-column half of the step, widened: 2 x 16 KB of shared memory, or
+    // 2 x 32 tensor-memory columns (two fp16 of K per 32-bit column).
     static constexpr uint32_t kInStage = 2 * kRawTile + 2 * BN * 128u;
-    static constexpr uint32_t kOpStage = 2 * kW16Tile;
-    static constexpr int kFit = static_cast<int>(
-        (227 * 1024 - kF8Fixed - kF8OpStages * kOpStage) / kInStage);
-    static constexpr int ST = kFit < kF8MaxStages ? kFit : kF8MaxStages;
     static constexpr int kAccCols = 2 * BN;
-    static constexpr uint32_t kTmemCols = 2u * kAccCols;
+    static constexpr int OPS = kTA ? (512 - 2 * kAccCols) / 64 : kF8OpStages;
+    static constexpr uint32_t kOpStage = kTA ? 0u : 2 * kW16Tile;  // shared memory
+    static constexpr uint32_t kOpCol0 = 2u * kAccCols;            // tensor memory
+    static constexpr int kFit = static_cast<int>(
+        (227 * 1024 - kF8Fixed - OPS * kOpStage) / kInStage);
+    static constexpr int ST = kFit < kF8MaxStages ? kFit : kF8MaxStages;
+    static constexpr uint32_t kTmemCols = kTA ? 512u : 2u * kAccCols;
     static constexpr size_t kSmem =
-        kF8Fixed + static_cast<size_t>(ST) * kInStage + kF8OpStages * kOpStage;
+        kF8Fixed + static_cast<size_t>(ST) * kInStage + OPS * kOpStage;
+    static_assert(OPS >= 2 && OPS <= kF8MaxOps, "operand ring");
+    static_assert(!kTA || kOpCol0 + 64u * OPS <= kTmemCols, "tensor-memory operands");
     static_assert(ST >= 2, "pipeline depth");
     static_assert(kTmemCols >= 32 && kTmemCols <= 512, "tensor memory");
     static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -185,12 +199,26 @@ __device__ __forceinline__ int f8_scan(int v, int lane)
     return v;
 }
 
-// Two e4m3 codes (low byte first) to two fp16 values (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two)
+// Widening by bit moves: an e4m3 code s.eeee.mmm placed as the fp16 bit
+// pattern s.0eeee.mmm0000000 is the code's value times 2^-8 -- the exponent
+// field keeps its bits while the bias goes from 7 to 15, and e4m3 subnormals
+// (e = 0, value m/8 * 2^-6) land on fp16 subnormals (m/8 * 2^-14).  Every
+// e4m3 value times 2^-8 is an fp16 value, so the widening is exact; the
+// epilogue folds the 2^8 into the row scale, and since every product of the
+// MMA is scaled by the same power of two, the fp32 sums are exact multiples
+// of the unscaled ones.  It costs the converters integer operations only.
+constexpr float kF8WidenScale = 256.0f;
+
+// Four e4m3 codes (low byte first) to four fp16 values times 2^-8, two per
+// word.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t v, uint32_t &lo, uint32_t &hi)
 {
-    const __half2_raw h =
-        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+    // Per code: the high byte of the fp16 (s, 0, e3..e0, m2, m1) and the low
+    // byte (m0, then zeros).
+    const uint32_t hb = ((v >> 1) & 0x3f3f3f3fu) | (v & 0x80808080u);
+    const uint32_t lb = (v << 7) & 0x80808080u;
+    lo = __byte_perm(lb, hb, 0x5140);  // codes 0, 1
+    hi = __byte_perm(lb, hb, 0x7362);  // codes 2, 3
 }
 
 // Instruction descriptor of kind::f16 with fp16 A/B, fp32 D, both K-major.
@@ -215,13 +243,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     const int lane = threadIdx.x & 31;
 
     constexpr int ST = C::ST;
-    uint8_t *ops = smem;                                       // [2] fp16 weight operands
-    uint8_t *ins = smem + kF8OpStages * C::kOpStage;          // [ST] e4m3 tiles + token rows
+    constexpr int OPS = C::OPS;
+    uint8_t *ops = smem;                                       // [OPS] fp16 weight operands
+    uint8_t *ins = smem + OPS * C::kOpStage;                   // [ST] e4m3 tiles + token rows
     uint64_t *in_full = reinterpret_cast<uint64_t *>(ins + ST * C::kInStage);
     uint64_t *in_empty = in_full + kF8MaxStages;
     uint64_t *op_full = in_empty + kF8MaxStages;
-    uint64_t *op_empty = op_full + kF8OpStages;
-    uint64_t *tfull = op_empty + kF8OpStages;  // [2]
+    uint64_t *op_empty = op_full + kF8MaxOps;
+    uint64_t *tfull = op_empty + kF8MaxOps;  // [2]
     uint64_t *tempty = tfull + 2;             // [2]
     uint64_t *drain = tempty + 2;             // [1]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -243,7 +272,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             ptx::mbar_init(&in_full[s], 1);
             ptx::mbar_init(&in_empty[s], kF8ConvWarps + 1);  // converters (e4m3 read) + MMA (rows read)
         }
-        for (int s = 0; s < kF8OpStages; ++s) {
+        for (int s = 0; s < OPS; ++s) {
             ptx::mbar_init(&op_full[s], kF8ConvWarps);
             ptx::mbar_init(&op_empty[s], 1);
         }
@@ -406,21 +435,34 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                             break;
                         }
                         ptx::tc_fence_after();
-                        const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
                         const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage +
                                                            2 * kRawTile + hf * BN * 128);
+                        if constexpr (C::kTA) {
+                            // A: tile t of the stage at columns
+                            // kOpCol0 + 64 ost + 32 t, 16 K elements per 8 columns.
+                            const uint32_t ta = tmem + C::kOpCol0 + 64u * ost;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
-                            const uint32_t acc = ((ks - w.k_beg) | hf | kk) ? 1u : 0u;
-                            ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc,
-                                             idesc, acc);
-                            ptx::tc_mma_bf16(d0 + BN,
-                                             ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
-                                             bdesc, idesc, acc);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
+                                const uint32_t acc = ((ks - w.k_beg) | hf | kk) ? 1u : 0u;
+                                ptx::tc_mma_f16_ts(d0, ta + 8u * kk, bdesc, idesc, acc);
+                                ptx::tc_mma_f16_ts(d0 + BN, ta + 32u + 8u * kk, bdesc, idesc, acc);
+                            }
+                        } else {
+                            const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
+                                const uint32_t acc = ((ks - w.k_beg) | hf | kk) ? 1u : 0u;
+                                ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc,
+                                                 idesc, acc);
+                                ptx::tc_mma_bf16(d0 + BN,
+                                                 ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
+                                                 bdesc, idesc, acc);
+                            }
                         }
                         ptx::tc_commit(&op_empty[ost]);
-                        if (++ost == static_cast<uint32_t>(kF8OpStages)) {
+                        if (++ost == static_cast<uint32_t>(OPS)) {
                             ost = 0;
                             ophase ^= 1u;
                         }
@@ -438,70 +480,131 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             f8_drain_wait(drain, 0u);
         }
     } else if (warp >= 6) {
-        // Converters: thread (t, r) widens row r of weight tile t of a step.
-        const int t = (threadIdx.x - 192) >> 7;  // 0, 1
-        const int r = (threadIdx.x - 192) & 127;
+        // Converters: warp w widens rows 32 (w % 4) .. 32 (w % 4) + 31 of
+        // weight tile (w - 6) / 4 of a step, one row per thread -- the rows
+        // of the tensor-memory lanes the warp may access.
+        const int t = (warp - 6) >> 2;  // 0, 1
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + C::kOpCol0 +
+                               32u * static_cast<uint32_t>(t);
         uint32_t stage = 0, phase = 0;    // input ring
         uint32_t ost = 0, ophase = 0;     // operand ring
         bool stop = false;
-        for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
-            const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
-            for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
-                const bool ok =
-                    bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    *abort_flag = 1u;
-                    stop = true;
-                    break;
-                }
-                const uint8_t *ra = ins + stage * C::kInStage;
-                for (int hf = 0; hf < 2; ++hf) {
-                    const bool oke =
-                        bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag, p.err, kErrTimeoutMma);
-                    if (!__all_sync(0xffffffffu, oke)) {
+        if constexpr (C::kTA) {
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+                for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
+                    const bool ok =
+                        bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma);
+                    if (!__all_sync(0xffffffffu, ok)) {
                         *abort_flag = 1u;
                         stop = true;
                         break;
                     }
-                    uint8_t *op = ops + ost * C::kOpStage;
                     // Raw row r: 128 bytes, 16-byte chunk j stored at chunk
-                    // j ^ (r & 7) (128-byte swizzle); this half is chunks
-                    // 4hf..4hf+3, i.e. columns 64hf..64hf+63.
-                    const uint8_t *src = ra + t * kRawTile + r * 128;
-                    uint8_t *dst = op + t * kW16Tile + (r >> 3) * 1024 + (r & 7) * 128;
+                    // j ^ (r & 7) (128-byte swizzle).
+                    const uint8_t *src = ins + stage * C::kInStage + t * kRawTile + r * 128;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const bool oke = bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag,
+                                                      p.err, kErrTimeoutMma);
+                        if (!__all_sync(0xffffffffu, oke)) {
+                            *abort_flag = 1u;
+                            stop = true;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        // Codes 64hf .. 64hf + 63 of the row (chunks 4hf ..
+                        // 4hf + 3) -> the tile's 32 columns of the stage.
+                        uint32_t v32[32];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(
-                            src + (((4 * hf + j) ^ (r & 7)) << 4));
-                        // 16 codes = columns 16j..16j+15 of the half -> two
-                        // 16-byte fp16 chunks 2j and 2j+1 of the operand row.
-                        uint4 lo, hi;
-                        lo.x = e4m3x2_to_f16x2(v.x);
-                        lo.y = e4m3x2_to_f16x2(v.x >> 16);
-                        lo.z = e4m3x2_to_f16x2(v.y);
-                        lo.w = e4m3x2_to_f16x2(v.y >> 16);
-                        hi.x = e4m3x2_to_f16x2(v.z);
-                        hi.y = e4m3x2_to_f16x2(v.z >> 16);
-                        hi.z = e4m3x2_to_f16x2(v.w);
-                        hi.w = e4m3x2_to_f16x2(v.w >> 16);
-                        *reinterpret_cast<uint4 *>(dst + (((2 * j) ^ (r & 7)) << 4)) = lo;
-                        *reinterpret_cast<uint4 *>(dst + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(
+                                src + (((4 * hf + j) ^ (r & 7)) << 4));
+                            e4m3x4_to_f16x4(v.x, v32[8 * j + 0], v32[8 * j + 1]);
+                            e4m3x4_to_f16x4(v.y, v32[8 * j + 2], v32[8 * j + 3]);
+                            e4m3x4_to_f16x4(v.z, v32[8 * j + 4], v32[8 * j + 5]);
+                            e4m3x4_to_f16x4(v.w, v32[8 * j + 6], v32[8 * j + 7]);
+                        }
+                        ptx::tmem_st16(t_row + 64u * ost,
+                                       *reinterpret_cast<const uint32_t(*)[16]>(&v32[0]));
+                        ptx::tmem_st16(t_row + 64u * ost + 16u,
+                                       *reinterpret_cast<const uint32_t(*)[16]>(&v32[16]));
+                        // The MMA thread reads the operand after the arrival.
+                        ptx::tc_wait_st();
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&op_full[ost]);
+                        if (++ost == static_cast<uint32_t>(OPS)) {
+                            ost = 0;
+                            ophase ^= 1u;
+                        }
                     }
-                    // The MMA reads the operand through the async proxy.
-                    f8_fence_proxy_async_shared();
+                    if (stop) break;
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&op_full[ost]);
-                    if (++ost == static_cast<uint32_t>(kF8OpStages)) {
-                        ost = 0;
-                        ophase ^= 1u;
+                    if (lane == 0) ptx::mbar_arrive(&in_empty[stage]);
+                    if (++stage == static_cast<uint32_t>(ST)) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
-                if (stop) break;
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&in_empty[stage]);
-                if (++stage == static_cast<uint32_t>(ST)) {
-                    stage = 0;
-                    phase ^= 1u;
+            }
+        } else {
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
+                for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
+                    const bool ok =
+                        bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        *abort_flag = 1u;
+                        stop = true;
+                        break;
+                    }
+                    const uint8_t *ra = ins + stage * C::kInStage;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const bool oke =
+                            bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag, p.err, kErrTimeoutMma);
+                        if (!__all_sync(0xffffffffu, oke)) {
+                            *abort_flag = 1u;
+                            stop = true;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        // Raw row r: 128 bytes, 16-byte chunk j stored at chunk
+                        // j ^ (r & 7) (128-byte swizzle); this half is chunks
+                        // 4hf..4hf+3, i.e. columns 64hf..64hf+63.
+                        const uint8_t *src = ra + t * kRawTile + r * 128;
+                        uint8_t *op = ops + ost * C::kOpStage;
+                        uint8_t *dst = op + t * kW16Tile + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(
+                                src + (((4 * hf + j) ^ (r & 7)) << 4));
+                            // 16 codes = columns 16j..16j+15 of the half -> two
+                            // 16-byte fp16 chunks 2j and 2j+1 of the operand row.
+                            uint4 lo, hi;
+                            e4m3x4_to_f16x4(v.x, lo.x, lo.y);
+                            e4m3x4_to_f16x4(v.y, lo.z, lo.w);
+                            e4m3x4_to_f16x4(v.z, hi.x, hi.y);
+                            e4m3x4_to_f16x4(v.w, hi.z, hi.w);
+                            *reinterpret_cast<uint4 *>(dst + (((2 * j) ^ (r & 7)) << 4)) = lo;
+                            *reinterpret_cast<uint4 *>(dst + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+                        }
+                        // The MMA reads the operand through the async proxy.
+                        f8_fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&op_full[ost]);
+                        if (++ost == static_cast<uint32_t>(OPS)) {
+                            ost = 0;
+                            ophase ^= 1u;
+                        }
+                    }
+                    if (stop) break;
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&in_empty[stage]);
+                    if (++stage == static_cast<uint32_t>(ST)) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
         }
@@ -522,12 +625,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             float sa, sb;
             if (w.up) {
                 const int f = w.blk * 128 + row_in_blk;
-                sa = p.s1[static_cast<size_t>(w.e) * p.d_ff + f];
-                sb = p.s3[static_cast<size_t>(w.e) * p.d_ff + f];
+                sa = kF8WidenScale * p.s1[static_cast<size_t>(w.e) * p.d_ff + f];
+                sb = kF8WidenScale * p.s3[static_cast<size_t>(w.e) * p.d_ff + f];
             } else {
                 const int o0 = w.blk * 256 + row_in_blk;
-                sa = o0 < p.d ? p.s2[static_cast<size_t>(w.e) * p.d + o0] : 0.0f;
-                sb = o0 + 128 < p.d ? p.s2[static_cast<size_t>(w.e) * p.d + o0 + 128] : 0.0f;
+                sa = o0 < p.d ? kF8WidenScale * p.s2[static_cast<size_t>(w.e) * p.d + o0] : 0.0f;
+                sb = o0 + 128 < p.d
+                         ? kF8WidenScale * p.s2[static_cast<size_t>(w.e) * p.d + o0 + 128]
+                         : 0.0f;
             }
             for (int c0 = 0; c0 < w.valid; c0 += 32) {
                 uint32_t a[32], b[32];

@@ -13,6 +13,11 @@
 //   down units (e, 256 output columns, tile):
 //       even CTA A = W2_e rows o0..o0+127, odd CTA A = rows o0+128..o0+255
 //       Y[r, o] = (A H^T)[o, r]                  -- fp32
+//       or, for top-k with k <= 2, the gate-weighted combine in place:
+//       out[t, o] += w[t, j] * (A H^T)[o, r] for the slot (t, j) of row r
+//       ("MoE" (theaiera.top) sec. 10.4, the weighted index_add back to the
+//       tokens), onto an out the scatter zeroed; at most two terms reach an
+//       element, and two terms added onto zero give one sum in either order
 // The weights are the MMA's A operand (M = 256 over the pair), the tile's
 // rows its B operand (N = rows rounded up to 16; each CTA holds N/2 of them),
 // so a ragged segment costs only the MMA columns it needs.  Per CTA and
@@ -33,7 +38,7 @@
 // even CTA issues the MMAs into one of two tensor-memory accumulators and
 // signals both CTAs, warps 2..9 drain the accumulator: up units exchange the
 // W1 and W3 products between lane quarters through shared memory and store
-// H; down units write their fp32 outputs.
+// H; down units write their fp32 outputs (or add them, weighted, into out).
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward; "Mixtral and MoE
@@ -89,6 +94,14 @@ struct PairParams {
     uint32_t *sched;         // unit counter, zero before the launch
     uint32_t *err;
     int act;                 // expert activation: 0 silu(g) * b, 1 sigmoid(g) * b
+    // Weighted output (k <= 2): when out is set, the down units add
+    // gate_w[s] * y into out[s / k] (s = slot_of_row[row]) instead of
+    // writing Y.  Two terms added onto zero give the same sum in either
+    // order, so the result does not depend on which unit finishes first.
+    float *out;
+    const int32_t *slot_of_row;
+    const float *gate_w;
+    int k;
 };
 
 struct PUnit {
@@ -561,7 +574,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     uint32_t r[32];
                     ptx::tmem_ld32(tb + static_cast<uint32_t>(c0), r);
                     ptx::tc_wait_ld();
-                    if (has) {
+                    if (p.out != nullptr) {
+                        // Lane j fetches the slot and gate weight of row
+                        // r0 + c0 + j; row j's values go to all lanes.
+                        int sl = -1;
+                        float gw = 0.0f;
+                        if (c0 + lane < w.valid) {
+                            const int v = p.slot_of_row[w.r0 + c0 + lane];
+                            if (static_cast<unsigned>(v) < static_cast<unsigned>(p.S)) {
+                                sl = v;
+                                gw = p.gate_w[v];
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int slj = __shfl_sync(0xffffffffu, sl, j);
+                            const float gwj = __shfl_sync(0xffffffffu, gw, j);
+                            if (has && slj >= 0)
+                                atomicAdd(p.out + static_cast<size_t>(slj / p.k) * p.d + o,
+                                          gwj * __uint_as_float(r[j]));
+                        }
+                    } else if (has) {
                         float *yc = p.Y + static_cast<size_t>(w.r0 + c0) * p.d + o;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
@@ -654,6 +687,10 @@ cudaError_t launch_ffn_pair(const FfnLaunch &a, uint32_t *sched, cudaStream_t s)
     p.sched = sched;
     p.err = a.err;
     p.act = a.act;
+    p.out = a.out;
+    p.slot_of_row = a.slot_of_row;
+    p.gate_w = a.gate_w;
+    p.k = a.k < 1 ? 1 : a.k;
 
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kPThreads);

@@ -52,6 +52,11 @@ struct ScatterLaunch {
     uint32_t *err;
     bool pdl;  // launched right after another kernel of this library
     bool to_f16;  // write x_perm as fp16 (the FP8 expert path) instead of bf16
+    // For the expert kernel's weighted output (FfnLaunch::out), when set:
+    // slot_of_row[row] = t*k + j for every row that got a slot, and out[T, d]
+    // set to zero.
+    int32_t *slot_of_row;
+    float *out_zero;
 };
 
 struct FfnLaunch {
@@ -82,6 +87,15 @@ struct FfnLaunch {
     int x_rows;
     const int32_t *counts;    // [E] rows per segment (the router's totals); offsets are
     int32_t *offsets_out;     // their exclusive prefix, written here [E+1]
+    // CTA-pair kernel only: when out is set, the down units add their rows,
+    // weighted, into out[T, d] (zero before the launch) instead of writing Y:
+    // out[s / k] += gate_w[s] * y_row with s = slot_of_row[row].  For k <= 2
+    // and no K split, where two terms added onto zero give the same sum in
+    // either order.
+    float *out;
+    const int32_t *slot_of_row;
+    const float *gate_w;
+    int k;
 };
 
 struct CombineLaunch {

@@ -239,7 +239,11 @@ SMALL_FORWARD = [synth.small(), *synth.sweep(),
                  Workload("T1", 1, 512, 8, 1024, 2),
                  Workload("T129_ragged", 129, 384, 16, 640, 3),
                  Workload("E256_k8_small", 200, 256, 256, 128, 8),
-                 Workload("shared_small", 150, 256, 32, 256, 4, d_ff_shared=384)]
+                 Workload("shared_small", 150, 256, 32, 256, 4, d_ff_shared=384),
+                 # wide layers on the CTA-pair expert kernel with k <= 2: the
+                 # down units add the gate-weighted rows into out themselves
+                 Workload("wide_pair_T1100_d1152_E8_k2", 1100, 1152, 8, 512, 2),
+                 Workload("wide_pair_T1200_d1152_E4_k1", 1200, 1152, 4, 256, 1)]
 
 
 @pytest.mark.parametrize("wl", SMALL_FORWARD, ids=lambda w: w.name)
@@ -286,13 +290,16 @@ def test_forward_is_deterministic_and_graph_capturable():
     assert torch.equal(out, a)
 
 
-@pytest.mark.parametrize("wl", [synth.sweep()[-1], Workload("E64_k4_T1000", 1000, 384, 64, 256, 4)],
+@pytest.mark.parametrize("wl", [synth.sweep()[-1], Workload("E64_k4_T1000", 1000, 384, 64, 256, 4),
+                                Workload("wide_pair_T1100_d1152_E8_k2", 1100, 1152, 8, 512, 2)],
                          ids=lambda w: w.name)
-def test_forward_narrow_repeatable_whatever_the_slot_order(wl):
+def test_forward_repeatable_whatever_the_order(wl):
     # Narrow layers place each expert's rows in the order the router's
-    # atomics hand out positions, which differs from run to run; the output
-    # must not (each row's expert output is independent of its position and
-    # slots are summed in order).
+    # atomics hand out positions, and wide layers with k <= 2 add each
+    # token's weighted rows into out in the order their units finish; both
+    # orders differ from run to run, the output must not (each row's expert
+    # output is independent of its position, narrow slots are summed in
+    # order, and two terms added onto zero give one sum in either order).
     inp = _inputs(wl)
     ws = workspace(wl)
     first = gpu_forward(wl, inp, ws).clone()
