@@ -553,9 +553,21 @@ def gpu_arm(args):
     if any(w.d <= 1024 for w in wls):
         kinds.append("ffn_small_kernel (d <= 1024: x rows gathered through the experts' token "
                      "lists, W1|W3 + SwiGLU and W2 per hidden chunk, one persistent launch)")
-    if any(w.d > 1024 for w in wls):
-        kinds.append("ffn_kernel (grouped W1|W3 + SwiGLU, then W2, one persistent launch)")
-    roof["kernel"] = "; ".join(kinds)
+    for w in wls:
+        if w.d <= 1024:
+            continue
+        # the library's choice: CTA pairs once a segment is expected to hold
+        # more than 64 rows (1.5x the mean), one CTA per SM below that
+        if is_fp8(w):
+            kinds.append("ffn_fp8_kernel (e4m3 weights widened in tensor memory, W1|W3 + "
+                         "SwiGLU, then W2, one persistent launch)")
+        elif 3 * w.T * w.k > 128 * w.E:
+            kinds.append("ffn_pair_kernel (cta_group::2 MMAs on CTA pairs, W1|W3 + SwiGLU, then W2"
+                         + (", gate-weighted rows added into out" if w.k <= 2 and not w.d_ff_shared
+                            else "") + ", one persistent launch)")
+        else:
+            kinds.append("ffn_kernel (grouped W1|W3 + SwiGLU, then W2, one persistent launch)")
+    roof["kernel"] = "; ".join(dict.fromkeys(kinds))
     roof["algorithmic_bytes_per_launch"] = sum(up_bytes) / len(up_bytes)
     roof["flops_per_launch"] = sum(up_flops) / len(up_flops)
     roof["launch_ms"] = sum(up_time) / len(up_time)

@@ -66,8 +66,14 @@ constexpr int kPStages = 3;
 constexpr int kPMaxN = 256;              // token rows per tile (MMA N)
 constexpr uint32_t kPATile = 128 * 128;  // 128 weight rows x 64 bf16 (16 KB)
 constexpr uint32_t kPBTile = 128 * 128;  // 128 token rows x 64 bf16 (16 KB): a CTA copies
-                                         // 128 rows whatever its N/2 (fewer, larger copies
+                                         // 128 rows for N/2 > kPBShort (fewer, larger copies
                                          // measured faster than copies of just the rows used)
+// Token tiles of at most 2 * kPBShort rows (the two-tile segments of the
+// 256-expert layer, about 136 rows each) copy kPBShort rows per CTA instead:
+// the weight stream then needs fewer bytes in flight to stay ahead of the
+// MMAs, whose work per K step shrinks with N.
+constexpr int kPBShort = 80;
+constexpr uint32_t kPBShortTile = kPBShort * 128;  // 10 KB, a multiple of the 1 KB swizzle atom
 constexpr int kPAtoms = 2;               // 64-column atoms per K step (128 columns)
 constexpr uint32_t kPStage = kPAtoms * (kPATile + kPBTile);  // [A atoms][B atoms], 64 KB
 constexpr int kPSlots = 4;               // unit-number ring
@@ -221,6 +227,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     const __grid_constant__ CUtensorMap tmW2,   // 128 rows x 2 atoms
                     const __grid_constant__ CUtensorMap tmX,    // 128 rows x 2 atoms
                     const __grid_constant__ CUtensorMap tmH,    // 128 rows x 2 atoms
+                    const __grid_constant__ CUtensorMap tmXs,   // kPBShort rows x 2 atoms
+                    const __grid_constant__ CUtensorMap tmHs,   // kPBShort rows x 2 atoms
                     const PairParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -278,6 +286,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         ptx::prefetch_tensormap(&tmW2);
         ptx::prefetch_tensormap(&tmX);
         ptx::prefetch_tensormap(&tmH);
+        ptx::prefetch_tensormap(&tmXs);
+        ptx::prefetch_tensormap(&tmHs);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(tmem_slot, kPTmemCols);
@@ -390,10 +400,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const PUnit w = decode_punit(static_cast<int>(u), u_up, s_off, s_pu, s_pd, s_tb, E);
                 const int ksteps = w.up ? KSU : KSD;
                 const int half = w.n >> 1;               // B rows this CTA holds
-                const uint32_t tx = 2u * kPStage;
+                const bool shrt = half <= kPBShort;
+                const uint32_t tx =
+                    2u * kPAtoms * (kPATile + (shrt ? kPBShortTile : kPBTile));
                 const int arow = w.up ? w.e * p.d_ff + w.blk * 128 + static_cast<int>(cta) * 64
                                       : w.e * p.d + w.blk * 256 + static_cast<int>(cta) * 128;
-                const CUtensorMap *tb = w.up ? &tmX : &tmH;
+                const CUtensorMap *tb = w.up ? (shrt ? &tmXs : &tmX) : (shrt ? &tmHs : &tmH);
                 const int brow = w.r0 + static_cast<int>(cta) * half;
                 for (int ks = 0; ks < ksteps; ++ks) {
                     if (!wait_cl(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
@@ -457,6 +469,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 if (u >= static_cast<uint32_t>(total)) break;
                 const PUnit w = decode_punit(static_cast<int>(u), u_up, s_off, s_pu, s_pd, s_tb, E);
                 const uint32_t idesc = ptx::idesc_bf16_f32(256, w.n);
+                // B atoms as the producer copied them: kPBShort or 128 rows.
+                const uint32_t bstride = (w.n >> 1) <= kPBShort ? kPBShortTile : kPBTile;
                 const int buf = static_cast<int>(i & 1u);
                 const uint32_t use = i >> 1;
                 if (!wait_cl(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.err, kErrTimeoutEpi))
@@ -478,7 +492,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         for (int kk = 0; kk < 4; ++kk)
                             ptx::tc_mma_bf16_pair(
                                 dacc, ptx::sw128_kmajor_desc(sa + a * kPATile + kk * 32),
-                                ptx::sw128_kmajor_desc(sb + a * kPBTile + kk * 32), idesc,
+                                ptx::sw128_kmajor_desc(sb + a * bstride + kk * 32), idesc,
                                 (ks | a | kk) ? 1u : 0u);
                     ptx::tc_commit_pair(&empty[stage], 0x3);
                     if (++stage == static_cast<uint32_t>(kPStages)) {
@@ -663,13 +677,15 @@ bool ffn_pair_eligible(int S, int E_seg, int ksplit)
 cudaError_t launch_ffn_pair(const FfnLaunch &a, uint32_t *sched, cudaStream_t s)
 {
     const int E = a.offsets ? a.E : 1;
-    CUtensorMap tW1, tW3, tW2, tX, tH;
+    CUtensorMap tW1, tW3, tW2, tX, tH, tXs, tHs;
     cudaError_t e = make_tmap_bf16(&tW1, a.W1, static_cast<uint64_t>(E) * a.d_ff, a.d, 64);
     if (e == cudaSuccess) e = make_tmap_bf16(&tW3, a.W3, static_cast<uint64_t>(E) * a.d_ff, a.d, 64);
     if (e == cudaSuccess)
         e = make_tmap_bf16_atoms(&tW2, a.W2, static_cast<uint64_t>(E) * a.d, a.d_ff, 128, 2);
     if (e == cudaSuccess) e = make_tmap_bf16_atoms(&tX, a.x, a.S, a.d, 128, 2);
     if (e == cudaSuccess) e = make_tmap_bf16_atoms(&tH, a.H, a.S, a.d_ff, 128, 2);
+    if (e == cudaSuccess) e = make_tmap_bf16_atoms(&tXs, a.x, a.S, a.d, kPBShort, 2);
+    if (e == cudaSuccess) e = make_tmap_bf16_atoms(&tHs, a.H, a.S, a.d_ff, kPBShort, 2);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kPSmem));
@@ -714,7 +730,7 @@ cudaError_t launch_ffn_pair(const FfnLaunch &a, uint32_t *sched, cudaStream_t s)
     if (grid < 2) grid = 2;
     cfg.gridDim = dim3(static_cast<unsigned>(grid & ~1));
     cfg.numAttrs = a.pdl ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, ffn_pair_kernel, tW1, tW3, tW2, tX, tH, p);
+    return cudaLaunchKernelEx(&cfg, ffn_pair_kernel, tW1, tW3, tW2, tX, tH, tXs, tHs, p);
 }
 
 }  // namespace moe

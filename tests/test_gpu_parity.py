@@ -483,3 +483,23 @@ def test_forward_fp8_mixtral_decode(T):
     idx, _, counts = gpu_route(wl, inp)
     tok = sample_tokens(T, 8, idx)
     _fp8_check(wl, inp, tokens=tok)
+
+
+@pytest.mark.parametrize("T", [8, 1000])
+def test_forward_fp8_every_code(T):
+    # Every finite e4m3 code (both zeros, the subnormals, +-448) in every
+    # weight row, rotated from row to row, through both operand paths of the
+    # FP8 expert kernel: widened rows in tensor memory (token tiles of up to
+    # 64 rows, T = 8) and in shared memory (128-row tiles, T = 1000).
+    wl = Workload(f"fp8_every_code_T{T}", T, 512, 4, 256, 2)
+    inp = synth.make_fp8_experts(wl, seed=11, device="cpu")
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    for name in ("q1", "q3", "q2"):
+        q = inp[name].numpy().copy()
+        for e in range(q.shape[0]):
+            for r in range(q.shape[1]):
+                q[e, r] = np.resize(np.roll(codes, 7 * r + 13 * e), q.shape[2])
+        inp[name] = torch.from_numpy(q)
+    assert all(len(np.unique(inp[n].numpy())) == 254 for n in ("q1", "q3", "q2"))
+    inp = {k: (None if v is None else v.to(DEV)) for k, v in inp.items()}
+    _fp8_check(wl, inp)
