@@ -170,7 +170,12 @@ MOE_API moe_status moe_combine(int T, int d, int k, const float *y_perm, const i
  * down units add w[t,j] * y into out[t], which the dispatch zeroed first.
  * At most two terms reach an element and two terms added onto zero give the
  * same sum in either order, so out is still the same from run to run (it
- * may differ in the last bit from moe_combine's fused multiply-add). */
+ * may differ in the last bit from moe_combine's fused multiply-add).  Other
+ * layers on that kernel (k > 2, or a shared expert) keep its per-slot rows,
+ * and the shared expert's rows, as bf16 in the workspace for the combine:
+ * each row is rounded once, as the hidden activations H are, which is where
+ * the result can differ from the composition of the separate calls (whose
+ * y_perm is fp32). */
 MOE_API moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
                        const moe_bf16 *Wg, const moe_bf16 *W1, const moe_bf16 *W3,
                        const moe_bf16 *W2, float *out, void *ws, size_t ws_bytes,

@@ -366,10 +366,11 @@ static moe_status ffn_impl(int S, int d, int E, int d_ff, int max_rows, const mo
                            const moe_bf16 *W2, moe_bf16 *H, float *y, uint32_t *h_ready,
                            uint32_t *sched, uint32_t *err, cudaStream_t s, bool pdl, int ksplit,
                            int act = 0, float *out = nullptr, const int32_t *slot_of_row = nullptr,
-                           const float *gate_w = nullptr, int k = 1)
+                           const float *gate_w = nullptr, int k = 1, bool y_bf16 = false)
 {
     FfnLaunch f{};
     f.act = act;
+    f.y_bf16 = y_bf16;
     f.out = out;
     f.slot_of_row = slot_of_row;
     f.gate_w = gate_w;
@@ -518,8 +519,14 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     // themselves: at most two terms reach each element, and two terms added
     // onto zero give one result in either order.  No Y round trip and no
     // combine launch then.
-    const bool fused_out =
-        !narrow && k <= 2 && d_ff_shared == 0 && ffn_pair_eligible(S, E, ksplit);
+    const bool pair = !narrow && ffn_pair_eligible(S, E, ksplit);
+    const bool fused_out = pair && k <= 2 && d_ff_shared == 0;
+    // The CTA-pair kernel's rows are complete sums (it never splits K); they
+    // go to the combine as bf16, which halves the bytes of the per-slot
+    // round trip (each row rounded once, as H is).  K-split partials stay
+    // fp32.
+    const bool y_bf16 = pair && !fused_out;
+    const bool ys_bf16 = d_ff_shared > 0 && ffn_pair_eligible(T, 1, 1);
     int32_t *slotrow = reinterpret_cast<int32_t *>(wsb + L.slotrow);
     if ((st = mark(events, 0, s)) != MOE_OK) return st;
     st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
@@ -580,7 +587,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         st = ffn_impl(S, d, E, d_ff, T, xperm, offsets, W1, W3, W2, H, Y,
                       reinterpret_cast<uint32_t *>(wsb + L.hready),
                       reinterpret_cast<uint32_t *>(wsb + 16), err, s, pdl, ksplit, act,
-                      fused_out ? out : nullptr, slotrow, w, k);
+                      fused_out ? out : nullptr, slotrow, w, k, y_bf16);
     }
     if (st != MOE_OK) return st;
 
@@ -591,7 +598,8 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
         st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys,
                       reinterpret_cast<uint32_t *>(wsb + L.hready_s),
-                      reinterpret_cast<uint32_t *>(wsb + 20), err, s, false, 1, act);
+                      reinterpret_cast<uint32_t *>(wsb + 20), err, s, false, 1, act, nullptr,
+                      nullptr, nullptr, 1, ys_bf16);
         if (st != MOE_OK) return st;
         shared_y = Ys;
     }
@@ -615,6 +623,8 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     cb.w = w;
     cb.shared_y = shared_y;
     cb.out = out;
+    cb.y_bf16 = y_bf16;
+    cb.shared_bf16 = ys_bf16;
     cb.pdl = false;  // after a persistent kernel an early launch only takes SM slots
     st = from_cuda(launch_combine(cb, s));
     if (st != MOE_OK) return st;

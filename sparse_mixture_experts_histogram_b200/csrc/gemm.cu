@@ -553,7 +553,7 @@ cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s)
 {
     if (a.sched != nullptr && ffn_pair_eligible(a.S, a.offsets ? a.E : 1, a.ksplit))
         return launch_ffn_pair(a, a.sched, s);
-    if (a.out != nullptr) return cudaErrorInvalidValue;  // weighted output: pair kernel only
+    if (a.out != nullptr || a.y_bf16) return cudaErrorInvalidValue;  // pair kernel only
     switch (ffn_token_tile(a.S, a.offsets ? a.E : 1)) {
     case 32: return launch_ffn_cfg<32, 6>(a, s);
     case 64: return launch_ffn_cfg<64, 5>(a, s);

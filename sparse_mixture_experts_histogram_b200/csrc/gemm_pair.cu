@@ -108,6 +108,7 @@ struct PairParams {
     const int32_t *slot_of_row;
     const float *gate_w;
     int k;
+    int y_bf16;              // Y as bf16 rows (otherwise fp32)
 };
 
 struct PUnit {
@@ -608,6 +609,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
                                 atomicAdd(p.out + static_cast<size_t>(slj / p.k) * p.d + o,
                                           gwj * __uint_as_float(r[j]));
                         }
+                    } else if (has && p.y_bf16) {
+                        __nv_bfloat16 *yc = reinterpret_cast<__nv_bfloat16 *>(p.Y) +
+                                            static_cast<size_t>(w.r0 + c0) * p.d + o;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c0 + j < w.valid)
+                                yc[static_cast<size_t>(j) * p.d] = __float2bfloat16_rn(__uint_as_float(r[j]));
                     } else if (has) {
                         float *yc = p.Y + static_cast<size_t>(w.r0 + c0) * p.d + o;
 #pragma unroll
@@ -707,6 +715,7 @@ cudaError_t launch_ffn_pair(const FfnLaunch &a, uint32_t *sched, cudaStream_t s)
     p.slot_of_row = a.slot_of_row;
     p.gate_w = a.gate_w;
     p.k = a.k < 1 ? 1 : a.k;
+    p.y_bf16 = a.y_bf16 ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kPThreads);

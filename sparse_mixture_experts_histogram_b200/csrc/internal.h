@@ -96,6 +96,9 @@ struct FfnLaunch {
     const int32_t *slot_of_row;
     const float *gate_w;
     int k;
+    // CTA-pair kernel only: Y holds bf16 rows [S, d] instead of fp32 (its
+    // rows are complete sums: that kernel never splits K).
+    bool y_bf16;
 };
 
 struct CombineLaunch {
@@ -110,6 +113,8 @@ struct CombineLaunch {
     const float *shared_y;
     float *out;
     bool pdl;                 // launched right after another kernel of this library
+    bool y_bf16;              // y holds bf16 rows [T*k, d] (ksplit 1), not fp32
+    bool shared_bf16;         // shared_y holds bf16 rows [T, d]
 };
 
 cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s);
