@@ -185,7 +185,14 @@ MOE_API moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_b
  * shared expert of hidden width d_ff_shared (0 = none; Ws1/Ws3/Ws2 may then
  * be NULL), whose output is added to every token with weight 1
  * (theaiera.top sec. 10.5).  The workspace must hold
- * moe_workspace_size_ex(..., d_ff_shared) bytes. */
+ * moe_workspace_size_ex(..., d_ff_shared) bytes.  The shared expert needs
+ * no routing, so it runs on a second stream of the library's own (one per
+ * device, created on first use, non-blocking): the call records an event on
+ * `stream`, the second stream waits for it, and `stream` waits for the
+ * second stream's event before the combine.  Everything stays ordered with
+ * `stream`, and the call can be captured into a CUDA graph (the fork and
+ * join are captured with it).  The second stream is not valid after
+ * cudaDeviceReset in the same process. */
 MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
                           const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
                           const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,

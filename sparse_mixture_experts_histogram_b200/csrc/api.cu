@@ -454,6 +454,42 @@ static moe_status mark(void *const *events, int i, cudaStream_t s)
     return from_cuda(cudaEventRecord(ev, s));
 }
 
+// A second stream per device for the shared expert, created on first use
+// (non-blocking, so it never orders against the legacy default stream).  A
+// call forks onto it with an event recorded on the caller's stream and joins
+// back with another, so the work stays ordered with the caller's stream and
+// the call can still be captured into a CUDA graph.
+std::mutex g_side_mu;
+cudaStream_t g_side[64];
+
+cudaStream_t side_stream()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    if (g_side[dev] == nullptr) {
+        cudaStream_t st = nullptr;
+        if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        g_side[dev] = st;
+    }
+    return g_side[dev];
+}
+
+// The shared expert's rows come from the CTA-pair kernel (complete sums, so
+// bf16 like the routed ones) whenever its single segment is large enough.
+static bool ys_bf16_for(int T) { return ffn_pair_eligible(T, 1, 1); }
+
+static moe_status shared_impl(int T, int d, int d_ffs, const moe_bf16 *x, const moe_bf16 *Ws1,
+                              const moe_bf16 *Ws3, const moe_bf16 *Ws2, uint8_t *wsb,
+                              const Layout &L, uint32_t *err, cudaStream_t s, int act, bool ys_bf16)
+{
+    return ffn_impl(T, d, 1, d_ffs, T, x, nullptr, Ws1, Ws3, Ws2,
+                    reinterpret_cast<moe_bf16 *>(wsb + L.Hs), reinterpret_cast<float *>(wsb + L.Ys),
+                    reinterpret_cast<uint32_t *>(wsb + L.hready_s),
+                    reinterpret_cast<uint32_t *>(wsb + 20), err, s, false, 1, act, nullptr, nullptr,
+                    nullptr, 1, ys_bf16);
+}
+
 static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
                                const moe_bf16 *Wg, const float *router_bias, const moe_bf16 *W1,
                                const moe_bf16 *W3, const moe_bf16 *W2, int d_ff_shared,
@@ -526,13 +562,54 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     // round trip (each row rounded once, as H is).  K-split partials stay
     // fp32.
     const bool y_bf16 = pair && !fused_out;
-    const bool ys_bf16 = d_ff_shared > 0 && ffn_pair_eligible(T, 1, 1);
+    const bool ys_bf16 = d_ff_shared > 0 && ys_bf16_for(T);
     int32_t *slotrow = reinterpret_cast<int32_t *>(wsb + L.slotrow);
     if ((st = mark(events, 0, s)) != MOE_OK) return st;
     st = route_impl(T, d, E, k, x, Wg, router_bias, idx, w,
                     reinterpret_cast<int32_t *>(wsb + L.counts), offsets, wsb, L, s, narrow, wmode,
                     cap);
     if (st != MOE_OK) return st;
+
+    // The shared expert needs neither the routing nor the dispatch: with a
+    // side stream it runs next to the scatter (which takes no shared memory,
+    // so its blocks fit beside the expert kernel's) and the routed experts.
+    // The traced form keeps it in line, between its events.
+    const float *shared_y = nullptr;
+    cudaStream_t s2 = nullptr;
+    // Joins the side stream back into the caller's stream when the call
+    // leaves this scope, on an early error return too.
+    struct Join {
+        cudaStream_t s;
+        cudaEvent_t ev = nullptr;
+        moe_status now()
+        {
+            if (ev == nullptr) return MOE_OK;
+            const cudaError_t e = cudaStreamWaitEvent(s, ev, 0);
+            cudaEventDestroy(ev);
+            ev = nullptr;
+            return from_cuda(e);
+        }
+        ~Join() { now(); }
+    } join{s};
+    if (d_ff_shared > 0 && events == nullptr && (s2 = side_stream()) != nullptr) {
+        cudaEvent_t ev_fork = nullptr;
+        if ((st = from_cuda(cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming))) != MOE_OK)
+            return st;
+        st = from_cuda(cudaEventRecord(ev_fork, s));
+        if (st == MOE_OK) st = from_cuda(cudaStreamWaitEvent(s2, ev_fork, 0));
+        cudaEventDestroy(ev_fork);
+        if (st != MOE_OK) return st;
+        st = shared_impl(T, d, d_ff_shared, x, Ws1, Ws3, Ws2, wsb, L, err, s2, act, ys_bf16_for(T));
+        cudaEvent_t ev = nullptr;
+        if (st == MOE_OK) st = from_cuda(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+        if (st == MOE_OK) {
+            st = from_cuda(cudaEventRecord(ev, s2));
+            if (st == MOE_OK) join.ev = ev;
+            else cudaEventDestroy(ev);
+        }
+        if (st != MOE_OK) return st;
+        shared_y = reinterpret_cast<const float *>(wsb + L.Ys);
+    }
 
     if ((st = mark(events, 1, s)) != MOE_OK) return st;
     if (!narrow) {
@@ -591,18 +668,13 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     }
     if (st != MOE_OK) return st;
 
-    const float *shared_y = nullptr;
     if ((st = mark(events, 3, s)) != MOE_OK) return st;
-    if (d_ff_shared > 0) {
-        moe_bf16 *Hs = reinterpret_cast<moe_bf16 *>(wsb + L.Hs);
-        float *Ys = reinterpret_cast<float *>(wsb + L.Ys);
-        st = ffn_impl(T, d, 1, d_ff_shared, T, x, nullptr, Ws1, Ws3, Ws2, Hs, Ys,
-                      reinterpret_cast<uint32_t *>(wsb + L.hready_s),
-                      reinterpret_cast<uint32_t *>(wsb + 20), err, s, false, 1, act, nullptr,
-                      nullptr, nullptr, 1, ys_bf16);
+    if (d_ff_shared > 0 && s2 == nullptr) {
+        st = shared_impl(T, d, d_ff_shared, x, Ws1, Ws3, Ws2, wsb, L, err, s, act, ys_bf16);
         if (st != MOE_OK) return st;
-        shared_y = Ys;
+        shared_y = reinterpret_cast<const float *>(wsb + L.Ys);
     }
+    if ((st = join.now()) != MOE_OK) return st;
     if ((st = mark(events, 4, s)) != MOE_OK) return st;
     if (fused_out) return mark(events, 5, s);
 

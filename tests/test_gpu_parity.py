@@ -290,6 +290,43 @@ def test_forward_is_deterministic_and_graph_capturable():
     assert torch.equal(out, a)
 
 
+SIDE_STREAM_CASES = [Workload("shared_side_narrow", 300, 256, 32, 256, 4, d_ff_shared=384),
+                     Workload("shared_side_wide", 300, 1152, 16, 256, 4, d_ff_shared=256)]
+
+
+@pytest.mark.parametrize("wl", SIDE_STREAM_CASES, ids=lambda w: w.name)
+def test_forward_shared_expert_side_stream_graph(wl):
+    # The shared expert runs on the library's side stream, forked after the
+    # routing and joined before the combine: the output matches the oracle,
+    # repeats from call to call, and a CUDA graph captured on another stream
+    # (the fork and join captured with it) replays the same bytes.
+    inp = _inputs(wl)
+    check_forward(wl, inp)
+    ws = workspace(wl)
+    a = gpu_forward(wl, inp, ws).clone()
+    out = torch.empty_like(a)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def call():
+        moe.moe_forward_ex(wl.T, wl.d, wl.E, wl.d_ff, wl.k, inp["x"], inp["Wg"], inp["bias"],
+                           inp["W1"], inp["W3"], inp["W2"], wl.d_ff_shared, inp["Ws1"], inp["Ws3"],
+                           inp["Ws2"], out, ws, stream=s)
+
+    with torch.cuda.stream(s):
+        call()
+    torch.cuda.synchronize()
+    assert torch.equal(out, a)
+    g = torch.cuda.CUDAGraph()
+    out.zero_()
+    with torch.cuda.graph(g, stream=s):
+        call()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, a)
+    assert moe.moe_get_device_error(ws)[0] == 0
+
+
 @pytest.mark.parametrize("wl", [synth.sweep()[-1], Workload("E64_k4_T1000", 1000, 384, 64, 256, 4),
                                 Workload("wide_pair_T1100_d1152_E8_k2", 1100, 1152, 8, 512, 2)],
                          ids=lambda w: w.name)
