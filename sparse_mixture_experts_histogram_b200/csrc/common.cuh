@@ -57,6 +57,28 @@ __device__ __forceinline__ bool bounded_wait_warp(uint64_t *bar, uint32_t parity
     return all;
 }
 
+// Readiness of up to 32 consecutive H blocks, counters ctr[0..n): bit i set
+// when ctr[i] >= target.  Relaxed loads, all issued before any result is
+// used, then one acquire fence for all of them (an acquire load per counter
+// would order each load after the previous one): a down unit whose blocks
+// were published long ago, the common case, pays one memory round trip for
+// the window instead of one per K step.  Blocks found not ready are then
+// waited for one by one.
+__device__ __forceinline__ uint32_t ready_window(const uint32_t *ctr, int n, uint32_t target)
+{
+    uint32_t v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        v[i] = target;
+        if (i < n) asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v[i]) : "l"(ctr + i) : "memory");
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m |= (v[i] >= target ? 1u : 0u) << i;
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    return m;
+}
+
 // Shared memory of one routing tile's histogram / rank computation.
 struct DispatchSmem {
     int32_t sel[kTileTokens][kMaxK];   // expert of (row, slot); -1 = no token

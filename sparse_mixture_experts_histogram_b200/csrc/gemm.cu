@@ -314,6 +314,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                 const int arow0 = w.up ? w.e * p.d_ff + w.blk * 128 : w.e * p.d + w.blk * 256;
                 const int arow1 = w.up ? arow0 : arow0 + 128;
                 int ready_blk = -1;
+                int win = -1;        // first H block of the readiness window
+                uint32_t wmask = 0;  // blocks of the window found ready
                 for (int ks = w.k_beg; ks < w.k_end; ++ks) {
                     if (!bounded_wait(&empty[stage], phase ^ 1u, abort_flag, p.err,
                                       kErrTimeoutMma)) {
@@ -330,7 +332,14 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                         // These 64 columns of H belong to 128-column block ks/2:
                         // wait until its up unit has stored and published it.
                         ready_blk = ks >> 1;
-                        if (!wait_counter(&p.h_ready[w.tile * MBU + ready_blk], ready_target,
+                        if (win < 0 || ready_blk >= win + 32) {
+                            win = ready_blk;
+                            const int nb = ((w.k_end + 1) >> 1) - ready_blk;
+                            wmask = ready_window(&p.h_ready[w.tile * MBU + ready_blk],
+                                                 nb < 32 ? nb : 32, ready_target);
+                        }
+                        if (!((wmask >> (ready_blk - win)) & 1u) &&
+                            !wait_counter(&p.h_ready[w.tile * MBU + ready_blk], ready_target,
                                           abort_flag, p.err)) {
                             stop = true;
                             break;
