@@ -85,6 +85,7 @@ struct F8Cfg {
     static constexpr size_t kSmem =
         kF8Fixed + static_cast<size_t>(ST) * kInStage + OPS * kOpStage;
     static_assert(OPS >= 2 && OPS <= kF8MaxOps, "operand ring");
+    static_assert(!kTA || OPS % 2 == 0, "operand stages taken in pairs");
     static_assert(!kTA || kOpCol0 + 64u * OPS <= kTmemCols, "tensor-memory operands");
     static_assert(ST >= 2, "pipeline depth");
     static_assert(kTmemCols >= 32 && kTmemCols <= 512, "tensor memory");
@@ -428,19 +429,27 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                         stop = true;
                         break;
                     }
-                    for (int hf = 0; hf < 2; ++hf) {
+                    if constexpr (C::kTA) {
+                        // Both halves' operands (stages ost, ost + 1: OPS is
+                        // even, so a pair never wraps), then all 16 MMAs of
+                        // the step.  Each wait stalls the MMA issue for a few
+                        // hundred cycles, which MMAs this short (N <= 64) do
+                        // not hide: one wait per 16 MMAs instead of per 8.
                         if (!bounded_wait(&op_full[ost], ophase, abort_flag, p.err,
+                                          kErrTimeoutTma) ||
+                            !bounded_wait(&op_full[ost + 1], ophase, abort_flag, p.err,
                                           kErrTimeoutTma)) {
                             stop = true;
                             break;
                         }
                         ptx::tc_fence_after();
-                        const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage +
-                                                           2 * kRawTile + hf * BN * 128);
-                        if constexpr (C::kTA) {
-                            // A: tile t of the stage at columns
-                            // kOpCol0 + 64 ost + 32 t, 16 K elements per 8 columns.
-                            const uint32_t ta = tmem + C::kOpCol0 + 64u * ost;
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage +
+                                                               2 * kRawTile + hf * BN * 128);
+                            // A: tile t of stage ost + hf at columns
+                            // kOpCol0 + 64 (ost + hf) + 32 t, 16 K elements per 8 columns.
+                            const uint32_t ta = tmem + C::kOpCol0 + 64u * (ost + hf);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
@@ -448,7 +457,27 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                                 ptx::tc_mma_f16_ts(d0, ta + 8u * kk, bdesc, idesc, acc);
                                 ptx::tc_mma_f16_ts(d0 + BN, ta + 32u + 8u * kk, bdesc, idesc, acc);
                             }
-                        } else {
+                        }
+                        ptx::tc_commit(&op_empty[ost]);
+                        ptx::tc_commit(&op_empty[ost + 1]);
+                        ost += 2;
+                        if (ost == static_cast<uint32_t>(OPS)) {
+                            ost = 0;
+                            ophase ^= 1u;
+                        }
+                    } else {
+                        // Shared-memory operands, two stages: one 64-column
+                        // half at a time, so the converters refill the first
+                        // stage while the MMAs read the second.
+                        for (int hf = 0; hf < 2; ++hf) {
+                            if (!bounded_wait(&op_full[ost], ophase, abort_flag, p.err,
+                                              kErrTimeoutTma)) {
+                                stop = true;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                            const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage +
+                                                               2 * kRawTile + hf * BN * 128);
                             const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
@@ -460,11 +489,11 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                                                  ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
                                                  bdesc, idesc, acc);
                             }
-                        }
-                        ptx::tc_commit(&op_empty[ost]);
-                        if (++ost == static_cast<uint32_t>(OPS)) {
-                            ost = 0;
-                            ophase ^= 1u;
+                            ptx::tc_commit(&op_empty[ost]);
+                            if (++ost == static_cast<uint32_t>(OPS)) {
+                                ost = 0;
+                                ophase ^= 1u;
+                            }
                         }
                     }
                     if (stop) break;
