@@ -11,13 +11,13 @@
 //     FP8 where the layer streams its weights from HBM (decode);
 //   * eight converter warps widen the tiles to fp16 by bit moves (exact: every
 //     e4m3 value times 2^-8 is an fp16 value; the 2^8 goes into the row
-//     scale), then release the raw stage and mark the operand stage full.  With token tiles of up to 64 rows (decode) the widened weights go
-//     to tensor memory, one weight row per lane, and the MMA reads its A
-//     operand from there: the shared-memory traffic per weight code is then
-//     the TMA write and one converter read, which leaves the converters and
-//     the memory system, not shared-memory bandwidth, as the limit.  With
-//     128-row token tiles the accumulators fill tensor memory, and the
-//     operands go to shared memory in the 128-byte-swizzled K-major layout;
+//     scale), then release the raw stage and mark the operand stage full.
+//     With token tiles of up to 64 rows (decode) the widened weights go to
+//     tensor memory, one weight row per lane, and the MMA reads its A operand
+//     from there: the shared-memory traffic per weight code is then the TMA
+//     write and one converter read.  With 128-row token tiles the
+//     accumulators fill tensor memory, and the operands go to shared memory
+//     in the 128-byte-swizzled K-major layout;
 //   * the MMA is kind::f16 with fp16 A and B (the token rows x_perm and the
 //     hidden activations H are fp16 in this path) and fp32 accumulators;
 //   * the epilogue multiplies each accumulator row by its weight row's scale
@@ -25,10 +25,14 @@
 //
 // Pipelines: a deep ring of input stages (the two e4m3 weight tiles of a K
 // step, the step's fp16 token rows) keeps enough bytes in flight to stream
-// HBM; the converters fill a ring of two fp16 operand stages from it.  An
+// HBM; the converters fill a ring of operand stages (64-column halves of a K
+// step: six or four in tensor memory, two in shared memory) from it.  An
 // input stage is free once the converters have read its tiles and the MMAs
-// its token rows.
-//
+// its token rows.  With tensor-memory operands the MMA thread waits for both
+// halves of a step and issues its 16 MMAs together: each wait stalls the
+// MMA issue for a few hundred cycles, which these short (N <= 64) MMAs do
+// not hide.
+
 // Roles: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warps 6..13 converters
 // (one weight row of one tile per thread).
 //
