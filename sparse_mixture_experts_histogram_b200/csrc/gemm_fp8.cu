@@ -33,8 +33,10 @@
 // MMA issue for a few hundred cycles, which these short (N <= 64) MMAs do
 // not hide.
 
-// Roles: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue, warps 6..13 converters
-// (one weight row of one tile per thread).
+// Roles: warp 0 TMA, warps 1 and 14 MMA (one weight tile each: a thread
+// issuing 128 x N x 16 MMAs with N <= 64 is itself the limit, at about 50
+// cycles per MMA, and two issuing warps double the rate), warps 2..5
+// epilogue, warps 6..13 converters (one weight row of one tile per thread).
 //
 // Method: the SwiGLU expert w2(silu(w1 x) * w3 x) ("Mistral 8x7B SMoE
 // architecture" (jsqmd.com) sec. 3.1 FeedForward) with quantised expert
@@ -54,7 +56,8 @@ namespace moe {
 
 namespace {
 
-constexpr int kF8Threads = 448;   // warp 0 TMA, 1 MMA, 2..5 epilogue, 6..13 converters
+constexpr int kF8Threads = 480;   // warp 0 TMA, 1 and 14 MMA, 2..5 epilogue, 6..13 converters
+constexpr int kF8MmaWarp1 = 14;   // issues the second weight tile's MMAs
 constexpr int kF8ConvWarps = 8;
 constexpr int kF8MaxStages = 8;
 constexpr int kF8MaxOps = 6;     // operand ring depth, tensor-memory operands
@@ -275,17 +278,17 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             ptx::mbar_init(&in_full[s], 1);
-            ptx::mbar_init(&in_empty[s], kF8ConvWarps + 1);  // converters (e4m3 read) + MMA (rows read)
+            ptx::mbar_init(&in_empty[s], kF8ConvWarps + 2);  // converters (e4m3 read) + 2 MMA warps (rows read)
         }
         for (int s = 0; s < OPS; ++s) {
             ptx::mbar_init(&op_full[s], kF8ConvWarps);
-            ptx::mbar_init(&op_empty[s], 1);
+            ptx::mbar_init(&op_empty[s], 2);
         }
         for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tfull[b], 2);
             ptx::mbar_init(&tempty[b], 4);
         }
-        ptx::mbar_init(drain, 1);
+        ptx::mbar_init(drain, 2);
         *abort_flag = 0u;
         ptx::fence_barrier_init();
     }
@@ -408,8 +411,13 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             for (int s = 0; s < ST; ++s)
                 if (issued & (1u << s)) f8_drain_wait(&in_full[s], last_parity[s]);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kF8MmaWarp1) {
         if (lane == 0) {
+            // This warp's weight tile: 0 (W1 rows, or W2 rows 0..127 of the
+            // down block) into accumulator d0, 1 (W3, or W2 rows 128..255)
+            // into d0 + BN.  Both warps wait for the same stages, and every
+            // barrier they release counts one commit from each.
+            const int t = warp == 1 ? 0 : 1;
             uint32_t stage = 0, phase = 0;    // input ring
             uint32_t ost = 0, ophase = 0;     // operand ring
             int i = 0;
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                                   kErrTimeoutEpi))
                     break;
                 ptx::tc_fence_after();
-                const uint32_t d0 = tmem + static_cast<uint32_t>(buf * C::kAccCols);
+                const uint32_t d0 = tmem + static_cast<uint32_t>(buf * C::kAccCols + t * BN);
                 for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
                     // The token rows came with the input stage; the weights
                     // were converted, one 64-column half at a time, into the
@@ -435,10 +443,10 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                     }
                     if constexpr (C::kTA) {
                         // Both halves' operands (stages ost, ost + 1: OPS is
-                        // even, so a pair never wraps), then all 16 MMAs of
-                        // the step.  Each wait stalls the MMA issue for a few
-                        // hundred cycles, which MMAs this short (N <= 64) do
-                        // not hide: one wait per 16 MMAs instead of per 8.
+                        // even, so a pair never wraps), then this tile's 8
+                        // MMAs of the step.  Each wait stalls the MMA issue
+                        // for a few hundred cycles, which MMAs this short
+                        // (N <= 64) do not hide: one wait per step.
                         if (!bounded_wait(&op_full[ost], ophase, abort_flag, p.err,
                                           kErrTimeoutTma) ||
                             !bounded_wait(&op_full[ost + 1], ophase, abort_flag, p.err,
@@ -453,13 +461,12 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                                                                2 * kRawTile + hf * BN * 128);
                             // A: tile t of stage ost + hf at columns
                             // kOpCol0 + 64 (ost + hf) + 32 t, 16 K elements per 8 columns.
-                            const uint32_t ta = tmem + C::kOpCol0 + 64u * (ost + hf);
+                            const uint32_t ta = tmem + C::kOpCol0 + 64u * (ost + hf) + 32u * t;
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
                                 const uint32_t acc = ((ks - w.k_beg) | hf | kk) ? 1u : 0u;
                                 ptx::tc_mma_f16_ts(d0, ta + 8u * kk, bdesc, idesc, acc);
-                                ptx::tc_mma_f16_ts(d0 + BN, ta + 32u + 8u * kk, bdesc, idesc, acc);
                             }
                         }
                         ptx::tc_commit(&op_empty[ost]);
@@ -482,16 +489,13 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                             ptx::tc_fence_after();
                             const uint32_t sb = ptx::smem_addr(ins + stage * C::kInStage +
                                                                2 * kRawTile + hf * BN * 128);
-                            const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage);
+                            const uint32_t sa = ptx::smem_addr(ops + ost * C::kOpStage + t * kW16Tile);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 const uint64_t bdesc = ptx::sw128_kmajor_desc(sb + kk * 32);
                                 const uint32_t acc = ((ks - w.k_beg) | hf | kk) ? 1u : 0u;
                                 ptx::tc_mma_bf16(d0, ptx::sw128_kmajor_desc(sa + kk * 32), bdesc,
                                                  idesc, acc);
-                                ptx::tc_mma_bf16(d0 + BN,
-                                                 ptx::sw128_kmajor_desc(sa + kW16Tile + kk * 32),
-                                                 bdesc, idesc, acc);
                             }
                             ptx::tc_commit(&op_empty[ost]);
                             if (++ost == static_cast<uint32_t>(OPS)) {
@@ -512,7 +516,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
             ptx::tc_commit(drain);
             f8_drain_wait(drain, 0u);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 6 && warp < 6 + kF8ConvWarps) {
         // Converters: warp w widens rows 32 (w % 4) .. 32 (w % 4) + 31 of
         // weight tile (w - 6) / 4 of a step, one row per thread -- the rows
         // of the tensor-memory lanes the warp may access.
@@ -641,7 +645,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                 }
             }
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // Epilogue: warps 2..5, one TMEM lane quarter each.
         const int q = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
