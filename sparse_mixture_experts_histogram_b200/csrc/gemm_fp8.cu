@@ -528,57 +528,58 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         uint32_t ost = 0, ophase = 0;     // operand ring
         bool stop = false;
         if constexpr (C::kTA) {
+            // Both 64-column halves of a step at once, as the MMA warps take
+            // them: one wait for free stages, one store wait, one arrival
+            // per stage.
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
                 const F8Unit w = decode_f8<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
                 for (int ks = w.k_beg; ks < w.k_end && !stop; ++ks) {
                     const bool ok =
-                        bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma);
+                        bounded_wait(&in_full[stage], phase, abort_flag, p.err, kErrTimeoutTma) &&
+                        bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag, p.err, kErrTimeoutMma) &&
+                        bounded_wait(&op_empty[ost + 1], ophase ^ 1u, abort_flag, p.err,
+                                     kErrTimeoutMma);
                     if (!__all_sync(0xffffffffu, ok)) {
                         *abort_flag = 1u;
                         stop = true;
                         break;
                     }
+                    ptx::tc_fence_after();
                     // Raw row r: 128 bytes, 16-byte chunk j stored at chunk
-                    // j ^ (r & 7) (128-byte swizzle).
+                    // j ^ (r & 7) (128-byte swizzle); codes 64hf .. 64hf + 63
+                    // (chunks 4hf .. 4hf + 3) go to the tile's 32 columns of
+                    // stage ost + hf.
                     const uint8_t *src = ins + stage * C::kInStage + t * kRawTile + r * 128;
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const bool oke = bounded_wait(&op_empty[ost], ophase ^ 1u, abort_flag,
-                                                      p.err, kErrTimeoutMma);
-                        if (!__all_sync(0xffffffffu, oke)) {
-                            *abort_flag = 1u;
-                            stop = true;
-                            break;
-                        }
-                        ptx::tc_fence_after();
-                        // Codes 64hf .. 64hf + 63 of the row (chunks 4hf ..
-                        // 4hf + 3) -> the tile's 32 columns of the stage.
-                        uint32_t v32[32];
+                    uint32_t v64[64];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint4 v = *reinterpret_cast<const uint4 *>(
-                                src + (((4 * hf + j) ^ (r & 7)) << 4));
-                            e4m3x4_to_f16x4(v.x, v32[8 * j + 0], v32[8 * j + 1]);
-                            e4m3x4_to_f16x4(v.y, v32[8 * j + 2], v32[8 * j + 3]);
-                            e4m3x4_to_f16x4(v.z, v32[8 * j + 4], v32[8 * j + 5]);
-                            e4m3x4_to_f16x4(v.w, v32[8 * j + 6], v32[8 * j + 7]);
-                        }
-                        ptx::tmem_st16(t_row + 64u * ost,
-                                       *reinterpret_cast<const uint32_t(*)[16]>(&v32[0]));
-                        ptx::tmem_st16(t_row + 64u * ost + 16u,
-                                       *reinterpret_cast<const uint32_t(*)[16]>(&v32[16]));
-                        // The MMA thread reads the operand after the arrival.
-                        ptx::tc_wait_st();
-                        ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&op_full[ost]);
-                        if (++ost == static_cast<uint32_t>(OPS)) {
-                            ost = 0;
-                            ophase ^= 1u;
-                        }
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(src + ((j ^ (r & 7)) << 4));
+                        e4m3x4_to_f16x4(v.x, v64[8 * j + 0], v64[8 * j + 1]);
+                        e4m3x4_to_f16x4(v.y, v64[8 * j + 2], v64[8 * j + 3]);
+                        e4m3x4_to_f16x4(v.z, v64[8 * j + 4], v64[8 * j + 5]);
+                        e4m3x4_to_f16x4(v.w, v64[8 * j + 6], v64[8 * j + 7]);
                     }
-                    if (stop) break;
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        ptx::tmem_st16(t_row + 64u * (ost + hf),
+                                       *reinterpret_cast<const uint32_t(*)[16]>(&v64[32 * hf]));
+                        ptx::tmem_st16(t_row + 64u * (ost + hf) + 16u,
+                                       *reinterpret_cast<const uint32_t(*)[16]>(&v64[32 * hf + 16]));
+                    }
+                    // The MMA warps read the operands after the arrivals.
+                    ptx::tc_wait_st();
+                    ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&in_empty[stage]);
+                    if (lane == 0) {
+                        ptx::mbar_arrive(&op_full[ost]);
+                        ptx::mbar_arrive(&op_full[ost + 1]);
+                        ptx::mbar_arrive(&in_empty[stage]);
+                    }
+                    ost += 2;
+                    if (ost == static_cast<uint32_t>(OPS)) {
+                        ost = 0;
+                        ophase ^= 1u;
+                    }
                     if (++stage == static_cast<uint32_t>(ST)) {
                         stage = 0;
                         phase ^= 1u;
