@@ -43,9 +43,11 @@
  *   finished the work.  Calls sharing a workspace must be ordered on one
  *   stream.
  * Co-residency: the expert kernels run one CTA (or CTA pair) per SM.  The
- *   large-batch kernel hands out its work through a global counter, so it
- *   finishes whatever number of its CTAs is resident at a time.  The
- *   small-batch (decode) kernels assign work to CTAs statically; a CTA that
+ *   large-batch kernel, and the bf16 decode kernel when it has at least
+ *   three work units per CTA, hand out their work through a global counter,
+ *   so they finish whatever number of their CTAs is resident at a time.  The
+ *   decode kernel with fewer units (one or two experts hit), the FP8 kernel
+ *   and moe_expert_ffn_static assign work to CTAs statically; a CTA that
  *   waits on another CTA's results spins (bounded) on the assumption that
  *   all CTAs of the launch are resident, which holds when the layer has the
  *   GPU to itself.  If other work keeps SMs occupied for longer than the

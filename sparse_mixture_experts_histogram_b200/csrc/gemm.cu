@@ -48,8 +48,9 @@ namespace {
 constexpr int kFfnThreads = 192;
 constexpr int kMaxStages = 8;
 constexpr uint32_t kWTile = 128 * 128;  // 128 weight rows x 64 bf16 = 16 KB
-constexpr size_t kFixedSmem = 1024 /* alignment slack */ + (2 * kMaxStages + 5) * 8 + 16 +
-                              4 * (kMaxE + 1) * sizeof(int32_t) + 64;
+constexpr int kSlots = 4;  // unit-number ring (see ffn_kernel)
+constexpr size_t kFixedSmem = 1024 /* alignment slack */ + (2 * kMaxStages + 5 + 2 * kSlots) * 8 +
+                              4 * kSlots + 16 + 4 * (kMaxE + 1) * sizeof(int32_t) + 64;
 constexpr size_t kSmemBudget = 227 * 1024;
 
 template <int BN, int ST>
@@ -80,6 +81,7 @@ struct FfnParams {
     uint32_t *err;
     int stream_weights;     // each weight block feeds one token tile: L2 evict-first
     int act;                // expert activation: 0 silu(g) * b, 1 sigmoid(g) * b
+    uint32_t *sched;        // unit counter, zero before the launch; or nullptr: static order
 };
 
 struct Unit {
@@ -194,7 +196,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     uint64_t *tfull = empty + kMaxStages;  // [2]
     uint64_t *tempty = tfull + 2;          // [2]
     uint64_t *drain = tempty + 2;          // [1]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *sfull = drain + 1;           // [kSlots] unit number posted
+    uint64_t *sempty = sfull + kSlots;     // [kSlots] read by the MMA thread and 4 epilogue warps
+    uint32_t *sched_id = reinterpret_cast<uint32_t *>(sempty + kSlots);  // [kSlots]
+    uint32_t *tmem_slot = sched_id + kSlots;
     volatile uint32_t *abort_flag = tmem_slot + 1;
     int32_t *s_off = reinterpret_cast<int32_t *>(tmem_slot + 4);
     int32_t *s_pu = s_off + (kMaxE + 1);   // up-unit prefix per expert
@@ -219,6 +224,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
             ptx::mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
         }
         ptx::mbar_init(drain, 1);
+        for (int k = 0; k < kSlots; ++k) {
+            ptx::mbar_init(&sfull[k], 1);
+            ptx::mbar_init(&sempty[k], 1 + 4);
+        }
         *abort_flag = 0u;
         ptx::fence_barrier_init();
     }
@@ -305,7 +314,30 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
             const uint64_t pol_w =
                 p.stream_weights ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             bool stop = false;
-            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+            // Unit numbers.  With a counter and at least three units per
+            // CTA, every unit comes from the counter (the next one fetched
+            // while the current one is issued): CTAs that finish early take
+            // more, and a down unit's H blocks come from units with smaller
+            // numbers, taken earlier by CTAs that are running, so its waits
+            // end whatever number of CTAs is resident.  With fewer units per
+            // CTA (one or two experts at small batches) the fixed order
+            // balances the coarse units better (measured): CTA b takes units
+            // b, b + grid, ...  Either way the number is posted to the MMA
+            // thread and the epilogue warps through the slot ring.
+            const bool dyn = p.sched != nullptr && total >= 3 * static_cast<int>(gridDim.x);
+            uint32_t next = dyn ? atomicAdd(p.sched, 1u) : blockIdx.x;
+            for (uint32_t i = 0; !stop; ++i) {
+                const uint32_t slot = i % kSlots;
+                if (!bounded_wait(&sempty[slot], ((i / kSlots) & 1u) ^ 1u, abort_flag, p.err,
+                                  kErrTimeoutEpi))
+                    break;
+                const uint32_t uu = next;
+                if (uu < static_cast<uint32_t>(total))
+                    next = dyn ? atomicAdd(p.sched, 1u) : uu + gridDim.x;
+                sched_id[slot] = uu;
+                ptx::mbar_arrive(&sfull[slot]);
+                if (uu >= static_cast<uint32_t>(total)) break;
+                const int u = static_cast<int>(uu);
                 const Unit w =
                     decode_unit<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
                 const CUtensorMap *ta0 = w.up ? &tmW1 : &tmW2;
@@ -360,9 +392,15 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
-            int i = 0;
             bool stop = false;
-            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x, ++i) {
+            for (uint32_t i = 0; !stop; ++i) {
+                const uint32_t slot = i % kSlots;
+                if (!bounded_wait(&sfull[slot], (i / kSlots) & 1u, abort_flag, p.err, kErrTimeoutEpi))
+                    break;
+                const uint32_t uu = *reinterpret_cast<volatile uint32_t *>(&sched_id[slot]);
+                ptx::mbar_arrive(&sempty[slot]);
+                if (uu >= static_cast<uint32_t>(total)) break;
+                const int u = static_cast<int>(uu);
                 const Unit w =
                     decode_unit<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
                 const int n = ((w.valid + 15) >> 4) << 4;
@@ -406,8 +444,16 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     } else {
         const int q = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-        int i = 0;
-        for (int u = blockIdx.x; u < total; u += gridDim.x, ++i) {
+        for (uint32_t i = 0;; ++i) {
+            const uint32_t slot = i % kSlots;
+            if (!bounded_wait_warp(&sfull[slot], (i / kSlots) & 1u, abort_flag, p.err,
+                                   kErrTimeoutEpi))
+                break;
+            const uint32_t uu = *reinterpret_cast<volatile uint32_t *>(&sched_id[slot]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sempty[slot]);
+            if (uu >= static_cast<uint32_t>(total)) break;
+            const int u = static_cast<int>(uu);
             const Unit w = decode_unit<BN>(u, u_up, s_off, s_pu, s_pd, s_tb, E, KSPLIT, KSU, KSD);
             const int buf = i & 1;
             const uint32_t use = static_cast<uint32_t>(i >> 1);
@@ -502,6 +548,7 @@ cudaError_t launch_ffn_cfg(const FfnLaunch &a, cudaStream_t s)
     p.err = a.err;
     p.stream_weights = a.max_rows <= BN ? 1 : 0;
     p.act = a.act;
+    p.sched = a.sched;
     // Upper bound of the work units: every segment rounds up to whole tiles.
     const long long tiles = (static_cast<long long>(a.S) + BN - 1) / BN + E;
     const long long units = tiles * (a.d_ff / 128) + tiles * ((a.d + 255) / 256) * p.ksplit;
