@@ -96,6 +96,7 @@ typedef enum {
 #define MOE_DEVERR_OFFSETS 0x8u      /* offsets[] not non-decreasing within [0, S] */
 #define MOE_DEVERR_INDEX 0x10u       /* an expert index or row index out of range */
 #define MOE_DEVERR_LAYOUT 0x20u      /* a kernel found its shared memory misplaced and did nothing */
+#define MOE_DEVERR_EP_COUNTS 0x40u   /* moe_ep_dispatch: counts_all disagrees with idx or overflows */
 
 /* Bytes of workspace every entry point below needs for these shapes
  * (the largest need over all of them).  0 if the shapes are unsupported. */
@@ -345,6 +346,108 @@ MOE_API moe_status moe_forward_fp8_traced(int T, int d, int E, int d_ff, int k,
  * if a timeout bit is set, MOE_ERR_DEVICE for any other bit, MOE_ERR_CUDA if
  * the wait or the read failed. */
 MOE_API moe_status moe_get_device_error(const void *ws, uint32_t *code, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism over R ranks, one GPU each (R <= 8, E a multiple of R).
+ * Rank q owns experts [q*E/R, (q+1)*E/R) and holds only their weights
+ * (W1, W3, W2 of moe_ep_expert_ffn are that block, [E/R, ...]).  Every rank
+ * keeps a receive buffer recv_x [recv_rows, d] bf16 and an output buffer
+ * recv_y [ksplit, recv_rows, d] fp32 that every other rank can address (its
+ * own allocation, mapped into the peers with moe_ipc_get_handle /
+ * moe_ipc_open_handle), with recv_rows = moe_ep_recv_rows(T_max, E, k, R).
+ * One layer step, on every rank, all on one stream:
+ *   1. moe_route on the rank's own T <= T_max tokens: idx, w, counts[E];
+ *   2. an all-gather of counts over the ranks into counts_all [R, E] (row r
+ *      = rank r's counts), e.g. an NCCL all-gather on the same stream;
+ *   3. moe_ep_dispatch: every (token, slot) row of x is stored straight into
+ *      its expert owner's recv_x (the all-to-all and the permutation in one
+ *      kernel);
+ *   4. a barrier across the ranks on the stream (e.g. an NCCL all-reduce of
+ *      one word), so that every row has arrived;
+ *   5. moe_ep_expert_ffn on the rank's own recv_x -> recv_y;
+ *   6. a barrier, so that every output row is complete;
+ *   7. moe_ep_combine: each token's k expert rows are read from their
+ *      owners' recv_y and summed, gate-weighted, in slot order.
+ * No kernel waits for another GPU: the ordering across GPUs is that of the
+ * caller's collectives in steps 2, 4 and 6, and nothing is read back to the
+ * host, so the step can be captured in a CUDA graph.  Step 2 of the next
+ * layer call also orders that call's stores after this call's reads.
+ * Receive layout of owner q: its experts in index order; inside an expert,
+ * the rows from rank 0, then rank 1, ...; inside one sender, token order.
+ * out equals moe_forward's result up to the order of the fp32 additions
+ * inside the expert kernels.
+ * Passages: jsqmd.com, deployment section, problem 4 (experts placed on
+ * several GPUs by hand to balance memory and load); theaiera.top sec. 10.4
+ * (per-expert gathering and weighted index_add, here across ranks). */
+
+/* Receive rows per rank: R * T_max * min(k, E/R) (every token of every rank
+ * may reach min(k, E/R) experts of one owner); 0 if the sizes are invalid. */
+MOE_API int moe_ep_recv_rows(int T_max, int E, int k, int R);
+
+/* Workspace bytes of one rank for steps 3 and 5 (0: unsupported sizes). */
+MOE_API size_t moe_ep_workspace_size(int T_max, int d, int E, int d_ff, int k, int R);
+
+/* K splits of the down projection moe_ep_expert_ffn uses when a rank
+ * expects rows_hint received rows (recv_y then holds that many partial
+ * outputs per row, summed by moe_ep_combine). */
+MOE_API int moe_ep_ffn_splits(int rows_hint, int d, int E_local, int d_ff);
+
+/* Step 3 on rank `rank`.
+ *   x [T,d] bf16, idx [T,k] int32 (this rank's routing), counts_all [R,E]
+ *   int32 (device), recv_x: host array of R device addresses (element r =
+ *   rank r's receive buffer as this GPU addresses it), recv_rows: rows of each.
+ *   pos_of_slot [T,k] int32 out: the receive row of (t, j) in the owner of
+ *   expert idx[t,j]; recv_offsets [E/R+1] int32 out: segment starts of this
+ *   rank's experts in its own recv_x (valid once every rank's counts are in
+ *   counts_all, which they are after step 2).
+ * If counts_all's own row differs from the counts of idx, or some owner
+ * would receive more than recv_rows rows, MOE_DEVERR_EP_COUNTS is set in the
+ * workspace's error word, nothing is sent and pos_of_slot is all -1.  Resets
+ * the error word (read with moe_get_device_error after step 5). */
+MOE_API moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank,
+                                   const moe_bf16 *x, const int32_t *idx,
+                                   const int32_t *counts_all, moe_bf16 *const *recv_x,
+                                   int recv_rows, int32_t *pos_of_slot, int32_t *recv_offsets,
+                                   void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Step 5: moe_expert_ffn over this rank's E/R experts on its receive buffer
+ * (recv_rows = moe_ep_recv_rows(T_max, E, k, R) rows, segments from
+ * recv_offsets).  rows_hint: rows the rank expects to receive (T*k with
+ * balanced experts; it picks the kernel's tiling, not the result); ksplit must be
+ * moe_ep_ffn_splits(rows_hint, d, E/R, d_ff).  recv_y [ksplit, recv_rows, d]
+ * fp32 out (rows beyond the segments are not written).  Keeps the error
+ * word of the step's dispatch. */
+MOE_API moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R,
+                                     int rows_hint, int ksplit, const moe_bf16 *recv_x,
+                                     const int32_t *recv_offsets, const moe_bf16 *W1,
+                                     const moe_bf16 *W3, const moe_bf16 *W2, float *recv_y,
+                                     void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Step 7: out[t] = sum_{j<k} w[t,j] * (sum_q recv_y_o[q, pos_of_slot[t,j]])
+ * (+ shared_y[t]), o = owner of idx[t,j], slots in order j = 0..k-1, the K
+ * split partials q in order.  recv_y: host array of R device addresses of
+ * the ranks' output buffers.  A slot with pos_of_slot -1 adds nothing.
+ * out [T,d] fp32 (overwritten). */
+MOE_API moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int ksplit,
+                                  const int32_t *idx, const int32_t *pos_of_slot, const float *w,
+                                  const float *const *recv_y, const float *shared_y, float *out,
+                                  moe_stream_t stream);
+
+/* Size of an inter-process memory handle (cudaIpcMemHandle_t). */
+#define MOE_IPC_HANDLE_BYTES 64
+
+/* Handle of the device allocation that holds dev_ptr, for another process
+ * on this node: handle (MOE_IPC_HANDLE_BYTES) out, *offset out = dev_ptr's
+ * offset in that allocation. */
+MOE_API moe_status moe_ipc_get_handle(const void *dev_ptr, void *handle, size_t *offset);
+
+/* Maps another process's allocation into this one (peer access enabled):
+ * *base out = its first byte here; add the sender's offset.  Not for a
+ * handle of this process's own memory. */
+MOE_API moe_status moe_ipc_open_handle(const void *handle, void **base);
+
+/* Unmaps a base returned by moe_ipc_open_handle. */
+MOE_API moe_status moe_ipc_close(void *base);
 
 /* Static description of a status code; never NULL. */
 MOE_API const char *moe_status_string(moe_status status);

@@ -13,6 +13,7 @@ from .oracle import (  # noqa: F401
     build,
     capacity_limit,
     e4m3_to_double,
+    ep_plan,
     forward_fp8,
     num_threads,
     route,

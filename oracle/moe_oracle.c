@@ -512,3 +512,47 @@ int oracle_swiglu(int n, int d, int dff, const uint16_t *x, const uint16_t *W1,
     }
     return err ? -1 : 0;
 }
+
+/* Expert parallelism: where every (rank, token, slot) pair lands when the E
+ * experts are split over R ranks in contiguous blocks (owner of expert e:
+ * e / (E/R)).  The pages place experts on GPUs by hand (jsqmd.com,
+ * deployment section, problem 4) and fix no order inside a GPU; the order
+ * below is the one this library defines, written out as nested loops:
+ *   for each owner q, for each of its experts e in index order,
+ *     for each sending rank r in order, for each token t in order, slot j:
+ *       if idx_r[t, j] == e, the pair takes the owner's next receive row.
+ * T_of[r]: tokens of rank r; idx_all: the R ranks' [T_r, k] arrays back to
+ * back; pos_all out (same layout): the receive row of each pair (-1 if its
+ * expert is outside [0, E)); offsets out [R][E/R + 1]: each owner's segment
+ * starts. */
+int oracle_ep_plan(int R, int E, int k, const int32_t *T_of, const int32_t *idx_all,
+                   int32_t *pos_all, int32_t *offsets)
+{
+    if (R < 1 || E < R || E % R != 0 || k < 1 || !T_of || !pos_all || !offsets) return -1;
+    const int El = E / R;
+    size_t total = 0;
+    for (int r = 0; r < R; ++r) {
+        if (T_of[r] < 0) return -1;
+        total += (size_t)T_of[r] * (size_t)k;
+    }
+    if (total > 0 && !idx_all) return -1;
+    for (size_t i = 0; i < total; ++i) pos_all[i] = -1;
+    for (int q = 0; q < R; ++q) {
+        int32_t row = 0;
+        int32_t *seg = offsets + (size_t)q * (size_t)(El + 1);
+        seg[0] = 0;
+        for (int e = q * El; e < (q + 1) * El; ++e) {
+            size_t first = 0;  /* rank r's first pair in idx_all */
+            for (int r = 0; r < R; ++r) {
+                for (int t = 0; t < T_of[r]; ++t)
+                    for (int j = 0; j < k; ++j) {
+                        const size_t i = first + (size_t)t * (size_t)k + (size_t)j;
+                        if (idx_all[i] == e) pos_all[i] = row++;
+                    }
+                first += (size_t)T_of[r] * (size_t)k;
+            }
+            seg[e - q * El + 1] = row;
+        }
+    }
+    return 0;
+}

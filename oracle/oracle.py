@@ -62,6 +62,8 @@ def _load():
                                            _P, _P, _P, _P, _P]
         lib.oracle_swiglu.restype = _I
         lib.oracle_swiglu.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P]
+        lib.oracle_ep_plan.restype = _I
+        lib.oracle_ep_plan.argtypes = [_I, _I, _I, _P, _P, _P, _P]
         _lib = lib
     return _lib
 
@@ -206,3 +208,29 @@ def forward_fp8(x, Wg, q1, s1, q3, s3, q2, s2, k: int, bias=None, tokens=None, f
     if rc != 0:
         raise ValueError("oracle_forward_fp8 rejected its arguments")
     return out
+
+
+
+def ep_plan(idx_per_rank, E: int, R: int):
+    """Receive layout of the layer split over R ranks by experts (see
+    ``oracle_ep_plan`` in moe_oracle.c for the order).  ``idx_per_rank[r]``:
+    rank r's [T_r, k] expert indices.  Returns ``(pos, offsets)``: pos[r]
+    [T_r, k] int32, the receive row of each pair in the owner of its expert;
+    offsets[q] [E/R + 1] int32, owner q's segment starts."""
+    assert R >= 1 and E % R == 0 and len(idx_per_rank) == R
+    arrs = [np.ascontiguousarray(i, dtype=np.int32) for i in idx_per_rank]
+    k = arrs[0].shape[1]
+    assert all(a.ndim == 2 and a.shape[1] == k for a in arrs)
+    T_of = np.array([a.shape[0] for a in arrs], np.int32)
+    idx_all = np.ascontiguousarray(np.concatenate([a.ravel() for a in arrs]), dtype=np.int32)
+    pos_all = np.empty_like(idx_all)
+    offsets = np.empty((R, E // R + 1), np.int32)
+    rc = _load().oracle_ep_plan(R, E, k, _ptr(T_of), _ptr(idx_all), _ptr(pos_all),
+                                _ptr(offsets))
+    if rc != 0:
+        raise ValueError("oracle_ep_plan rejected its arguments")
+    pos, start = [], 0
+    for a in arrs:
+        pos.append(pos_all[start:start + a.size].reshape(a.shape))
+        start += a.size
+    return pos, [offsets[q] for q in range(R)]

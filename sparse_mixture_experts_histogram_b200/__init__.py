@@ -16,6 +16,12 @@ from .binding import (  # noqa: F401
     MoEVariant,
     load_library,
     moe_combine,
+    moe_ep_combine,
+    moe_ep_dispatch,
+    moe_ep_expert_ffn,
+    moe_ep_ffn_splits,
+    moe_ep_recv_rows,
+    moe_ep_workspace_size,
     moe_expert_ffn,
     moe_expert_ffn_static,
     moe_expert_ffn_static_bytes,
@@ -27,6 +33,9 @@ from .binding import (  # noqa: F401
     moe_forward_traced,
     moe_forward_variant,
     moe_get_device_error,
+    moe_ipc_close,
+    moe_ipc_get_handle,
+    moe_ipc_open_handle,
     moe_permute,
     moe_route,
     moe_route_variant,

@@ -21,7 +21,9 @@ STATUS_NAMES = {
     4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE", 6: "MOE_ERR_TIMEOUT",
 }
 DEVERR_BITS = {0x1: "TIMEOUT_TMA", 0x2: "TIMEOUT_MMA", 0x4: "TIMEOUT_EPI", 0x8: "OFFSETS",
-               0x10: "INDEX", 0x20: "LAYOUT"}
+               0x10: "INDEX", 0x20: "LAYOUT", 0x40: "EP_COUNTS"}
+#: Bytes of an inter-process memory handle (MOE_IPC_HANDLE_BYTES).
+IPC_HANDLE_BYTES = 64
 
 #: Every symbol the C header declares (checked against ``include/moe.h`` by the tests).
 ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "moe_permute",
@@ -29,7 +31,10 @@ ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "mo
                  "moe_forward_traced", "moe_get_device_error", "moe_status_string",
                  "moe_expert_ffn_static", "moe_expert_ffn_static_bytes",
                  "moe_expert_ffn_static_error", "moe_forward_variant", "moe_route_variant",
-                 "moe_forward_fp8", "moe_forward_fp8_traced")
+                 "moe_forward_fp8", "moe_forward_fp8_traced", "moe_ep_recv_rows",
+                 "moe_ep_workspace_size", "moe_ep_ffn_splits", "moe_ep_dispatch",
+                 "moe_ep_expert_ffn", "moe_ep_combine", "moe_ipc_get_handle",
+                 "moe_ipc_open_handle", "moe_ipc_close")
 TRACE_EVENTS = 6
 #: What each of moe_forward_traced's events marks (event i = start of stage i).
 TRACE_STAGES = ("route", "scatter", "expert_ffn", "shared_ffn", "combine")
@@ -90,6 +95,15 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
             "moe_expert_ffn_static_bytes": (_SZ, [_I] * 3),
             "moe_expert_ffn_static_error": (_I, [_P, _P]),
             "moe_status_string": (ctypes.c_char_p, [_I]),
+            "moe_ep_recv_rows": (_I, [_I] * 4),
+            "moe_ep_workspace_size": (_SZ, [_I] * 6),
+            "moe_ep_ffn_splits": (_I, [_I] * 4),
+            "moe_ep_dispatch": (_I, [_I] * 6 + [_P] * 4 + [_I] + [_P] * 3 + [_SZ, _P]),
+            "moe_ep_expert_ffn": (_I, [_I] * 8 + [_P] * 7 + [_SZ, _P]),
+            "moe_ep_combine": (_I, [_I] * 7 + [_P] * 6 + [_P]),
+            "moe_ipc_get_handle": (_I, [_P, _P, _P]),
+            "moe_ipc_open_handle": (_I, [_P, _P]),
+            "moe_ipc_close": (_I, [_P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -270,3 +284,75 @@ def moe_get_device_error(ws, stream=None) -> tuple[int, int]:
     code = ctypes.c_uint32(0)
     st = load_library().moe_get_device_error(_ptr(ws), ctypes.byref(code), _stream(stream))
     return int(st), int(code.value)
+
+
+# ------------------------------------------------------- expert parallelism
+
+def _ptr_array(ptrs):
+    return (ctypes.c_void_p * len(ptrs))(*[_ptr(p) for p in ptrs])
+
+
+def moe_ep_recv_rows(T_max, E, k, R) -> int:
+    return int(load_library().moe_ep_recv_rows(T_max, E, k, R))
+
+
+def moe_ep_workspace_size(T_max, d, E, d_ff, k, R) -> int:
+    return int(load_library().moe_ep_workspace_size(T_max, d, E, d_ff, k, R))
+
+
+def moe_ep_ffn_splits(rows_hint, d, E_local, d_ff) -> int:
+    return int(load_library().moe_ep_ffn_splits(rows_hint, d, E_local, d_ff))
+
+
+def moe_ep_dispatch(T, d, E, k, R, rank, x, idx, counts_all, recv_x, recv_rows, pos_of_slot,
+                    recv_offsets, ws, stream=None):
+    """``recv_x``: the R ranks' receive buffers (tensors or device addresses
+    as this GPU sees them), in rank order."""
+    if len(recv_x) != R:
+        raise ValueError(f"need {R} receive buffers")
+    _check(load_library().moe_ep_dispatch(T, d, E, k, R, rank, _ptr(x), _ptr(idx),
+                                          _ptr(counts_all), _ptr_array(recv_x), recv_rows,
+                                          _ptr(pos_of_slot), _ptr(recv_offsets), _ptr(ws),
+                                          _ws_bytes(ws), _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_expert_ffn(T_max, d, E, d_ff, k, R, rows_hint, ksplit, recv_x, recv_offsets, W1, W3,
+                      W2, recv_y, ws, stream=None):
+    _check(load_library().moe_ep_expert_ffn(T_max, d, E, d_ff, k, R, rows_hint, ksplit,
+                                            _ptr(recv_x), _ptr(recv_offsets), _ptr(W1), _ptr(W3),
+                                            _ptr(W2), _ptr(recv_y), _ptr(ws), _ws_bytes(ws),
+                                            _stream(stream)), "moe_ep_expert_ffn")
+
+
+def moe_ep_combine(T, d, E, k, R, recv_rows, ksplit, idx, pos_of_slot, w, recv_y, shared_y, out,
+                   stream=None):
+    """``recv_y``: the R ranks' output buffers, in rank order."""
+    if len(recv_y) != R:
+        raise ValueError(f"need {R} output buffers")
+    _check(load_library().moe_ep_combine(T, d, E, k, R, recv_rows, ksplit, _ptr(idx),
+                                         _ptr(pos_of_slot), _ptr(w), _ptr_array(recv_y),
+                                         _ptr(shared_y), _ptr(out), _stream(stream)),
+           "moe_ep_combine")
+
+
+def moe_ipc_get_handle(dev_ptr) -> tuple[bytes, int]:
+    """(handle bytes, offset of dev_ptr in its allocation)."""
+    h = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t(0)
+    _check(load_library().moe_ipc_get_handle(_ptr(dev_ptr), h, ctypes.byref(off)),
+           "moe_ipc_get_handle")
+    return h.raw, int(off.value)
+
+
+def moe_ipc_open_handle(handle: bytes) -> int:
+    """Base address of another process's allocation, mapped here."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes")
+    h = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+    base = ctypes.c_void_p(0)
+    _check(load_library().moe_ipc_open_handle(h, ctypes.byref(base)), "moe_ipc_open_handle")
+    return int(base.value)
+
+
+def moe_ipc_close(base: int) -> None:
+    _check(load_library().moe_ipc_close(base), "moe_ipc_close")

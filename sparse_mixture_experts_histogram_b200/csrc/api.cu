@@ -26,6 +26,8 @@ constexpr size_t kHeaderBytes = 256;  // error word @0, routing counter @4, rank
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
+constexpr int kMaxRanksHost = 8;  // ranks of one expert-parallel group (kMaxRanks of ep.cu)
+
 struct Layout {
     size_t tilectr, hready, hready_s, gcnt;
     size_t zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
@@ -115,6 +117,19 @@ void load_encode()
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+PFN_cuMemGetAddressRange_v3020 g_range = nullptr;
+std::once_flag g_range_once;
+
+void load_range()
+{
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
 }
 
 constexpr int kMaxDevices = 64;
@@ -214,6 +229,68 @@ int device_sm_count()
         n = 148;
     g_sm_count[dev].store(n, std::memory_order_relaxed);
     return n;
+}
+
+// ------------------------------------------------------- expert parallelism
+// Receive rows per rank: every rank may send each of its T_max tokens to at
+// most min(k, E/R) experts of one owner.
+long long ep_recv_rows_ll(int T_max, int E, int k, int R)
+{
+    if (T_max < 1 || R < 1 || R > kMaxRanksHost || E < R || E % R != 0 || k < 1 || k > E) return 0;
+    return static_cast<long long>(R) * T_max * std::min(k, E / R);
+}
+
+// Workspace of one rank: the dispatch's part (sized by the call's T), then
+// the expert kernel's part, placed after the dispatch part of T_max so that
+// it does not move with the T of a step.
+struct EpLayout {
+    size_t tilecnt, tilebase, rank, offsets, base, ok, disp_end;
+    size_t ffnctr;      // expert kernel: work counter @0, readiness counters @kAlign
+    size_t H, total;
+};
+
+EpLayout ep_layout(int T, int T_max, int E, int d_ff, int k, int R)
+{
+    EpLayout L{};
+    auto dispatch_part = [&](int Tn, EpLayout &D) {
+        size_t o = kHeaderBytes;
+        auto take = [&](size_t bytes) {
+            const size_t r = o;
+            o += align_up(bytes);
+            return r;
+        };
+        const size_t ntiles = (static_cast<size_t>(Tn) + 127) / 128;
+        D.tilecnt = take(ntiles * E * 4);
+        D.tilebase = take(ntiles * E * 4);
+        D.rank = take(static_cast<size_t>(Tn) * k * 4);
+        D.offsets = take((static_cast<size_t>(E) + 1) * 4);
+        D.base = take(static_cast<size_t>(E) * 4);
+        D.ok = take(4);
+        D.disp_end = o;
+    };
+    EpLayout M{};
+    dispatch_part(T_max, M);
+    dispatch_part(T, L);
+    const int rows = static_cast<int>(ep_recv_rows_ll(T_max, E, k, R));
+    size_t o = M.disp_end;
+    L.ffnctr = o;
+    o += align_up(kAlign + ffn_ready_counters(rows, E / R, d_ff) * 4);
+    L.H = o;
+    o += align_up(static_cast<size_t>(rows) * d_ff * 2);
+    L.total = o;
+    return L;
+}
+
+// Shapes of one rank of an expert-parallel layer.
+moe_status ep_check(int T, int d, int E, int d_ff, int k, int R)
+{
+    if (R < 1 || T < 1 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+    if (R > kMaxRanksHost) return MOE_ERR_UNSUPPORTED;
+    if (E % R != 0 || k > E) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_shapes(T, d, E, d_ff, k, 0);
+    if (st != MOE_OK) return st;
+    const long long rows = ep_recv_rows_ll(T, E, k, R);
+    return check_shapes(static_cast<int>(std::min<long long>(rows, 1 << 30)), d, E / R, d_ff, 1, 0);
 }
 
 }  // namespace moe
@@ -874,6 +951,193 @@ moe_status moe_get_device_error(const void *ws, uint32_t *code, moe_stream_t str
     if (word & (MOE_DEVERR_TIMEOUT_TMA | MOE_DEVERR_TIMEOUT_MMA | MOE_DEVERR_TIMEOUT_EPI))
         return MOE_ERR_TIMEOUT;
     return MOE_ERR_DEVICE;
+}
+
+
+// ------------------------------------------------------- expert parallelism
+
+int moe_ep_recv_rows(int T_max, int E, int k, int R)
+{
+    const long long rows = ep_recv_rows_ll(T_max, E, k, R);
+    return rows > (1LL << 30) ? 0 : static_cast<int>(rows);
+}
+
+size_t moe_ep_workspace_size(int T_max, int d, int E, int d_ff, int k, int R)
+{
+    if (ep_check(T_max, d, E, d_ff, k, R) != MOE_OK) return 0;
+    return ep_layout(T_max, T_max, E, d_ff, k, R).total;
+}
+
+int moe_ep_ffn_splits(int rows_hint, int d, int E_local, int d_ff)
+{
+    if (rows_hint < 1 || E_local < 1 || d < 128 || d_ff < 128) return 0;
+    return down_ksplit(rows_hint, E_local, d, d_ff);
+}
+
+moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank, const moe_bf16 *x,
+                           const int32_t *idx, const int32_t *counts_all,
+                           moe_bf16 *const *recv_x, int recv_rows, int32_t *pos_of_slot,
+                           int32_t *recv_offsets, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = ep_check(T, d, E, 128, k, R);
+    if (st != MOE_OK) return st;
+    if (rank < 0 || rank >= R || recv_rows < 1 || recv_x == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!ok_ptr(x) || !ok_ptr(idx) || !ok_ptr(counts_all) || !ok_ptr(pos_of_slot) ||
+        !ok_ptr(recv_offsets) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    for (int r = 0; r < R; ++r)
+        if (!ok_ptr(recv_x[r])) return MOE_ERR_INVALID_ARG;
+    const EpLayout L = ep_layout(T, T, E, 128, k, R);
+    if (ws_bytes < L.disp_end) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
+    if (st != MOE_OK) return st;
+    RanksLaunch r{};
+    r.T = T;
+    r.E = E;
+    r.k = k;
+    r.idx = idx;
+    r.offsets = reinterpret_cast<int32_t *>(wsb + L.offsets);
+    r.tilecnt = reinterpret_cast<int32_t *>(wsb + L.tilecnt);
+    r.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
+    r.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
+    r.done = reinterpret_cast<uint32_t *>(wsb + 8);
+    r.err = reinterpret_cast<uint32_t *>(wsb);
+    st = from_cuda(launch_ranks(r, s));
+    if (st != MOE_OK) return st;
+    EpDispatchLaunch a{};
+    a.T = T;
+    a.d = d;
+    a.E = E;
+    a.k = k;
+    a.R = R;
+    a.rank = rank;
+    a.recv_rows = recv_rows;
+    a.x = x;
+    a.idx = idx;
+    a.counts_all = counts_all;
+    a.offsets = r.offsets;
+    a.tilebase = r.tilebase;
+    a.rank_of_pair = r.rank;
+    a.base = reinterpret_cast<int32_t *>(wsb + L.base);
+    a.ok = reinterpret_cast<uint32_t *>(wsb + L.ok);
+    a.recv_x = recv_x;
+    a.pos_of_slot = pos_of_slot;
+    a.recv_offsets = recv_offsets;
+    a.err = r.err;
+    return from_cuda(launch_ep_dispatch(a, s));
+}
+
+moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R, int rows_hint,
+                             int ksplit, const moe_bf16 *recv_x, const int32_t *recv_offsets,
+                             const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2,
+                             float *recv_y, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status st = ep_check(T_max, d, E, d_ff, k, R);
+    if (st != MOE_OK) return st;
+    const int E_local = E / R;
+    const int recv_rows = moe_ep_recv_rows(T_max, E, k, R);
+    if (recv_rows < 1 || rows_hint < 1) return MOE_ERR_INVALID_ARG;
+    if (ksplit != moe_ep_ffn_splits(rows_hint, d, E_local, d_ff)) return MOE_ERR_INVALID_ARG;
+    if (!ok_ptr(recv_x) || !ok_ptr(recv_offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+        !ok_ptr(recv_y) || !ok_ptr(ws))
+        return MOE_ERR_INVALID_ARG;
+    const EpLayout L = ep_layout(T_max, T_max, E, d_ff, k, R);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    // Counters only: the error word keeps what the dispatch of this step found.
+    const size_t ctr = kAlign + ffn_ready_counters(recv_rows, E_local, d_ff) * 4;
+    st = from_cuda(cudaMemsetAsync(wsb + L.ffnctr, 0, ctr, s));
+    if (st != MOE_OK) return st;
+    FfnLaunch f{};
+    f.E = E_local;
+    f.d = d;
+    f.d_ff = d_ff;
+    f.S = recv_rows;
+    f.S_hint = rows_hint;
+    f.max_rows = std::min(recv_rows, R * T_max);
+    f.ksplit = ksplit;
+    f.offsets = recv_offsets;
+    f.W1 = W1;
+    f.W3 = W3;
+    f.W2 = W2;
+    f.x = recv_x;
+    f.H = reinterpret_cast<moe_bf16 *>(wsb + L.H);
+    f.Y = recv_y;
+    f.h_ready = reinterpret_cast<uint32_t *>(wsb + L.ffnctr + kAlign);
+    f.sched = reinterpret_cast<uint32_t *>(wsb + L.ffnctr);
+    f.err = reinterpret_cast<uint32_t *>(wsb);
+    f.pdl = false;
+    f.k = 1;
+    return from_cuda(launch_ffn(f, s));
+}
+
+moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int ksplit,
+                          const int32_t *idx, const int32_t *pos_of_slot, const float *w,
+                          const float *const *recv_y, const float *shared_y, float *out,
+                          moe_stream_t stream)
+{
+    if (T < 1 || d < 1 || E < 1 || k < 1 || R < 1 || recv_rows < 1 || ksplit < 1)
+        return MOE_ERR_INVALID_ARG;
+    if (R > kMaxRanksHost || k > 8 || T > (1 << 24) || d % 128 || d > 16384 || E > 256 ||
+        ksplit > 8)
+        return MOE_ERR_UNSUPPORTED;
+    if (E % R != 0 || k > E || recv_y == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!ok_ptr(idx) || !ok_ptr(pos_of_slot) || !ok_ptr(w) || !ok_ptr(out))
+        return MOE_ERR_INVALID_ARG;
+    if (shared_y != nullptr && !aligned16(shared_y)) return MOE_ERR_INVALID_ARG;
+    for (int r = 0; r < R; ++r)
+        if (!ok_ptr(recv_y[r])) return MOE_ERR_INVALID_ARG;
+    EpCombineLaunch c{};
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.k = k;
+    c.R = R;
+    c.recv_rows = recv_rows;
+    c.ksplit = ksplit;
+    c.idx = idx;
+    c.pos_of_slot = pos_of_slot;
+    c.w = w;
+    c.recv_y = recv_y;
+    c.shared_y = shared_y;
+    c.out = out;
+    return from_cuda(launch_ep_combine(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ipc_get_handle(const void *dev_ptr, void *handle, size_t *offset)
+{
+    if (dev_ptr == nullptr || handle == nullptr || offset == nullptr) return MOE_ERR_INVALID_ARG;
+    std::call_once(g_range_once, load_range);
+    if (g_range == nullptr) return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t bytes = 0;
+    if (g_range(&base, &bytes, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+        return MOE_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) return MOE_ERR_CUDA;
+    static_assert(sizeof(h) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+    std::memcpy(handle, &h, sizeof(h));
+    *offset = static_cast<size_t>(reinterpret_cast<uintptr_t>(dev_ptr) - base);
+    return MOE_OK;
+}
+
+moe_status moe_ipc_open_handle(const void *handle, void **base)
+{
+    if (handle == nullptr || base == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    if (cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_ipc_close(void *base)
+{
+    if (base == nullptr) return MOE_ERR_INVALID_ARG;
+    return from_cuda(cudaIpcCloseMemHandle(base));
 }
 
 }  // extern "C"

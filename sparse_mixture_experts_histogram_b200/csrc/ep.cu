@@ -1,0 +1,365 @@
+// ep.cu -- expert parallelism: the E experts are split in contiguous blocks
+// of E/R over R ranks (one GPU each); every (token, slot) row travels to the
+// rank that owns its expert, and the expert's output row travels back.
+//
+//  * ep_plan_kernel: from every rank's per-expert pair counts (all-gathered
+//    by the caller into counts_all[R, E]), the first receive row of each
+//    (expert, this source rank) block in its owner's buffer, and this rank's
+//    own receive segments (its experts' offsets).
+//  * ep_dispatch_kernel: x[t] is stored straight into the owner's receive
+//    buffer (peer memory over NVLink when the owner is another GPU) at the
+//    block's first row + the pair's rank in token order.  The scatter of the
+//    single-GPU layer and the all-to-all of rows are one pass over x.
+//  * ep_combine_kernel: each slot's expert output row is loaded from its
+//    owner's output buffer (peer memory) and the k rows are summed,
+//    gate-weighted, in slot order.
+//
+// Receive layout on owner q: its experts in index order; inside an expert,
+// the rows sent by rank 0, then rank 1, ...; inside one sender, token order.
+// Every row's place follows from the routing alone, so the result does not
+// depend on timing or on which rank finishes first.
+//
+// Method: the placement of experts on several GPUs ("Mistral 8x7B SMoE
+// architecture", jsqmd.com, problem 4 of the deployment section: experts
+// assigned to GPUs by hand to even out memory and load); the per-expert
+// gathering and weighted index_add of "MoE" (theaiera.top, LLMs-from-scratch
+// ch.10) sec. 10.4, done across ranks.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "launch.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaxRanks = 8;          // ranks of one expert-parallel group
+constexpr uint32_t kErrEpCounts = 0x40u;  // MOE_DEVERR_EP_COUNTS
+constexpr int kPlanThreads = 256;  // one thread per expert (E <= kMaxE = 256)
+static_assert(kPlanThreads >= kMaxE, "one plan thread per expert");
+
+struct PlanParams {
+    int E, R, rank, El;
+    int recv_rows;               // rows of every rank's receive buffer
+    const int32_t *counts_all;   // [R, E]
+    const int32_t *offsets;      // [E+1] this rank's own expert segments (ranks_kernel)
+    int32_t *base;               // [E] out: first receive row of (expert e, this rank)
+    int32_t *recv_offsets;       // [El+1] out: this rank's receive segments
+    uint32_t *ok;                // out: 1 when the counts are consistent
+    uint32_t *err;
+};
+
+// Exclusive prefix over the block's threads (kPlanThreads values).
+__device__ int block_excl_scan(int v, int *warp_tot)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    return before + incl - v;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(const __grid_constant__ PlanParams p)
+{
+    __shared__ int warp_tot[kPlanThreads / 32];
+    __shared__ int excl_s[kMaxE + 1];
+    __shared__ int bad_s;
+    const int e = threadIdx.x;
+    if (e == 0) bad_s = 0;
+    __syncthreads();
+    int colsum = 0, below = 0;
+    bool bad = false;
+    if (e < p.E) {
+        for (int r = 0; r < p.R; ++r) {
+            const int c = p.counts_all[static_cast<size_t>(r) * p.E + e];
+            if (c < 0) bad = true;
+            colsum += c;
+            if (r < p.rank) below += c;
+        }
+        // This rank's row of counts_all must be what its own idx holds.
+        const int mine = p.counts_all[static_cast<size_t>(p.rank) * p.E + e];
+        if (mine != p.offsets[e + 1] - p.offsets[e]) bad = true;
+    }
+    const int excl = block_excl_scan(e < p.E ? colsum : 0, warp_tot);
+    if (e < p.E) excl_s[e] = excl;
+    if (e == p.E - 1) excl_s[p.E] = excl + colsum;
+    if (bad) atomicOr(&bad_s, 1);
+    __syncthreads();
+    if (e < p.E) {
+        const int q0 = (e / p.El) * p.El;  // first expert of e's owner
+        p.base[e] = excl - excl_s[q0] + below;
+    }
+    // Rows each owner receives must fit its buffer.
+    if (e < p.R && excl_s[(e + 1) * p.El] - excl_s[e * p.El] > p.recv_rows) atomicOr(&bad_s, 1);
+    const int q0 = p.rank * p.El;
+    for (int i = e; i <= p.El; i += kPlanThreads) p.recv_offsets[i] = excl_s[q0 + i] - excl_s[q0];
+    __syncthreads();
+    if (e == 0) {
+        *p.ok = bad_s ? 0u : 1u;
+        if (bad_s) atomicOr(p.err, kErrEpCounts);
+    }
+}
+
+struct EpDispatchParams {
+    int T, d, E, k, El, R;
+    int recv_rows;
+    const uint4 *x;
+    const int32_t *idx, *rank, *tilebase, *offsets, *base;
+    const uint32_t *ok;
+    uint4 *recv[kMaxRanks];  // every rank's receive buffer [recv_rows, d] bf16
+    int32_t *pos_of_slot;    // [T, k] out
+    uint32_t *err;
+    int chunks;              // 16-byte-vector chunks of kEpVec*32 per row
+};
+
+constexpr int kEpWarps = 8;
+constexpr int kEpVec = 4;  // 16-byte vectors per lane per chunk
+
+// The receive buffer of owner q, picked with constant indices so that the
+// pointer table stays in the parameter space.
+template <typename P>
+__device__ __forceinline__ P pick_rank(P const (&tab)[kMaxRanks], int q)
+{
+    P r = tab[0];
+#pragma unroll
+    for (int i = 1; i < kMaxRanks; ++i)
+        if (q == i) r = tab[i];
+    return r;
+}
+
+// One warp per (token, chunk of 32*kEpVec 16-byte vectors), as the
+// single-GPU scatter: lanes 0..k-1 find the destination (owner, row) of the
+// token's slots, every lane loads its vectors of x once and stores them to
+// the k destinations.
+__global__ void __launch_bounds__(32 * kEpWarps) ep_dispatch_kernel(const __grid_constant__ EpDispatchParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kEpWarps + (threadIdx.x >> 5);
+    const int t = gw / p.chunks;
+    const int c = gw - t * p.chunks;
+    if (t >= p.T) return;
+    const bool ok = *p.ok != 0u;  // inconsistent counts: nothing is sent
+    int my_pos = -1, my_q = 0;
+    if (lane < p.k && ok) {
+        const size_t s = static_cast<size_t>(t) * p.k + lane;
+        const int e = p.idx[s];
+        const int r = p.rank[s];
+        if (e >= 0 && e < p.E && r >= 0) {
+            const int row = p.tilebase[static_cast<size_t>(t / kTileTokens) * p.E + e] + r;
+            const int pos = p.base[e] + (row - p.offsets[e]);
+            if (pos >= 0 && pos < p.recv_rows) {
+                my_pos = pos;
+                my_q = e / p.El;
+            }
+        }
+        if (c == 0) {
+            if (my_pos < 0) atomicOr(p.err, kErrIndex);
+            p.pos_of_slot[s] = my_pos;
+        }
+    } else if (lane < p.k && c == 0) {
+        p.pos_of_slot[static_cast<size_t>(t) * p.k + lane] = -1;
+    }
+    if (!ok) return;
+    const int nv = p.d >> 3;
+    const uint4 *src = p.x + static_cast<size_t>(t) * nv;
+    uint4 val[kEpVec];
+#pragma unroll
+    for (int u = 0; u < kEpVec; ++u) {
+        const int v = (c * kEpVec + u) * 32 + lane;
+        if (v < nv) val[u] = __ldg(src + v);
+    }
+    bool stored = false;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        const int pos = __shfl_sync(0xffffffffu, my_pos, j);
+        const int q = __shfl_sync(0xffffffffu, my_q, j);
+        if (j < p.k && pos >= 0) {
+            uint4 *dst = pick_rank(p.recv, q) + static_cast<size_t>(pos) * nv;
+#pragma unroll
+            for (int u = 0; u < kEpVec; ++u) {
+                const int v = (c * kEpVec + u) * 32 + lane;
+                if (v < nv) dst[v] = val[u];
+            }
+            stored = true;
+        }
+    }
+    // Stores to another GPU's memory are made visible system-wide before the
+    // kernel ends; the caller's collective that follows orders them before
+    // the owner's expert kernel.
+    if (stored) __threadfence_system();
+}
+
+struct EpCombineParams {
+    int T, d, E, k, El;
+    int ksplit;              // partial outputs per receive row, summed in order
+    size_t part_stride;      // 4-element vectors between partial outputs (recv_rows * d / 4)
+    int recv_rows;
+    const int32_t *idx, *pos_of_slot;
+    const float *w;
+    const float4 *y[kMaxRanks];  // every rank's output buffer [ksplit, recv_rows, d] fp32
+    const float4 *shared_y;      // [T, d] or nullptr
+    float4 *out;
+    int chunks;              // chunks of 32*kEpOutVec float4 per row
+};
+
+constexpr int kEpOutVec = 2;
+
+// One warp per (token, chunk): y_j = sum of the K-split partials of slot j's
+// row (in order), out = sum_j w_j * y_j in slot order (+ shared_y).  The
+// order of every addition is fixed.
+__global__ void __launch_bounds__(32 * kEpWarps) ep_combine_kernel(const __grid_constant__ EpCombineParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * kEpWarps + (threadIdx.x >> 5);
+    const int t = gw / p.chunks;
+    const int c = gw - t * p.chunks;
+    if (t >= p.T) return;
+    int my_pos = -1, my_q = 0;
+    float my_w = 0.0f;
+    if (lane < p.k) {
+        const size_t s = static_cast<size_t>(t) * p.k + lane;
+        const int e = p.idx[s];
+        const int pos = p.pos_of_slot[s];
+        if (e >= 0 && e < p.E && pos >= 0 && pos < p.recv_rows) {
+            my_pos = pos;
+            my_q = e / p.El;
+        }
+        my_w = p.w[s];
+    }
+    const int nv = p.d >> 2;
+    float4 acc[kEpOutVec];
+#pragma unroll
+    for (int u = 0; u < kEpOutVec; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < p.k; ++j) {
+        const int pos = __shfl_sync(0xffffffffu, my_pos, j);
+        const int q = __shfl_sync(0xffffffffu, my_q, j);
+        const float wj = __shfl_sync(0xffffffffu, my_w, j);
+        if (pos < 0) continue;
+        const float4 *row = pick_rank(p.y, q) + static_cast<size_t>(pos) * nv;
+        float4 yj[kEpOutVec];
+#pragma unroll
+        for (int u = 0; u < kEpOutVec; ++u) {
+            const int v = (c * kEpOutVec + u) * 32 + lane;
+            yj[u] = v < nv ? row[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int sp = 1; sp < p.ksplit; ++sp) {
+#pragma unroll
+            for (int u = 0; u < kEpOutVec; ++u) {
+                const int v = (c * kEpOutVec + u) * 32 + lane;
+                if (v < nv) {
+                    const float4 b = row[sp * p.part_stride + v];
+                    yj[u].x += b.x;
+                    yj[u].y += b.y;
+                    yj[u].z += b.z;
+                    yj[u].w += b.w;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kEpOutVec; ++u) {
+            acc[u].x = fmaf(wj, yj[u].x, acc[u].x);
+            acc[u].y = fmaf(wj, yj[u].y, acc[u].y);
+            acc[u].z = fmaf(wj, yj[u].z, acc[u].z);
+            acc[u].w = fmaf(wj, yj[u].w, acc[u].w);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kEpOutVec; ++u) {
+        const int v = (c * kEpOutVec + u) * 32 + lane;
+        if (v < nv) {
+            if (p.shared_y != nullptr) {
+                const float4 b = p.shared_y[static_cast<size_t>(t) * nv + v];
+                acc[u].x += b.x;
+                acc[u].y += b.y;
+                acc[u].z += b.z;
+                acc[u].w += b.w;
+            }
+            p.out[static_cast<size_t>(t) * nv + v] = acc[u];
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s)
+{
+    if (a.R < 1 || a.R > kMaxRanks || a.E % a.R != 0 || a.E > kMaxE) return cudaErrorInvalidValue;
+    PlanParams pp{};
+    pp.E = a.E;
+    pp.R = a.R;
+    pp.rank = a.rank;
+    pp.El = a.E / a.R;
+    pp.recv_rows = a.recv_rows;
+    pp.counts_all = a.counts_all;
+    pp.offsets = a.offsets;
+    pp.base = a.base;
+    pp.recv_offsets = a.recv_offsets;
+    pp.ok = a.ok;
+    pp.err = a.err;
+    ep_plan_kernel<<<1, kPlanThreads, 0, s>>>(pp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    EpDispatchParams p{};
+    p.T = a.T;
+    p.d = a.d;
+    p.E = a.E;
+    p.k = a.k;
+    p.El = pp.El;
+    p.R = a.R;
+    p.recv_rows = a.recv_rows;
+    p.x = reinterpret_cast<const uint4 *>(a.x);
+    p.idx = a.idx;
+    p.rank = a.rank_of_pair;
+    p.tilebase = a.tilebase;
+    p.offsets = a.offsets;
+    p.base = a.base;
+    p.ok = a.ok;
+    for (int r = 0; r < kMaxRanks; ++r)
+        p.recv[r] = reinterpret_cast<uint4 *>(r < a.R ? a.recv_x[r] : a.recv_x[0]);
+    p.pos_of_slot = a.pos_of_slot;
+    p.err = a.err;
+    const int nv = a.d / 8;
+    p.chunks = (nv + 32 * kEpVec - 1) / (32 * kEpVec);
+    const long long warps = static_cast<long long>(a.T) * p.chunks;
+    const int blocks = static_cast<int>((warps + kEpWarps - 1) / kEpWarps);
+    ep_dispatch_kernel<<<blocks, 32 * kEpWarps, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine(const EpCombineLaunch &a, cudaStream_t s)
+{
+    if (a.R < 1 || a.R > kMaxRanks || a.E % a.R != 0) return cudaErrorInvalidValue;
+    EpCombineParams p{};
+    p.T = a.T;
+    p.d = a.d;
+    p.E = a.E;
+    p.k = a.k;
+    p.El = a.E / a.R;
+    p.ksplit = a.ksplit < 1 ? 1 : a.ksplit;
+    p.recv_rows = a.recv_rows;
+    p.part_stride = static_cast<size_t>(a.recv_rows) * (a.d / 4);
+    p.idx = a.idx;
+    p.pos_of_slot = a.pos_of_slot;
+    p.w = a.w;
+    for (int r = 0; r < kMaxRanks; ++r)
+        p.y[r] = reinterpret_cast<const float4 *>(r < a.R ? a.recv_y[r] : a.recv_y[0]);
+    p.shared_y = reinterpret_cast<const float4 *>(a.shared_y);
+    p.out = reinterpret_cast<float4 *>(a.out);
+    const int nv = a.d / 4;
+    p.chunks = (nv + 32 * kEpOutVec - 1) / (32 * kEpOutVec);
+    const long long warps = static_cast<long long>(a.T) * p.chunks;
+    const int blocks = static_cast<int>((warps + kEpWarps - 1) / kEpWarps);
+    ep_combine_kernel<<<blocks, 32 * kEpWarps, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -607,10 +607,11 @@ int down_ksplit(int S, int E_seg, int d, int d_ff)
 
 cudaError_t launch_ffn(const FfnLaunch &a, cudaStream_t s)
 {
-    if (a.sched != nullptr && ffn_pair_eligible(a.S, a.offsets ? a.E : 1, a.ksplit))
+    const int rows = a.S_hint > 0 ? a.S_hint : a.S;
+    if (a.sched != nullptr && ffn_pair_eligible(rows, a.offsets ? a.E : 1, a.ksplit))
         return launch_ffn_pair(a, a.sched, s);
     if (a.out != nullptr || a.y_bf16) return cudaErrorInvalidValue;  // pair kernel only
-    switch (ffn_token_tile(a.S, a.offsets ? a.E : 1)) {
+    switch (ffn_token_tile(rows, a.offsets ? a.E : 1)) {
     case 32: return launch_ffn_cfg<32, 6>(a, s);
     case 64: return launch_ffn_cfg<64, 5>(a, s);
     default: return launch_ffn_cfg<128, 4>(a, s);

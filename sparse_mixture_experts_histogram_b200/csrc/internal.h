@@ -63,6 +63,8 @@ struct FfnLaunch {
     int E;                    // segments (ignored when offsets is null: one segment [0, S))
     int d, d_ff;
     int S;                    // rows of x / H / Y
+    int S_hint;               // rows expected (0: S); picks the token tile when S is only
+                              // a capacity and the segments are filled on the device
     int max_rows;             // upper bound of rows in one segment (weights streamed once if <= tile)
     int ksplit;               // K ranges of the down projection: partial outputs
                               // [ksplit, S, d] summed by the caller (the combine)
@@ -116,6 +118,39 @@ struct CombineLaunch {
     bool y_bf16;              // y holds bf16 rows [T*k, d] (ksplit 1), not fp32
     bool shared_bf16;         // shared_y holds bf16 rows [T, d]
 };
+
+// Expert parallelism (ep.cu): rank `rank` of R owns experts
+// [rank*E/R, (rank+1)*E/R), R <= 8.  recv_x / recv_y hold every rank's
+// receive and output buffer, as addresses this GPU can use (its own, or a
+// peer's mapped here).
+struct EpDispatchLaunch {
+    int T, d, E, k, R, rank;
+    int recv_rows;               // rows of each receive buffer
+    const uint16_t *x;           // [T, d] bf16
+    const int32_t *idx;          // [T, k]
+    const int32_t *counts_all;   // [R, E]
+    const int32_t *offsets, *tilebase, *rank_of_pair;  // this rank's ranks_kernel output
+    int32_t *base;               // [E] scratch
+    uint32_t *ok;                // scratch word
+    uint16_t *const *recv_x;     // [R] host array of device addresses
+    int32_t *pos_of_slot;        // [T, k] out
+    int32_t *recv_offsets;       // [E/R + 1] out
+    uint32_t *err;
+};
+
+struct EpCombineLaunch {
+    int T, d, E, k, R;
+    int recv_rows;
+    int ksplit;                  // partial outputs per receive row
+    const int32_t *idx, *pos_of_slot;
+    const float *w;
+    const float *const *recv_y;  // [R] host array of device addresses
+    const float *shared_y;       // [T, d] or nullptr
+    float *out;
+};
+
+cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s);
+cudaError_t launch_ep_combine(const EpCombineLaunch &a, cudaStream_t s);
 
 cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s);
 cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s);

@@ -53,6 +53,13 @@ MUTANTS = {
                                "for (int i = 0; i < d; ++i) b += s3[0] * e4m3_to_double(r3[i]) * xt[i];"),
     "fp8_w2_scale_by_hidden_index": ("acc += s2[o] * e4m3_to_double(r2[f]) * h[f];",
                                      "acc += s2[f % d] * e4m3_to_double(r2[f]) * h[f];"),
+    "ep_tokens_reversed": ("for (int t = 0; t < T_of[r]; ++t)\n                    for (int j = 0; j < k; ++j) {",
+                           "for (int t = T_of[r] - 1; t >= 0; --t)\n                    for (int j = 0; j < k; ++j) {"),
+    "ep_slot_major": ("for (int t = 0; t < T_of[r]; ++t)\n                    for (int j = 0; j < k; ++j) {",
+                      "for (int j = 0; j < k; ++j)\n                    for (int t = 0; t < T_of[r]; ++t) {"),
+    "ep_offsets_shifted": ("seg[e - q * El + 1] = row;", "seg[e - q * El] = row;"),
+    "ep_rows_continue_across_owners": ("int32_t row = 0;\n        int32_t *seg",
+                                       "static int32_t row = 0;\n        int32_t *seg"),
     "logits_without_bias": ("if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);",
                             "if (logits) { memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);"
                             " if (bias) for (int e = 0; e < E; ++e) logits[(size_t)t * E + e] -= bias[e]; }"),

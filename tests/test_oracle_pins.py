@@ -487,3 +487,67 @@ def test_fp8_layer_is_linear_in_the_w2_and_w3_scales():
     assert np.array_equal(oracle.forward_fp8(*args(s1, s3, 2 * s2), k=2), 2 * base)
     assert np.array_equal(oracle.forward_fp8(*args(s1, 2 * s3, s2), k=2), 2 * base)
     assert _rel(oracle.forward_fp8(*args(2 * s1, s3, s2), k=2), base) > 1e-3
+
+
+# ---------------------------------------------------------- expert parallelism
+def _ep_random_idx(rng, Ts, E, k):
+    return [np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+            if T else np.zeros((0, k), np.int32) for T in Ts]
+
+
+@pytest.mark.parametrize("R,E,k,Ts", [(1, 4, 2, [9]), (2, 4, 2, [5, 7]), (3, 9, 2, [4, 0, 6]),
+                                      (4, 8, 3, [3, 8, 1, 5]), (2, 6, 6, [4, 3])])
+def test_ep_plan_is_a_sort_by_expert_sender_token(R, E, k, Ts):
+    # A second formulation of the receive layout: collect each owner's pairs
+    # and sort them by (expert, sending rank, token); a pair's receive row is
+    # its place in that order.  Segment starts are running sums of the
+    # per-expert counts over all ranks.
+    rng = np.random.default_rng(R * 100 + E)
+    idx = _ep_random_idx(rng, Ts, E, k)
+    pos, off = oracle.ep_plan(idx, E, R)
+    El = E // R
+    for q in range(R):
+        keys = [(int(idx[r][t, j]), r, t, j) for r in range(R) for t in range(Ts[r])
+                for j in range(k) if idx[r][t, j] // El == q]
+        for place, (e, r, t, j) in enumerate(sorted(keys)):
+            assert pos[r][t, j] == place
+        cnt = sum(np.bincount(i.ravel(), minlength=E) for i in idx)[q * El:(q + 1) * El]
+        assert np.array_equal(off[q], np.concatenate([[0], np.cumsum(cnt)]))
+    assert all((p >= 0).all() for p in pos)
+
+
+def test_ep_layer_assembled_from_the_plan_is_the_layer():
+    # The split layer written with the plan (rows sent to their owner, each
+    # owner's experts applied to its segments, rows read back through pos and
+    # summed in slot order) reproduces oracle.forward on every rank's tokens.
+    R, E, k, d, dff = 3, 6, 2, 32, 24
+    Ts = [7, 3, 5]
+    wl, inp = _inputs(sum(Ts), d, E, dff, k, seed=11)
+    x = bits(inp["x"])
+    xs = np.split(x, np.cumsum(Ts)[:-1])
+    W1, W3, W2, Wg = (bits(inp[n]) for n in ("W1", "W3", "W2", "Wg"))
+    routes = [oracle.route(xr, Wg, k) for xr in xs]
+    idx = [r["idx"] for r in routes]
+    pos, off = oracle.ep_plan(idx, E, R)
+    El = E // R
+    y = []
+    for q in range(R):
+        recv = np.zeros((int(off[q][-1]), d), np.uint16)
+        for r in range(R):
+            t, j = np.nonzero(idx[r] // El == q)
+            recv[pos[r][t, j]] = xs[r][t]
+        yq = np.zeros((recv.shape[0], d))
+        for i in range(El):
+            a, b = off[q][i], off[q][i + 1]
+            if b > a:
+                e = q * El + i
+                yq[a:b] = oracle.swiglu(recv[a:b], W1[e], W3[e], W2[e])
+        y.append(yq)
+    for r in range(R):
+        out = np.zeros((Ts[r], d))
+        for j in range(k):
+            owner = idx[r][:, j] // El
+            rows = np.stack([y[owner[t]][pos[r][t, j]] for t in range(Ts[r])])
+            out += routes[r]["w"][:, j:j + 1] * rows
+        ref = oracle.forward(xs[r], Wg, W1, W3, W2, k)
+        assert _rel(out, ref) < 1e-13
