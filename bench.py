@@ -691,6 +691,140 @@ def gpu_arm(args):
     return 0
 
 
+def ep_arm(args):
+    """``--ep-emulate R``: the expert-parallel layer (experts split over R
+    ranks) with its R ranks emulated on this one GPU: the same kernels and
+    buffers as on R GPUs, the ranks one after another on one stream, stream
+    order in place of the collectives, every transfer a local store.  Prints
+    one JSON line (``"impl": "ep_emulated"``): the group's tokens/s on this
+    GPU and, per rank, the device time of its own kernels (route, dispatch,
+    its experts, combine with the rank's shared expert), which is what one
+    GPU of an R-GPU group spends in kernels; the NVLink transfers and the
+    collectives are not in it."""
+    import sparse_mixture_experts_histogram_b200 as moe
+    from sparse_mixture_experts_histogram_b200 import ep
+    wls = workload(args.workload)
+    if len(wls) != 1 or is_fp8(wls[0]):
+        raise SystemExit("--ep-emulate takes one bf16 layer")
+    wl, R = wls[0], args.ep_emulate
+    T = wl.T
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    moe.load_library()
+    inp = synth.make_inputs(dataclasses.replace(wl, T=R * T), seed=42, device=dev)
+    xs = [inp["x"][r * T:(r + 1) * T] for r in range(R)]
+    outs = [torch.empty(T, wl.d, dtype=torch.float32, device=dev) for _ in range(R)]
+    shared = (inp["Ws1"], inp["Ws3"], inp["Ws2"]) if wl.d_ff_shared else None
+    layer = ep.EmulatedExpertParallel(R, T, wl.d, wl.E, wl.d_ff, wl.k, wl.d_ff_shared, device=dev)
+    p = layer.plan
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    phases = ("route", "dispatch", "expert_ffn", "combine")
+
+    def step(mark=lambda key: None):
+        rx = [b.recv_x for b in layer.ranks]
+        ry = [b.recv_y for b in layer.ranks]
+        for r in range(R):
+            b = layer.ranks[r]
+            mark(("route", r))
+            ep._route(p, b, xs[r], inp["Wg"], inp["bias"], b.counts)
+            layer.counts_all[r].copy_(b.counts)
+        for r in range(R):
+            mark(("dispatch", r))
+            ep._dispatch(p, layer.ranks[r], r, xs[r], layer.counts_all, rx)
+        for r in range(R):
+            lo, hi = ep.expert_block(wl.E, R, r)
+            mark(("expert_ffn", r))
+            ep._ffn(p, layer.ranks[r], inp["W1"][lo:hi], inp["W3"][lo:hi], inp["W2"][lo:hi])
+        for r in range(R):
+            mark(("combine", r))
+            sy = ep._shared(p, layer.ranks[r], xs[r], shared)
+            ep._combine(p, layer.ranks[r], T, ry, sy, outs[r])
+        mark(("end", 0))
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    errs = [moe.moe_get_device_error(b.ws, stream)[1] for b in layer.ranks]
+    if any(errs):
+        raise SystemExit(f"device error words {errs}")
+    rows = [int(b.recv_offsets[-1].item()) for b in layer.ranks]
+    hit = [int((b.recv_offsets[1:] > b.recv_offsets[:-1]).sum().item()) for b in layer.ranks]
+
+    # Whole emulated step: K steps in one CUDA graph between events.
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(args.steps):
+            step()
+    sampler = ClockSampler(0)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = sampler.mark()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    t1 = sampler.mark()
+    clocks = sampler.stop(t0, t1)
+    ms = e0.elapsed_time(e1) / args.steps
+
+    # Per rank and phase: a one-step graph with an event node at every
+    # boundary, replayed K times.
+    per = {ph: [[] for _ in range(R)] for ph in phases}
+    order = [(ph, r) for ph in phases for r in range(R)] + [("end", 0)]
+    ev = {key: torch.cuda.Event(enable_timing=True, external=True) for key in order}
+    g_tr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_tr, stream=stream):
+        step(lambda key: ev[key].record(stream))
+    for _ in range(args.steps):
+        with torch.cuda.stream(stream):
+            g_tr.replay()
+        stream.synchronize()
+        for a, b in zip(order, order[1:]):
+            per[a[0]][a[1]].append(ev[a].elapsed_time(ev[b]) * 1e3)
+    med = {ph: [statistics.median(v) for v in per[ph]] for ph in phases}
+    rank_us = [sum(med[ph][r] for ph in phases) for r in range(R)]
+
+    pk, src = peaks()
+    ffn = []
+    for r in range(R):
+        flops = acc.ffn_flops(rows[r], wl.d, wl.d_ff, 1)
+        byts = 2 * 3 * hit[r] * wl.d * wl.d_ff + 2 * rows[r] * wl.d + 4 * p.ksplit * rows[r] * wl.d
+        t = med["expert_ffn"][r] * 1e-6
+        ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+        if byts and flops / byts > ridge:
+            a = flops / t / 1e12
+            ffn.append({"rows": rows[r], "experts_hit": hit[r], "bound": "tensor",
+                        "achieved": a, "unit": "TFLOP/s",
+                        "frac": a / pk["bf16_tflops_sustained"]})
+        else:
+            a = byts / t / 1e9
+            ffn.append({"rows": rows[r], "experts_hit": hit[r], "bound": "hbm", "bytes": byts,
+                        "achieved": a, "unit": "GB/s", "frac": a / pk["hbm_gbs"]})
+    line = {
+        "impl": "ep_emulated", "metric": METRIC, "value": R * T / (ms * 1e-3), "unit": UNIT,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload}_ep{R}_emulated", "ep_ranks": R,
+                   "tokens_per_rank": T, "layer": describe(wls, args.workload)["layers"][0],
+                   "recv_rows_per_rank": p.recv_rows, "down_ksplit": p.ksplit,
+                   "l2": "weights larger than L2 stream from HBM every step"
+                   if 2 * 3 * wl.E * wl.d * wl.d_ff > L2_BYTES else "may be L2-resident"},
+        "ep": {"per_rank_us": med, "rank_kernels_us_max": max(rank_us),
+               "rank_kernels_us": rank_us, "expert_ffn": ffn, "peaks": src,
+               "note": "R ranks emulated on one GPU: per-rank times are this GPU's kernel time "
+                       "for that rank's work; NVLink transfers and the three collectives per "
+                       "step are not included"},
+        "clocks": {k: v for k, v in clocks.items() if k != "samples"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -704,6 +838,8 @@ def main():
     ap.add_argument("--oracle-step-s", type=float, default=4.0,
                     help="seconds of host work per oracle step (bounded sample)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ep-emulate", type=int, default=0, metavar="R",
+                    help="time the expert-parallel layer with R ranks emulated on one GPU")
     ap.add_argument("--profile", action="store_true",
                     help="run the layers --steps times untimed and exit (for ncu captures)")
     args = ap.parse_args()
@@ -713,6 +849,8 @@ def main():
         return reference_arm(args)
     if args.profile:
         return profile_arm(args)
+    if args.ep_emulate:
+        return ep_arm(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

@@ -107,8 +107,10 @@ def _shared(p: _Plan, b: _Rank, x, shared):
     if shared is None:
         return None
     T = x.shape[0]
-    b.shared_off[0] = 0
-    b.shared_off[1] = T
+    # [0, T] as the one segment's bounds, set by a device fill (no host copy,
+    # so the call can be captured in a CUDA graph).
+    b.shared_off[0].fill_(0)
+    b.shared_off[1].fill_(T)
     Ws1, Ws3, Ws2 = shared
     B.moe_expert_ffn(T, p.d, 1, p.d_ff_shared, x, b.shared_off, Ws1, Ws3, Ws2, b.shared_y,
                      b.shared_ws)
