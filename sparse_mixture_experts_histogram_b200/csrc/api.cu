@@ -993,19 +993,6 @@ moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank, const mo
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     st = from_cuda(cudaMemsetAsync(wsb, 0, kHeaderBytes, s));
     if (st != MOE_OK) return st;
-    RanksLaunch r{};
-    r.T = T;
-    r.E = E;
-    r.k = k;
-    r.idx = idx;
-    r.offsets = reinterpret_cast<int32_t *>(wsb + L.offsets);
-    r.tilecnt = reinterpret_cast<int32_t *>(wsb + L.tilecnt);
-    r.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
-    r.rank = reinterpret_cast<int32_t *>(wsb + L.rank);
-    r.done = reinterpret_cast<uint32_t *>(wsb + 8);
-    r.err = reinterpret_cast<uint32_t *>(wsb);
-    st = from_cuda(launch_ranks(r, s));
-    if (st != MOE_OK) return st;
     EpDispatchLaunch a{};
     a.T = T;
     a.d = d;
@@ -1017,15 +1004,17 @@ moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank, const mo
     a.x = x;
     a.idx = idx;
     a.counts_all = counts_all;
-    a.offsets = r.offsets;
-    a.tilebase = r.tilebase;
-    a.rank_of_pair = r.rank;
+    a.offsets = reinterpret_cast<int32_t *>(wsb + L.offsets);
+    a.tilecnt = reinterpret_cast<int32_t *>(wsb + L.tilecnt);
+    a.tilebase = reinterpret_cast<int32_t *>(wsb + L.tilebase);
+    a.rank_of_pair = reinterpret_cast<int32_t *>(wsb + L.rank);
+    a.done = reinterpret_cast<uint32_t *>(wsb + 8);
     a.base = reinterpret_cast<int32_t *>(wsb + L.base);
     a.ok = reinterpret_cast<uint32_t *>(wsb + L.ok);
     a.recv_x = recv_x;
     a.pos_of_slot = pos_of_slot;
     a.recv_offsets = recv_offsets;
-    a.err = r.err;
+    a.err = reinterpret_cast<uint32_t *>(wsb);
     return from_cuda(launch_ep_dispatch(a, s));
 }
 

@@ -2,10 +2,12 @@
 // of E/R over R ranks (one GPU each); every (token, slot) row travels to the
 // rank that owns its expert, and the expert's output row travels back.
 //
-//  * ep_plan_kernel: from every rank's per-expert pair counts (all-gathered
-//    by the caller into counts_all[R, E]), the first receive row of each
-//    (expert, this source rank) block in its owner's buffer, and this rank's
-//    own receive segments (its experts' offsets).
+//  * ep_ranks_plan_kernel: the stable ranks of this rank's (token, slot)
+//    pairs per expert (as the single-GPU dispatch), then, in the CTA that
+//    completes the expert offsets, the plan: from every rank's per-expert
+//    pair counts (all-gathered by the caller into counts_all[R, E]) the first
+//    receive row of each (expert, this source rank) block in its owner's
+//    buffer, and this rank's own receive segments (its experts' offsets).
 //  * ep_dispatch_kernel: x[t] is stored straight into the owner's receive
 //    buffer (peer memory over NVLink when the owner is another GPU) at the
 //    block's first row + the pair's rank in token order.  The scatter of the
@@ -36,76 +38,120 @@ namespace {
 
 constexpr int kMaxRanks = 8;          // ranks of one expert-parallel group
 constexpr uint32_t kErrEpCounts = 0x40u;  // MOE_DEVERR_EP_COUNTS
-constexpr int kPlanThreads = 256;  // one thread per expert (E <= kMaxE = 256)
-static_assert(kPlanThreads >= kMaxE, "one plan thread per expert");
 
-struct PlanParams {
-    int E, R, rank, El;
+struct RanksPlanParams {
+    int T, E, k, R, rank, El;
     int recv_rows;               // rows of every rank's receive buffer
+    const int32_t *idx;          // [T, k] this rank's routing
     const int32_t *counts_all;   // [R, E]
-    const int32_t *offsets;      // [E+1] this rank's own expert segments (ranks_kernel)
+    DispatchOut dout;            // per-tile ranks and this rank's expert offsets
     int32_t *base;               // [E] out: first receive row of (expert e, this rank)
     int32_t *recv_offsets;       // [El+1] out: this rank's receive segments
     uint32_t *ok;                // out: 1 when the counts are consistent
     uint32_t *err;
 };
 
-// Exclusive prefix over the block's threads (kPlanThreads values).
-__device__ int block_excl_scan(int v, int *warp_tot)
+// The receive plan, run by the CTA that finished the expert offsets (all
+// kTileTokens threads; E <= kMaxE).  For every expert e (owner q = e / El):
+//   colsum[e] = sum_r counts_all[r, e]          (rows the owner gets for e)
+//   seg[e]    = sum of colsum over q's experts before e (e's segment start)
+//   base[e]   = seg[e] + sum_{r < rank} counts_all[r, e]
+// and this rank's own segment starts.  Checks: this rank's row of
+// counts_all equals the counts of its own idx (offs), no count is negative,
+// and no owner receives more than recv_rows rows.
+__device__ void ep_plan(const RanksPlanParams &p, const int32_t *offs, int32_t *colsum,
+                        int32_t *excl, int *bad)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    if (tid == 0) *bad = 0;
     __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    return before + incl - v;
+    for (int e = tid; e < p.E; e += kTileTokens) {
+        int c = 0;
+        bool b = false;
+        for (int r = 0; r < p.R; ++r) {
+            const int v = p.counts_all[static_cast<size_t>(r) * p.E + e];
+            b |= v < 0;
+            c += v;
+        }
+        b |= p.counts_all[static_cast<size_t>(p.rank) * p.E + e] != offs[e + 1] - offs[e];
+        colsum[e] = c;
+        if (b) atomicOr(bad, 1);
+    }
+    __syncthreads();
+    // Exclusive scan of colsum by the first warp (per-lane runs of experts).
+    if (tid < 32) {
+        const int per = (p.E + 31) >> 5;
+        const int first = lane * per;
+        int local = 0;
+        for (int i = 0; i < per; ++i)
+            if (first + i < p.E) local += colsum[first + i];
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        int run = incl - local;
+        for (int i = 0; i < per; ++i) {
+            if (first + i < p.E) {
+                excl[first + i] = run;
+                run += colsum[first + i];
+            }
+        }
+        if (lane == 31) excl[p.E] = incl;
+    }
+    __syncthreads();
+    for (int e = tid; e < p.E; e += kTileTokens) {
+        int below = 0;
+        for (int r = 0; r < p.rank; ++r) below += p.counts_all[static_cast<size_t>(r) * p.E + e];
+        p.base[e] = excl[e] - excl[(e / p.El) * p.El] + below;
+    }
+    for (int q = tid; q < p.R; q += kTileTokens)
+        if (excl[(q + 1) * p.El] - excl[q * p.El] > p.recv_rows) atomicOr(bad, 1);
+    const int q0 = p.rank * p.El;
+    for (int i = tid; i <= p.El; i += kTileTokens) p.recv_offsets[i] = excl[q0 + i] - excl[q0];
+    __syncthreads();
+    if (tid == 0) {
+        *p.ok = *bad ? 0u : 1u;
+        if (*bad) atomicOr(p.err, kErrEpCounts);
+    }
 }
 
-__global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(const __grid_constant__ PlanParams p)
+// Per 128-token tile: the expert histogram and stable ranks of idx (as the
+// single-GPU dispatch), and, in the CTA that completes the expert offsets,
+// the receive plan.
+__global__ void __launch_bounds__(kTileTokens) ep_ranks_plan_kernel(
+    const __grid_constant__ RanksPlanParams p)
 {
-    __shared__ int warp_tot[kPlanThreads / 32];
-    __shared__ int excl_s[kMaxE + 1];
-    __shared__ int bad_s;
-    const int e = threadIdx.x;
-    if (e == 0) bad_s = 0;
-    __syncthreads();
-    int colsum = 0, below = 0;
-    bool bad = false;
-    if (e < p.E) {
-        for (int r = 0; r < p.R; ++r) {
-            const int c = p.counts_all[static_cast<size_t>(r) * p.E + e];
-            if (c < 0) bad = true;
-            colsum += c;
-            if (r < p.rank) below += c;
+    __shared__ DispatchSmem ds;
+    __shared__ int32_t colsum[kMaxE];
+    __shared__ int32_t excl[kMaxE + 1];
+    __shared__ int bad;
+    ptx::grid_dep_launch();
+    const int row = threadIdx.x;
+    const int tile = blockIdx.x;
+    const int t = tile * kTileTokens + row;
+    for (int j = 0; j < kMaxK; ++j) {
+        int e = -1;
+        if (t < p.T && j < p.k) {
+            e = p.idx[static_cast<size_t>(t) * p.k + j];
+            bool b = (e < 0 || e >= p.E);
+            for (int jj = 0; jj < j; ++jj) b |= (ds.sel[row][jj] == e);  // repeated expert
+            if (b) {
+                atomicOr(p.err, kErrIndex);
+                e = -1;
+            }
         }
-        // This rank's row of counts_all must be what its own idx holds.
-        const int mine = p.counts_all[static_cast<size_t>(p.rank) * p.E + e];
-        if (mine != p.offsets[e + 1] - p.offsets[e]) bad = true;
+        ds.sel[row][j] = e;
     }
-    const int excl = block_excl_scan(e < p.E ? colsum : 0, warp_tot);
-    if (e < p.E) excl_s[e] = excl;
-    if (e == p.E - 1) excl_s[p.E] = excl + colsum;
-    if (bad) atomicOr(&bad_s, 1);
+    dispatch_tile(ds, row, tile, p.T, p.E, p.k, p.dout, 1);
+    // Only the CTA that wrote the offsets goes on (the only one when there
+    // is a single tile).
+    if (p.dout.ntiles > 1 && !ds.is_last) return;
     __syncthreads();
-    if (e < p.E) {
-        const int q0 = (e / p.El) * p.El;  // first expert of e's owner
-        p.base[e] = excl - excl_s[q0] + below;
-    }
-    // Rows each owner receives must fit its buffer.
-    if (e < p.R && excl_s[(e + 1) * p.El] - excl_s[e * p.El] > p.recv_rows) atomicOr(&bad_s, 1);
-    const int q0 = p.rank * p.El;
-    for (int i = e; i <= p.El; i += kPlanThreads) p.recv_offsets[i] = excl_s[q0 + i] - excl_s[q0];
-    __syncthreads();
-    if (e == 0) {
-        *p.ok = bad_s ? 0u : 1u;
-        if (bad_s) atomicOr(p.err, kErrEpCounts);
-    }
+    __threadfence();
+    ep_plan(p, p.dout.offsets, colsum, excl, &bad);
 }
 
 struct EpDispatchParams {
@@ -146,11 +192,22 @@ __global__ void __launch_bounds__(32 * kEpWarps) ep_dispatch_kernel(const __grid
     const int t = gw / p.chunks;
     const int c = gw - t * p.chunks;
     if (t >= p.T) return;
+    // x and idx were written before the plan kernel started, so they are
+    // read while it finishes; everything it writes is read after the wait.
+    const int nv = p.d >> 3;
+    const uint4 *src = p.x + static_cast<size_t>(t) * nv;
+    uint4 val[kEpVec];
+#pragma unroll
+    for (int u = 0; u < kEpVec; ++u) {
+        const int v = (c * kEpVec + u) * 32 + lane;
+        if (v < nv) val[u] = __ldg(src + v);
+    }
+    const size_t s = static_cast<size_t>(t) * p.k + lane;
+    const int e = lane < p.k ? p.idx[s] : -1;
+    ptx::grid_dep_wait();  // the ranks and the plan of ep_ranks_plan_kernel
     const bool ok = *p.ok != 0u;  // inconsistent counts: nothing is sent
     int my_pos = -1, my_q = 0;
     if (lane < p.k && ok) {
-        const size_t s = static_cast<size_t>(t) * p.k + lane;
-        const int e = p.idx[s];
         const int r = p.rank[s];
         if (e >= 0 && e < p.E && r >= 0) {
             const int row = p.tilebase[static_cast<size_t>(t / kTileTokens) * p.E + e] + r;
@@ -165,17 +222,9 @@ __global__ void __launch_bounds__(32 * kEpWarps) ep_dispatch_kernel(const __grid
             p.pos_of_slot[s] = my_pos;
         }
     } else if (lane < p.k && c == 0) {
-        p.pos_of_slot[static_cast<size_t>(t) * p.k + lane] = -1;
+        p.pos_of_slot[s] = -1;
     }
     if (!ok) return;
-    const int nv = p.d >> 3;
-    const uint4 *src = p.x + static_cast<size_t>(t) * nv;
-    uint4 val[kEpVec];
-#pragma unroll
-    for (int u = 0; u < kEpVec; ++u) {
-        const int v = (c * kEpVec + u) * 32 + lane;
-        if (v < nv) val[u] = __ldg(src + v);
-    }
     bool stored = false;
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
@@ -211,10 +260,13 @@ struct EpCombineParams {
 };
 
 constexpr int kEpOutVec = 2;
+constexpr int kEpBatch = 4;  // (slot, partial) rows whose loads are in flight together
 
 // One warp per (token, chunk): y_j = sum of the K-split partials of slot j's
 // row (in order), out = sum_j w_j * y_j in slot order (+ shared_y).  The
-// order of every addition is fixed.
+// (slot, partial) pairs are visited slot-major in batches of kEpBatch whose
+// loads are all issued before any is used; the order of every addition is
+// fixed.
 __global__ void __launch_bounds__(32 * kEpWarps) ep_combine_kernel(const __grid_constant__ EpCombineParams p)
 {
     const int lane = threadIdx.x & 31;
@@ -235,40 +287,75 @@ __global__ void __launch_bounds__(32 * kEpWarps) ep_combine_kernel(const __grid_
         my_w = p.w[s];
     }
     const int nv = p.d >> 2;
-    float4 acc[kEpOutVec];
+    const int npairs = p.k * p.ksplit;
+    float4 acc[kEpOutVec], yj[kEpOutVec];
 #pragma unroll
-    for (int u = 0; u < kEpOutVec; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < p.k; ++j) {
-        const int pos = __shfl_sync(0xffffffffu, my_pos, j);
-        const int q = __shfl_sync(0xffffffffu, my_q, j);
-        const float wj = __shfl_sync(0xffffffffu, my_w, j);
-        if (pos < 0) continue;
-        const float4 *row = pick_rank(p.y, q) + static_cast<size_t>(pos) * nv;
-        float4 yj[kEpOutVec];
+    for (int u = 0; u < kEpOutVec; ++u) {
+        acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        yj[u] = acc[u];
+    }
+    // (j0, sp0): slot and partial of the batch's first pair, advanced
+    // without divisions.
+    int j0 = 0, sp0 = 0;
+    for (int p0 = 0; p0 < npairs; p0 += kEpBatch) {
+        float4 val[kEpBatch][kEpOutVec];
+        int jj[kEpBatch], ss[kEpBatch];
+        {
+            int j = j0, sp = sp0;
 #pragma unroll
-        for (int u = 0; u < kEpOutVec; ++u) {
-            const int v = (c * kEpOutVec + u) * 32 + lane;
-            yj[u] = v < nv ? row[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < kEpBatch; ++i) {
+                jj[i] = j;
+                ss[i] = sp;
+                if (++sp == p.ksplit) {
+                    sp = 0;
+                    ++j;
+                }
+            }
+            j0 = j;
+            sp0 = sp;
         }
-        for (int sp = 1; sp < p.ksplit; ++sp) {
+#pragma unroll
+        for (int i = 0; i < kEpBatch; ++i) {
+            const int pi = p0 + i;
+            const int pos = __shfl_sync(0xffffffffu, my_pos, jj[i] & 31);
+            const int q = __shfl_sync(0xffffffffu, my_q, jj[i] & 31);
+            const bool ok = pi < npairs && pos >= 0;
+            const float4 *row = pick_rank(p.y, q) + ss[i] * p.part_stride +
+                                static_cast<size_t>(ok ? pos : 0) * nv;
 #pragma unroll
             for (int u = 0; u < kEpOutVec; ++u) {
                 const int v = (c * kEpOutVec + u) * 32 + lane;
-                if (v < nv) {
-                    const float4 b = row[sp * p.part_stride + v];
-                    yj[u].x += b.x;
-                    yj[u].y += b.y;
-                    yj[u].z += b.z;
-                    yj[u].w += b.w;
-                }
+                val[i][u] = (ok && v < nv) ? __ldg(row + v) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kEpOutVec; ++u) {
-            acc[u].x = fmaf(wj, yj[u].x, acc[u].x);
-            acc[u].y = fmaf(wj, yj[u].y, acc[u].y);
-            acc[u].z = fmaf(wj, yj[u].z, acc[u].z);
-            acc[u].w = fmaf(wj, yj[u].w, acc[u].w);
+        for (int i = 0; i < kEpBatch; ++i) {
+            const int pi = p0 + i;
+            if (pi < npairs) {
+                const int j = jj[i];
+                const int sp = ss[i];
+#pragma unroll
+                for (int u = 0; u < kEpOutVec; ++u) {
+                    if (sp == 0) {
+                        yj[u] = val[i][u];
+                    } else {
+                        yj[u].x += val[i][u].x;
+                        yj[u].y += val[i][u].y;
+                        yj[u].z += val[i][u].z;
+                        yj[u].w += val[i][u].w;
+                    }
+                }
+                if (sp == p.ksplit - 1) {
+                    const float wj = __shfl_sync(0xffffffffu, my_w, j & 31);
+#pragma unroll
+                    for (int u = 0; u < kEpOutVec; ++u) {
+                        acc[u].x = fmaf(wj, yj[u].x, acc[u].x);
+                        acc[u].y = fmaf(wj, yj[u].y, acc[u].y);
+                        acc[u].z = fmaf(wj, yj[u].z, acc[u].z);
+                        acc[u].w = fmaf(wj, yj[u].w, acc[u].w);
+                    }
+                }
+            }
         }
     }
 #pragma unroll
@@ -292,19 +379,29 @@ __global__ void __launch_bounds__(32 * kEpWarps) ep_combine_kernel(const __grid_
 cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s)
 {
     if (a.R < 1 || a.R > kMaxRanks || a.E % a.R != 0 || a.E > kMaxE) return cudaErrorInvalidValue;
-    PlanParams pp{};
+    RanksPlanParams pp{};
+    pp.T = a.T;
     pp.E = a.E;
+    pp.k = a.k;
     pp.R = a.R;
     pp.rank = a.rank;
     pp.El = a.E / a.R;
     pp.recv_rows = a.recv_rows;
+    pp.idx = a.idx;
     pp.counts_all = a.counts_all;
-    pp.offsets = a.offsets;
+    pp.dout.tilecnt = a.tilecnt;
+    pp.dout.tilebase = a.tilebase;
+    pp.dout.rank = a.rank_of_pair;
+    pp.dout.offsets = a.offsets;
+    pp.dout.counts = nullptr;
+    pp.dout.done = a.done;
+    pp.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
+    pp.dout.cap = -1;
     pp.base = a.base;
     pp.recv_offsets = a.recv_offsets;
     pp.ok = a.ok;
     pp.err = a.err;
-    ep_plan_kernel<<<1, kPlanThreads, 0, s>>>(pp);
+    ep_ranks_plan_kernel<<<pp.dout.ntiles, kTileTokens, 0, s>>>(pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -331,8 +428,7 @@ cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s)
     p.chunks = (nv + 32 * kEpVec - 1) / (32 * kEpVec);
     const long long warps = static_cast<long long>(a.T) * p.chunks;
     const int blocks = static_cast<int>((warps + kEpWarps - 1) / kEpWarps);
-    ep_dispatch_kernel<<<blocks, 32 * kEpWarps, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(ep_dispatch_kernel, dim3(blocks), dim3(32 * kEpWarps), 0, s, true, p);
 }
 
 cudaError_t launch_ep_combine(const EpCombineLaunch &a, cudaStream_t s)

@@ -129,7 +129,10 @@ struct EpDispatchLaunch {
     const uint16_t *x;           // [T, d] bf16
     const int32_t *idx;          // [T, k]
     const int32_t *counts_all;   // [R, E]
-    const int32_t *offsets, *tilebase, *rank_of_pair;  // this rank's ranks_kernel output
+    int32_t *offsets;            // [E+1] scratch: this rank's expert segments
+    int32_t *tilecnt, *tilebase; // [ntiles, E] scratch
+    int32_t *rank_of_pair;       // [T, k] scratch
+    uint32_t *done;              // tile counter, zero before the first launch (left zero)
     int32_t *base;               // [E] scratch
     uint32_t *ok;                // scratch word
     uint16_t *const *recv_x;     // [R] host array of device addresses
