@@ -169,29 +169,40 @@ class EmulatedExpertParallel:
         return [B.moe_get_device_error(b.ws)[1] for b in self.ranks]
 
 
-def peer_addresses(rank, entries, local, open_handle):
+def peer_addresses(rank, entries, local, open_handle, opened=None):
     """Addresses of every rank's buffers as this process sees them.
 
     ``entries[r]`` is rank r's ``(handle, offset)`` of one buffer (gathered
-    from all ranks in rank order); ``local`` this rank's own address.  Peers'
-    handles are opened with ``open_handle`` (a base address is returned and
-    the sender's offset added); this rank's own entry is never opened.
-    Returns (addresses in rank order, opened bases to close later)."""
-    addrs, opened = [], []
+    from all ranks in rank order); ``local`` this rank's own address.  A
+    peer's handle is opened with ``open_handle`` (which returns the base
+    address of the allocation holding the buffer) and the sender's offset is
+    added; this rank's own entry is never opened.  ``opened`` maps handles
+    already opened in this process to their bases: an allocation is mapped
+    once however many buffers it holds (CUDA maps a handle once per
+    process).  Returns (addresses in rank order, the handle -> base map)."""
+    opened = {} if opened is None else opened
+    addrs = []
     for r, (handle, offset) in enumerate(entries):
         if r == rank:
             addrs.append(int(local))
         else:
-            base = open_handle(handle)
-            opened.append(base)
-            addrs.append(int(base) + int(offset))
+            if handle not in opened:
+                opened[handle] = int(open_handle(handle))
+            addrs.append(opened[handle] + int(offset))
     return addrs, opened
 
 
 class ExpertParallelLayer:
-    """One rank of an expert-parallel layer (torch.distributed, NCCL, one
-    process per GPU on one node).  Holds this rank's expert block
-    W1/W3/W2[E/R, ...] and the replicated router (and shared expert)."""
+    """One rank of an expert-parallel layer (torch.distributed, one process
+    per GPU on one node).  Holds this rank's expert block W1/W3/W2[E/R, ...]
+    and the replicated router (and shared expert).
+
+    With an NCCL group the collectives are stream-ordered: nothing waits on
+    the host and a step can be captured in a CUDA graph.  With any other
+    backend (gloo) the same steps are ordered on the host instead: the
+    counts go through host memory and each barrier first waits for this
+    process's stream.  That form is slower; it serves hosts without NCCL
+    and processes that share one GPU."""
 
     def __init__(self, T_max, d, E, d_ff, k, Wg, W1_local, W3_local, W2_local, group=None,
                  router_bias=None, shared=None):
@@ -210,6 +221,7 @@ class ExpertParallelLayer:
         self.router_bias, self.shared = router_bias, shared
         self.counts_all = torch.empty(R, E, dtype=torch.int32, device=device)
         self.flag = torch.zeros(1, dtype=torch.int32, device=device)
+        self.host_ordered = dist.get_backend(group) != "nccl"
         self._opened = []
         if R == 1:
             self.recv_x_all, self.recv_y_all = [self.buf.recv_x], [self.buf.recv_y]
@@ -217,21 +229,39 @@ class ExpertParallelLayer:
         mine = (B.moe_ipc_get_handle(self.buf.recv_x), B.moe_ipc_get_handle(self.buf.recv_y))
         gathered = [None] * R
         dist.all_gather_object(gathered, mine, group=group)
-        self.recv_x_all, ox = peer_addresses(self.rank, [g[0] for g in gathered],
-                                             self.buf.recv_x.data_ptr(), B.moe_ipc_open_handle)
-        self.recv_y_all, oy = peer_addresses(self.rank, [g[1] for g in gathered],
-                                             self.buf.recv_y.data_ptr(), B.moe_ipc_open_handle)
-        self._opened = ox + oy
+        opened = {}
+        self.recv_x_all, _ = peer_addresses(self.rank, [g[0] for g in gathered],
+                                            self.buf.recv_x.data_ptr(), B.moe_ipc_open_handle,
+                                            opened)
+        self.recv_y_all, _ = peer_addresses(self.rank, [g[1] for g in gathered],
+                                            self.buf.recv_y.data_ptr(), B.moe_ipc_open_handle,
+                                            opened)
+        self._opened = list(opened.values())
+
+    def _gather_counts(self):
+        b = self.buf
+        if self.host_ordered:
+            host = torch.empty(self.counts_all.numel(), dtype=torch.int32)
+            self.dist.all_gather_into_tensor(host, b.counts.cpu(), group=self.group)
+            self.counts_all.copy_(host.view_as(self.counts_all))
+        else:
+            self.dist.all_gather_into_tensor(self.counts_all.view(-1), b.counts, group=self.group)
 
     def _barrier(self):
-        # One-word all-reduce on the current stream: returns on no rank before
-        # every rank's stream reached it.
-        self.dist.all_reduce(self.flag, group=self.group)
+        if self.host_ordered:
+            # This process's kernels (and their stores into peers) are done
+            # before the host barrier lets any rank go on.
+            torch.cuda.current_stream().synchronize()
+            self.dist.barrier(group=self.group)
+        else:
+            # One-word all-reduce on the current stream: returns on no rank
+            # before every rank's stream reached it.
+            self.dist.all_reduce(self.flag, group=self.group)
 
     def forward(self, x, out):
         p, b = self.plan, self.buf
         _route(p, b, x, self.Wg, self.router_bias, b.counts)
-        self.dist.all_gather_into_tensor(self.counts_all, b.counts, group=self.group)
+        self._gather_counts()
         _dispatch(p, b, self.rank, x, self.counts_all, self.recv_x_all)
         self._barrier()
         _ffn(p, b, self.W1, self.W3, self.W2)

@@ -94,8 +94,13 @@ def test_peer_addresses_open_only_the_peers():
     entries = [(b"h0", 16), (b"h1", 0), (b"h2", 256)]
     addrs, bases = ep.peer_addresses(1, entries, 0xABC, fake_open)
     assert addrs == [1016, 0xABC, 3256]
-    assert bases == [1000, 3000]
+    assert bases == {b"h0": 1000, b"h2": 3000}
     assert opened == [b"h0", b"h2"]     # this rank's own handle is never opened
+    # A second buffer in the same allocations reuses the mappings.
+    addrs2, bases2 = ep.peer_addresses(1, [(b"h0", 64), (b"h1", 8), (b"h2", 512)], 0xDEF,
+                                       fake_open, bases)
+    assert addrs2 == [1064, 0xDEF, 3512]
+    assert opened == [b"h0", b"h2"] and bases2 is bases
 
 
 def _free_port():
@@ -118,9 +123,10 @@ def _worker(rank, world, port, q):
         gathered = [None] * world
         dist.all_gather_object(gathered, mine)
         base_of = lambda h: 1_000_000 * (h[0] + 1)
-        xs, ox = ep.peer_addresses(rank, [g[0] for g in gathered], 7 + rank, base_of)
-        ys, oy = ep.peer_addresses(rank, [g[1] for g in gathered], 70 + rank, base_of)
-        q.put((rank, xs, ys, len(ox + oy)))
+        opened = {}
+        xs, _ = ep.peer_addresses(rank, [g[0] for g in gathered], 7 + rank, base_of, opened)
+        ys, _ = ep.peer_addresses(rank, [g[1] for g in gathered], 70 + rank, base_of, opened)
+        q.put((rank, xs, ys, len(opened)))
     finally:
         dist.destroy_process_group()
 

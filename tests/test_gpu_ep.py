@@ -236,3 +236,85 @@ def test_ep_layer_over_nccl_with_one_rank(tmp_path):
                          shared=(bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"])),
                          forced=got["idx"])
     assert_close(got["out"].astype(np.float64), ref, "EP over NCCL, one rank")
+
+
+_TWO_PROCS = r'''
+import datetime, os, sys
+import numpy as np, torch, torch.distributed as dist
+sys.path.insert(0, os.environ["REPO"])
+from sparse_mixture_experts_histogram_b200 import ep, synth
+from sparse_mixture_experts_histogram_b200.synth import Workload
+rank, R = int(os.environ["RANK"]), 2
+torch.cuda.set_device(0)
+dist.init_process_group("gloo", init_method="tcp://127.0.0.1:" + os.environ["PORT"], rank=rank,
+                        world_size=R, timeout=datetime.timedelta(seconds=60))
+try:
+    Ts = [150, 97]
+    wl = Workload("ep_ipc", sum(Ts), 512, 8, 512, 2, d_ff_shared=256)
+    inp = {k: (None if v is None else v.cuda()) for k, v in synth.make_inputs(wl, seed=9).items()}
+    lo, hi = ep.expert_block(8, R, rank)
+    x = inp["x"][sum(Ts[:rank]):sum(Ts[:rank + 1])]
+    layer = ep.ExpertParallelLayer(160, 512, 8, 512, 2, inp["Wg"], inp["W1"][lo:hi],
+                                   inp["W3"][lo:hi], inp["W2"][lo:hi],
+                                   shared=(inp["Ws1"], inp["Ws3"], inp["Ws2"]))
+    assert layer.host_ordered and len(layer._opened) >= 1
+    out = torch.empty(x.shape[0], 512, device="cuda")
+    for _ in range(3):
+        layer.forward(x, out)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    n = x.shape[0]
+    np.savez(os.environ["OUT"] + f".{rank}.npz", out=out.cpu().numpy(),
+             idx=layer.buf.idx[:n].cpu().numpy(), pos=layer.buf.pos[:n].cpu().numpy(),
+             seg=layer.buf.recv_offsets.cpu().numpy())
+    layer.close()
+finally:
+    dist.destroy_process_group()
+'''
+
+
+def test_ep_layer_two_processes_one_gpu_over_ipc(tmp_path):
+    """Two processes on one GPU, each one rank of the split layer: the peer
+    buffers are mapped across the processes with CUDA IPC (moe_ipc_*), the
+    dispatch stores into the other process's receive buffer and the combine
+    reads the other's output buffer; a gloo group orders the steps on the
+    host (no kernel waits on the other process).  Layout against the
+    oracle's plan, outputs against the oracle layer."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    base = str(tmp_path / "ep_ipc")
+    procs = [subprocess.Popen([sys.executable, "-c", _TWO_PROCS], stdout=subprocess.PIPE,
+                              stderr=subprocess.PIPE, text=True,
+                              env=dict(os.environ, REPO=root, PORT=str(port), OUT=base,
+                                       RANK=str(r)))
+             for r in range(2)]
+    errs = []
+    for p in procs:
+        try:
+            _, err = p.communicate(timeout=300)
+        except subprocess.TimeoutExpired:
+            p.kill()
+            _, err = p.communicate()
+        errs.append((p.returncode, err[-3000:]))
+    assert all(rc == 0 for rc, _ in errs), errs
+    got = [np.load(f"{base}.{r}.npz") for r in range(2)]
+    pos_ref, seg_ref = oracle.ep_plan([g["idx"] for g in got], 8, 2)
+    for r in range(2):
+        assert np.array_equal(got[r]["pos"], pos_ref[r])
+        assert np.array_equal(got[r]["seg"], seg_ref[r])
+    Ts = [150, 97]
+    wl = Workload("ep_ipc", sum(Ts), 512, 8, 512, 2, d_ff_shared=256)
+    inp = synth.make_inputs(wl, seed=9)
+    shared = (bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"]))
+    for r in range(2):
+        x = inp["x"][sum(Ts[:r]):sum(Ts[:r + 1])]
+        ref = oracle.forward(bits(x), bits(inp["Wg"]), bits(inp["W1"]), bits(inp["W3"]),
+                             bits(inp["W2"]), 2, shared=shared, forced=got[r]["idx"])
+        assert_close(got[r]["out"].astype(np.float64), ref, f"rank {r} over IPC")
