@@ -7,6 +7,9 @@ package, and this package imports nothing from the product.
 from .oracle import (  # noqa: F401
     ACT_SIGMOID,
     ACT_SILU,
+    ENTROPY_TAU,
+    ENTROPY_THRESHOLD,
+    W_ENTROPY,
     W_SIGMOID,
     W_SOFTMAX_ALL,
     W_SOFTMAX_TOPK,

@@ -140,10 +140,35 @@ static void swiglu_one(int d, int dff, const uint16_t *W1, const uint16_t *W3,
  *             (bjdmk.com.cn), Router.forward: softmax, then top-k of the
  *             probabilities)
  *   w_mode 2: the logistic sigmoid of each selected logit ("万亿 MoE"
- *             (m.xxqk.cn) forward listing: w = 1 / (1 + exp(-logit))) */
+ *             (m.xxqk.cn) forward listing: w = 1 / (1 + exp(-logit)))
+ *   w_mode 3: entropy-controlled k ("Mixtral 8x7B模型架构解析", routing-
+ *             strategy section, entropy_aware_routing): p = softmax(l / tau)
+ *             over all E logits with tau = 0.1, its entropy
+ *             H = -sum_e p_e ln p_e (a term with p_e = 0 counts 0); the token
+ *             keeps k experts when H > 0.8 and k - 1 otherwise (the listing's
+ *             3 and 2 for k = 3), weighted by their p, not renormalised.
+ * *k_used gets the number of slots the token uses (k except in w_mode 3);
+ * slots from *k_used on are unused. */
+#define ENTROPY_TAU 0.1
+#define ENTROPY_THRESHOLD 0.8
+
 static void variant_weights(int E, int k, const double *l, const int32_t *sel, int w_mode,
-                            double *w)
+                            double *w, int *k_used)
 {
+    *k_used = k;
+    if (w_mode == 3) {
+        double m = l[0], s = 0.0, H = 0.0;
+        for (int e = 1; e < E; ++e)
+            if (l[e] > m) m = l[e];
+        for (int e = 0; e < E; ++e) s += exp((l[e] - m) / ENTROPY_TAU);
+        for (int e = 0; e < E; ++e) {
+            double pe = exp((l[e] - m) / ENTROPY_TAU) / s;
+            if (pe > 0.0) H -= pe * log(pe);
+        }
+        *k_used = H > ENTROPY_THRESHOLD ? k : k - 1;
+        for (int j = 0; j < k; ++j) w[j] = exp((l[sel[j]] - m) / ENTROPY_TAU) / s;
+        return;
+    }
     if (w_mode == 1) {
         double m = l[0], s = 0.0;
         for (int e = 1; e < E; ++e)
@@ -188,7 +213,7 @@ int oracle_route_v(int T, int d, int E, int k, const uint16_t *x, const uint16_t
                    const double *bias, int w_mode, int32_t *idx, double *w, double *gap,
                    double *logits, int64_t *counts)
 {
-    if (w_mode < 0 || w_mode > 2) return -1;
+    if (w_mode < 0 || w_mode > 3 || (w_mode == 3 && k < 2)) return -1;
     if (T < 0 || d < 1 || E < 1 || k < 1 || k > E || !x || !Wg || !idx || !w) return -1;
     int err = 0;
 #pragma omp parallel
@@ -205,8 +230,14 @@ int oracle_route_v(int T, int d, int E, int k, const uint16_t *x, const uint16_t
                 for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)t * d + i]);
                 route_one(d, E, k, xt, Wg, bias, l, idx + (size_t)t * k, w + (size_t)t * k,
                           gap ? gap + t : NULL, taken);
-                if (w_mode)
-                    variant_weights(E, k, l, idx + (size_t)t * k, w_mode, w + (size_t)t * k);
+                if (w_mode) {
+                    int ku;
+                    variant_weights(E, k, l, idx + (size_t)t * k, w_mode, w + (size_t)t * k, &ku);
+                    for (int j = ku; j < k; ++j) {  /* unused slots */
+                        idx[(size_t)t * k + j] = -1;
+                        w[(size_t)t * k + j] = 0.0;
+                    }
+                }
                 if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);
             }
         }
@@ -217,7 +248,8 @@ int oracle_route_v(int T, int d, int E, int k, const uint16_t *x, const uint16_t
     if (err) return -1;
     if (counts) {
         for (int e = 0; e < E; ++e) counts[e] = 0;
-        for (size_t s = 0; s < (size_t)T * k; ++s) counts[idx[s]] += 1;
+        for (size_t s = 0; s < (size_t)T * k; ++s)
+            if (idx[s] >= 0) counts[idx[s]] += 1;
     }
     return 0;
 }
@@ -272,13 +304,18 @@ int oracle_forward_v(int n, const int32_t *tokens, int T, int d, int E, int dff,
     if (n < 0 || T < 1 || d < 1 || E < 1 || dff < 1 || k < 1 || k > E) return -1;
     if (!x || !Wg || !W1 || !W3 || !W2 || !out) return -1;
     if (dffs < 0 || (dffs > 0 && (!Ws1 || !Ws3 || !Ws2))) return -1;
-    if (w_mode < 0 || w_mode > 2 || act_mode < 0 || act_mode > 1) return -1;
+    if (w_mode < 0 || w_mode > 3 || act_mode < 0 || act_mode > 1) return -1;
+    if (w_mode == 3 && (k < 2 || cap >= 0)) return -1;
     for (int r = 0; r < n; ++r) {
         int t = tokens ? tokens[r] : r;
         if (t < 0 || t >= T) return -1;
+        /* In w_mode 3 a forced set may end in one unused slot (-1). */
         if (forced)
-            for (int j = 0; j < k; ++j)
-                if (forced[(size_t)r * k + j] < 0 || forced[(size_t)r * k + j] >= E) return -1;
+            for (int j = 0; j < k; ++j) {
+                int e = forced[(size_t)r * k + j];
+                int unused_ok = w_mode == 3 && j == k - 1 && e == -1;
+                if ((e < 0 || e >= E) && !unused_ok) return -1;
+            }
     }
     /* Capacity: which (token, slot) pairs are kept. */
     unsigned char *keep = NULL;
@@ -334,23 +371,35 @@ int oracle_forward_v(int n, const int32_t *tokens, int T, int d, int E, int dff,
                 int t = tokens ? tokens[r] : r;
                 for (int i = 0; i < d; ++i) xt[i] = bf16_bits_to_double(x[(size_t)t * d + i]);
                 route_one(d, E, k, xt, Wg, bias, l, sel, w, NULL, taken);
-                if (forced) {
-                    /* softmax over the forced experts' logits, in forced order */
-                    double m = -INFINITY, s = 0.0;
-                    for (int j = 0; j < k; ++j) {
-                        sel[j] = forced[(size_t)r * k + j];
-                        if (l[sel[j]] > m) m = l[sel[j]];
+                int ku = k;
+                if (forced && w_mode == 3) {
+                    /* the forced experts (an unused last slot allowed) with
+                     * their tempered probabilities */
+                    for (int j = 0; j < k; ++j) sel[j] = forced[(size_t)r * k + j];
+                    int ku_own;
+                    int32_t e_last = sel[k - 1];
+                    if (e_last < 0) sel[k - 1] = sel[0];  /* any valid index; not used */
+                    variant_weights(E, k, l, sel, w_mode, w, &ku_own);
+                    ku = e_last < 0 ? k - 1 : k;
+                } else {
+                    if (forced) {
+                        /* softmax over the forced experts' logits, in forced order */
+                        double m = -INFINITY, s = 0.0;
+                        for (int j = 0; j < k; ++j) {
+                            sel[j] = forced[(size_t)r * k + j];
+                            if (l[sel[j]] > m) m = l[sel[j]];
+                        }
+                        for (int j = 0; j < k; ++j) {
+                            w[j] = exp(l[sel[j]] - m);
+                            s += w[j];
+                        }
+                        for (int j = 0; j < k; ++j) w[j] /= s;
                     }
-                    for (int j = 0; j < k; ++j) {
-                        w[j] = exp(l[sel[j]] - m);
-                        s += w[j];
-                    }
-                    for (int j = 0; j < k; ++j) w[j] /= s;
+                    if (w_mode) variant_weights(E, k, l, sel, w_mode, w, &ku);
                 }
-                if (w_mode) variant_weights(E, k, l, sel, w_mode, w);
                 double *o = out + (size_t)r * d;
                 for (int i = 0; i < d; ++i) o[i] = 0.0;
-                for (int j = 0; j < k; ++j) {
+                for (int j = 0; j < ku; ++j) {
                     if (keep && !keep[(size_t)t * k + j]) continue;
                     int e = sel[j];
                     expert_one(d, dff, W1 + (size_t)e * dff * d, W3 + (size_t)e * dff * d,

@@ -86,8 +86,13 @@ def num_threads() -> int:
 #: Gate-weight rules: the method's softmax over the k selected logits, the
 #: softmax over all E logits without renormalisation ("Mixtral 8x7B模型架构解析"
 #: Router.forward), the sigmoid of each selected logit ("万亿 MoE" forward
-#: listing).
-W_SOFTMAX_TOPK, W_SOFTMAX_ALL, W_SIGMOID = 0, 1, 2
+#: listing), and the entropy-controlled k of "Mixtral 8x7B模型架构解析"
+#: (entropy_aware_routing: weights softmax(l / 0.1) over all experts, k kept
+#: when its entropy exceeds 0.8 nats, k - 1 otherwise; unused slots hold
+#: expert -1 and weight 0).
+W_SOFTMAX_TOPK, W_SOFTMAX_ALL, W_SIGMOID, W_ENTROPY = 0, 1, 2, 3
+#: The listing's temperature and entropy threshold.
+ENTROPY_TAU, ENTROPY_THRESHOLD = 0.1, 0.8
 #: Expert activations: SwiGLU silu(W1 x) * W3 x, and the "万亿 MoE" listing's
 #: sigmoid gate sigmoid(W1 x) * W3 x.
 ACT_SILU, ACT_SIGMOID = 0, 1
@@ -104,7 +109,8 @@ def route(x, Wg, k: int, bias=None, w_mode: int = W_SOFTMAX_TOPK):
     """Router of every token.  Returns dict with ``idx`` [T,k] int32, ``w``
     [T,k] f64, ``gap`` [T] f64 (k-th minus (k+1)-th logit, inf if k == E),
     ``logits`` [T,E] f64 and ``counts`` [E] int64.  ``w_mode`` picks the
-    gate-weight rule (the selected set does not depend on it)."""
+    gate-weight rule (the selected set does not depend on it, except that
+    W_ENTROPY may leave the last slot unused: expert -1, weight 0)."""
     x, Wg = _bits(x), _bits(Wg)
     T, d = x.shape
     E = Wg.shape[0]

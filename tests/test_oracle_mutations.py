@@ -60,6 +60,12 @@ MUTANTS = {
     "ep_offsets_shifted": ("seg[e - q * El + 1] = row;", "seg[e - q * El] = row;"),
     "ep_rows_continue_across_owners": ("int32_t row = 0;\n        int32_t *seg",
                                        "static int32_t row = 0;\n        int32_t *seg"),
+    "entropy_threshold_flipped": ("*k_used = H > ENTROPY_THRESHOLD ? k : k - 1;",
+                                  "*k_used = H > ENTROPY_THRESHOLD ? k - 1 : k;"),
+    "entropy_without_temperature": ("#define ENTROPY_TAU 0.1", "#define ENTROPY_TAU 1.0"),
+    "entropy_weights_unnormalised": ("for (int j = 0; j < k; ++j) w[j] = exp((l[sel[j]] - m) / ENTROPY_TAU) / s;",
+                                     "for (int j = 0; j < k; ++j) w[j] = exp((l[sel[j]] - m) / ENTROPY_TAU);"),
+    "entropy_in_bits": ("if (pe > 0.0) H -= pe * log(pe);", "if (pe > 0.0) H -= pe * log2(pe);"),
     "logits_without_bias": ("if (logits) memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);",
                             "if (logits) { memcpy(logits + (size_t)t * E, l, sizeof(double) * (size_t)E);"
                             " if (bias) for (int e = 0; e < E; ++e) logits[(size_t)t * E + e] -= bias[e]; }"),

@@ -402,6 +402,90 @@ def test_listing_layer_sigmoid_weights_and_sigmoid_gate():
     assert _rel(out, Y) < 1e-12
 
 
+def _entropy_route_torch(L, k):
+    """The "Mixtral 8x7B模型架构解析" entropy_aware_routing listing per token,
+    in torch fp64: probs = softmax(L / 0.1), entropy -sum p ln p (0 ln 0 = 0),
+    k where the entropy exceeds 0.8, else k - 1; the experts are the top of
+    probs (lower index first on equal values), weighted by their probs."""
+    L = torch.as_tensor(L, dtype=torch.float64)
+    P = torch.softmax(L / 0.1, dim=-1)
+    H = -torch.where(P > 0, P * torch.log(P), torch.zeros_like(P)).sum(-1)
+    kt = torch.where(H > 0.8, k, k - 1)
+    T, E = L.shape
+    idx = np.full((T, k), -1, np.int64)
+    w = np.zeros((T, k))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -P[t].numpy()))[:int(kt[t])]
+        idx[t, :len(order)] = order
+        w[t, :len(order)] = P[t].numpy()[order]
+    return idx, w, H.numpy(), kt.numpy()
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.05])
+@pytest.mark.parametrize("E,k", [(8, 3), (6, 2), (16, 4)])
+def test_entropy_controlled_k_is_the_listing(E, k, scale):
+    # Logits of the usual size (entropy mostly low: k - 1 experts) and ten
+    # times smaller ones (flat softmax: k experts), with a router bias.
+    wl, inp = _inputs(T=64, d=32, E=E, dff=8, k=k, seed=E + k)
+    Wg = (inp["Wg"].float() * scale).to(torch.bfloat16)
+    bias = np.linspace(-0.02, 0.03, E)
+    r = oracle.route(bits(inp["x"]), bits(Wg), k=k, bias=bias, w_mode=oracle.W_ENTROPY)
+    L = (_f64(inp["x"]) @ _f64(Wg).T + torch.from_numpy(bias)[None, :]).numpy()
+    idx, w, H, kt = _entropy_route_torch(L, k)
+    far = np.abs(H - 0.8) > 1e-9
+    assert np.array_equal(r["idx"][far], idx[far])
+    assert np.allclose(r["w"][far], w[far], rtol=1e-12, atol=1e-300)
+    assert np.array_equal(r["counts"], np.bincount(r["idx"][r["idx"] >= 0], minlength=E))
+    assert (r["w"][:, :k - 1] > 0).all()
+    if scale == 1.0:
+        assert (kt == k - 1).mean() > 0.5          # peaked softmax: mostly k - 1
+    else:
+        assert (kt == k).mean() > 0.5              # flat softmax: mostly k
+
+
+def test_entropy_controlled_k_closed_forms():
+    # Equal logits: p = 1/E and H = ln E, so E >= 3 keeps k experts (ln 3 >
+    # 0.8) with weights 1/E each; E = 2 (ln 2 < 0.8) keeps k - 1 = 1.
+    wl, inp = _inputs(T=5, d=16, E=5, dff=8, k=3)
+    r = oracle.route(bits(inp["x"]), bits(torch.zeros_like(inp["Wg"])), k=3,
+                     w_mode=oracle.W_ENTROPY)
+    assert (r["idx"] == np.arange(3)).all() and np.allclose(r["w"], 0.2, rtol=1e-15)
+    wl, inp = _inputs(T=5, d=16, E=2, dff=8, k=2)
+    r = oracle.route(bits(inp["x"]), bits(torch.zeros_like(inp["Wg"])), k=2,
+                     w_mode=oracle.W_ENTROPY)
+    assert (r["idx"][:, 0] == 0).all() and (r["idx"][:, 1] == -1).all()
+    assert np.allclose(r["w"][:, 0], 0.5, rtol=1e-15) and (r["w"][:, 1] == 0).all()
+    # One dominant logit (bias 5 on expert 3): H ~ 0, one expert fewer.
+    wl, inp = _inputs(T=6, d=16, E=4, dff=8, k=2)
+    bias = np.array([0.0, 0.0, 0.0, 5.0])
+    r = oracle.route(bits(inp["x"]), bits(torch.zeros_like(inp["Wg"])), k=2, bias=bias,
+                     w_mode=oracle.W_ENTROPY)
+    assert (r["idx"][:, 0] == 3).all() and (r["idx"][:, 1] == -1).all()
+    assert np.allclose(r["w"][:, 0], 1.0 / (1.0 + 3 * np.exp(-50.0)), rtol=1e-15)
+
+
+def test_entropy_controlled_layer_is_the_dense_masked_sum():
+    wl, inp = _inputs(T=12, d=16, E=6, dff=10, k=3, seed=8)
+    Wg = (inp["Wg"].float() * 0.1).to(torch.bfloat16)
+    names = ("x", "W1", "W3", "W2")
+    out = oracle.forward(bits(inp["x"]), bits(Wg), *(bits(inp[n]) for n in names[1:]), k=3,
+                         w_mode=oracle.W_ENTROPY)
+    L = (_f64(inp["x"]) @ _f64(Wg).T).numpy()
+    idx, w, H, kt = _entropy_route_torch(L, 3)
+    assert 0 < (kt == 2).sum() < 12                  # both branches occur
+    Y = np.zeros((12, 16))
+    for e in range(6):
+        ye = _swiglu_torch(inp["x"], inp["W1"][e], inp["W3"][e], inp["W2"][e]).numpy()
+        Y += (w * (idx == e)).sum(1, keepdims=True) * ye
+    assert _rel(out, Y) < 1e-12
+    # A forced set equal to the token's own (unused last slot included)
+    # reproduces it.
+    r = oracle.route(bits(inp["x"]), bits(Wg), k=3, w_mode=oracle.W_ENTROPY)
+    f = oracle.forward(bits(inp["x"]), bits(Wg), *(bits(inp[n]) for n in names[1:]), k=3,
+                       w_mode=oracle.W_ENTROPY, forced=r["idx"])
+    assert np.array_equal(f, out)
+
+
 def test_capacity_limit_closed_form():
     # floor(cf * T * k / E): capacity factor 1.2 ("Mistral 8x7B SMoE" sec. 2.4)
     # on the small layer and a few exact cases.
