@@ -212,6 +212,17 @@ MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const mo
  *                               Router.forward)
  *     MOE_WEIGHTS_SIGMOID       the logistic sigmoid of each selected logit
  *                               ("万亿 MoE" (m.xxqk.cn) forward listing)
+ *     MOE_WEIGHTS_ENTROPY       entropy-controlled k ("Mixtral 8x7B模型架构解析",
+ *                               routing-strategy section, entropy_aware_routing):
+ *                               p = softmax(logits / 0.1) over all E; a token
+ *                               keeps its top k experts when the entropy
+ *                               -sum p ln p exceeds 0.8, else its top k - 1,
+ *                               weighted by their p (not renormalised).  An
+ *                               unused slot holds expert -1 and weight 0 (in
+ *                               moe_route_variant's idx and w too) and has no
+ *                               row.  Needs k >= 2; not combined with a
+ *                               capacity (MOE_ERR_UNSUPPORTED).  The decision
+ *                               is taken in fp32.
  *   activation: expert hidden units
  *     MOE_ACT_SILU     silu(W1 x) * (W3 x), SwiGLU (the method)
  *     MOE_ACT_SIGMOID  sigmoid(W1 x) * (W3 x), the listing's a * sigmoid(g)
@@ -222,10 +233,12 @@ MOE_API moe_status moe_forward_ex(int T, int d, int E, int d_ff, int k, const mo
  *     expert only the first C in token order are computed; a dropped pair
  *     adds nothing to its token (the other slots keep their weights).
  *     Negative or non-finite values are MOE_ERR_INVALID_ARG.
- * Selection (top-k, ties to the lower index) is the same under every rule. */
+ * Selection (top-k, ties to the lower index) is the same under every rule
+ * (the entropy rule may drop the k-th). */
 #define MOE_WEIGHTS_SOFTMAX_TOPK 0
 #define MOE_WEIGHTS_SOFTMAX_ALL 1
 #define MOE_WEIGHTS_SIGMOID 2
+#define MOE_WEIGHTS_ENTROPY 3
 #define MOE_ACT_SILU 0
 #define MOE_ACT_SIGMOID 1
 

@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     ABI_FUNCTIONS,
     ACT_SIGMOID,
     ACT_SILU,
+    WEIGHTS_ENTROPY,
     WEIGHTS_SIGMOID,
     WEIGHTS_SOFTMAX_ALL,
     WEIGHTS_SOFTMAX_TOPK,

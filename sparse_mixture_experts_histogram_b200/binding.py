@@ -41,7 +41,7 @@ TRACE_STAGES = ("route", "scatter", "expert_ffn", "shared_ffn", "combine")
 
 
 #: Gate-weight rules and expert activations of ``moe_variant`` (include/moe.h).
-WEIGHTS_SOFTMAX_TOPK, WEIGHTS_SOFTMAX_ALL, WEIGHTS_SIGMOID = 0, 1, 2
+WEIGHTS_SOFTMAX_TOPK, WEIGHTS_SOFTMAX_ALL, WEIGHTS_SIGMOID, WEIGHTS_ENTROPY = 0, 1, 2, 3
 ACT_SILU, ACT_SIGMOID = 0, 1
 
 

@@ -374,7 +374,8 @@ moe_status moe_route_variant(int T, int d, int E, int k, const moe_bf16 *x, cons
                              const float *router_bias, int weights, int32_t *idx, float *w,
                              int32_t *counts, void *ws, size_t ws_bytes, moe_stream_t stream)
 {
-    if (weights < 0 || weights > 2) return MOE_ERR_INVALID_ARG;
+    if (weights < 0 || weights > MOE_WEIGHTS_ENTROPY) return MOE_ERR_INVALID_ARG;
+    if (weights == MOE_WEIGHTS_ENTROPY && k < 2) return MOE_ERR_INVALID_ARG;
     moe_status st = check_shapes(T, d, E, 128, k, 0);
     if (st != MOE_OK) return st;
     if (!ok_ptr(x) || !ok_ptr(Wg) || !ok_ptr(idx) || !ok_ptr(w) || !ok_ptr(ws))
@@ -579,8 +580,11 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
     const int wmode = variant ? variant->weights : MOE_WEIGHTS_SOFTMAX_TOPK;
     const int act = variant ? variant->activation : MOE_ACT_SILU;
     const double cf = variant ? variant->capacity_factor : 0.0;
-    if (wmode < 0 || wmode > 2 || act < 0 || act > 1 || !(cf >= 0.0) || cf > 1e9)
+    if (wmode < 0 || wmode > MOE_WEIGHTS_ENTROPY || act < 0 || act > 1 || !(cf >= 0.0) ||
+        cf > 1e9)
         return MOE_ERR_INVALID_ARG;
+    if (wmode == MOE_WEIGHTS_ENTROPY && k < 2) return MOE_ERR_INVALID_ARG;
+    if (wmode == MOE_WEIGHTS_ENTROPY && cf > 0.0) return MOE_ERR_UNSUPPORTED;
     // Per-expert capacity floor(cf * T * k / E); no expert ever receives more
     // than T pairs, so a capacity of T or more drops nothing.
     int cap = -1;
@@ -705,6 +709,7 @@ static moe_status forward_impl(int T, int d, int E, int d_ff, int k, const moe_b
         c.row_of_slot = row;
         c.slot_of_row = fused_out ? slotrow : nullptr;
         c.out_zero = fused_out ? out : nullptr;
+        c.allow_empty = wmode == MOE_WEIGHTS_ENTROPY;
         c.err = err;
         c.pdl = pdl;
         st = from_cuda(launch_scatter(c, s));

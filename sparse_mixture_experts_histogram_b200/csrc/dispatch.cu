@@ -61,6 +61,7 @@ struct ScatterParams {
     float4 *out_zero;      // or nullptr
     uint32_t *err;
     int S;
+    int allow_empty;  // expert -1 marks an unused slot (no row, no error)
     int to_f16;  // convert the rows to fp16 on the way
     int chunks;  // 16-byte-vector chunks of kScatterVec*32 per row
 };
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(32 * kScatterWarps) scatter_kernel(const Scatt
         const size_t s = static_cast<size_t>(t) * p.k + lane;
         const int e = p.idx[s];
         const int r = p.rank[s];
-        bool dropped = false;
+        bool dropped = p.allow_empty && e == -1;
         if (e >= 0 && e < p.E && r >= 0) {
             const int row = p.tilebase[static_cast<size_t>(t / kTileTokens) * p.E + e] + r;
             // With a capacity, a pair ranked at or beyond it in its expert's
@@ -190,6 +191,7 @@ cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s)
     p.out_zero = reinterpret_cast<float4 *>(a.out_zero);
     p.err = a.err;
     p.S = a.T * a.k;
+    p.allow_empty = a.allow_empty ? 1 : 0;
     p.to_f16 = a.to_f16 ? 1 : 0;
     const int nv = a.d / 8;
     p.chunks = (nv + 32 * kScatterVec - 1) / (32 * kScatterVec);

@@ -9,7 +9,8 @@ namespace moe {
 
 struct RouteLaunch {
     int T, d, E, k;
-    int wmode;           // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid
+    int wmode;           // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid,
+                         // 3 tempered softmax over all with entropy-controlled k (slot K-1 may be -1)
     const uint16_t *x;   // [T,d] bf16
     const uint16_t *Wg;  // [E,d] bf16
     const float *bias;   // [E] or nullptr
@@ -52,6 +53,7 @@ struct ScatterLaunch {
     uint32_t *err;
     bool pdl;  // launched right after another kernel of this library
     bool to_f16;  // write x_perm as fp16 (the FP8 expert path) instead of bf16
+    bool allow_empty;  // idx -1 marks an unused slot (entropy-controlled k), not an error
     // For the expert kernel's weighted output (FfnLaunch::out), when set:
     // slot_of_row[row] = t*k + j for every row that got a slot, and out[T, d]
     // set to zero.

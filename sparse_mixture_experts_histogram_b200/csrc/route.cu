@@ -30,7 +30,8 @@ constexpr uint32_t kRouteABytes = 128 * 128;   // 128 token rows x 64 bf16
 
 struct RouteParams {
     int T, d, E, Npad, stages, ntiles;
-    int wmode;      // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid
+    int wmode;      // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid,
+                    // 3 tempered softmax over all with entropy-controlled k
     uint32_t tmem_cols;
     const float *bias;
     int32_t *idx;
@@ -87,11 +88,20 @@ __device__ __forceinline__ void topk_insert(float (&tv)[K], int (&ti)[K], float 
 //            sum_all = sum_e exp(l_e - m_all); not renormalised over the
 //            selected ("Mixtral 8x7B模型架构解析" Router.forward)
 //   wmode 2: the sigmoid of each selected logit ("万亿 MoE" forward listing)
+//   wmode 3: the softmax of l / tau over all E logits (tau = 0.1), given
+//            m_all and sum_all = sum_e exp((l_e - m_all) / tau), not
+//            renormalised ("Mixtral 8x7B模型架构解析" entropy_aware_routing)
+constexpr float kEntropyInvTau = 10.0f;     // 1 / tau, tau = 0.1
+constexpr float kEntropyThreshold = 0.8f;   // nats
+
 template <int K>
 __device__ __forceinline__ void gate_weights(const float (&tv)[K], int wmode, float m_all,
                                              float sum_all, float (&w)[K])
 {
-    if (wmode == 1) {
+    if (wmode == 3) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) w[j] = expf((tv[j] - m_all) * kEntropyInvTau) / sum_all;
+    } else if (wmode == 1) {
 #pragma unroll
         for (int j = 0; j < K; ++j) w[j] = expf(tv[j] - m_all) / sum_all;
     } else if (wmode == 2) {
@@ -108,6 +118,19 @@ __device__ __forceinline__ void gate_weights(const float (&tv)[K], int wmode, fl
         for (int j = 0; j < K; ++j) w[j] = w[j] / s;
     }
 }
+
+// Slots a token keeps under wmode 3: K when the entropy of the tempered
+// softmax exceeds the threshold, K - 1 otherwise.  With Z = sum_e
+// exp((l_e - m) / tau) and A = sum_e exp((l_e - m) / tau) (l_e - m), the
+// entropy -sum_e p_e ln p_e of p_e = exp((l_e - m) / tau) / Z is
+// ln Z - A / (tau Z).
+template <int K>
+__device__ __forceinline__ int entropy_slots(float z, float a)
+{
+    const float h = logf(z) - a * kEntropyInvTau / z;
+    return h > kEntropyThreshold ? K : K - 1;
+}
+
 
 // Waits for the copies the producer issued into each stage to land, so that
 // no copy is still writing shared memory when the CTA exits after an abort.
@@ -237,7 +260,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         }
         // Running maximum and sum of exp(l - max) over all E logits (for the
         // softmax over all experts).
-        float run_m = -CUDART_INF_F, run_s = 0.0f;
+        float run_m = -CUDART_INF_F, run_s = 0.0f, run_a = 0.0f;
         if (ok) {
             const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
             for (int c0 = 0; c0 < p.Npad; c0 += 16) {
@@ -258,6 +281,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
                                 run_m = l;
                             } else {
                                 run_s += expf(l - run_m);
+                            }
+                        } else if (p.wmode == 3 && l > -CUDART_INF_F) {
+                            // Tempered running sum Z and A = sum exp(.)(l - m),
+                            // both rescaled when the maximum moves.
+                            if (run_s == 0.0f) {
+                                run_m = l;
+                                run_s = 1.0f;
+                            } else if (l > run_m) {
+                                const float f = expf((run_m - l) * kEntropyInvTau);
+                                run_a = f * (run_a + run_s * (run_m - l));
+                                run_s = run_s * f + 1.0f;
+                                run_m = l;
+                            } else {
+                                const float q = expf((l - run_m) * kEntropyInvTau);
+                                run_s += q;
+                                run_a += q * (l - run_m);
                             }
                         }
                     }
@@ -286,17 +325,20 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
         ptx::tc_fence_before();
 
         const bool valid = ok && (t < p.T);
+        // Slots in use: all K, or K - 1 under the entropy rule (the last
+        // slot then holds expert -1 and weight 0).
+        const int ku = p.wmode == 3 ? entropy_slots<K>(run_s, run_a) : K;
         if (valid) {
             float wv[K];
             gate_weights<K>(tv, p.wmode, run_m, run_s, wv);
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                p.idx[static_cast<size_t>(t) * K + j] = ti[j];
-                p.w[static_cast<size_t>(t) * K + j] = wv[j];
+                p.idx[static_cast<size_t>(t) * K + j] = j < ku ? ti[j] : -1;
+                p.w[static_cast<size_t>(t) * K + j] = j < ku ? wv[j] : 0.0f;
             }
         }
 #pragma unroll
-        for (int j = 0; j < K; ++j) ds.sel[row][j] = valid ? ti[j] : -1;
+        for (int j = 0; j < K; ++j) ds.sel[row][j] = (valid && j < ku) ? ti[j] : -1;
         if (p.slots)
             assign_slots(ds, tile * kTileTokens, kTileTokens, p.T, p.E, K, p.sout, row,
                          kTileTokens, 1);
@@ -327,7 +369,8 @@ constexpr int kSmallThreads = 256;
 
 struct SmallRouteParams {
     int T, d, E;
-    int wmode;      // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid
+    int wmode;      // gate weights: 0 softmax over the selected, 1 softmax over all, 2 sigmoid,
+                    // 3 tempered softmax over all with entropy-controlled k
     const uint4 *x;
     const uint4 *Wg;
     const float *bias;
@@ -492,7 +535,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
         }
         // Sum of exp(l - max) over all E logits (the softmax over all
         // experts); tv[0] is the maximum.
-        float sum_all = 0.0f;
+        float sum_all = 0.0f, sum_a = 0.0f;
         if (p.wmode == 1) {
 #pragma unroll
             for (int i = 0; i < kMaxE / 32; ++i)
@@ -500,15 +543,32 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(const SmallR
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1)
                 sum_all += __shfl_xor_sync(0xffffffffu, sum_all, off);
+        } else if (p.wmode == 3) {
+            // Tempered softmax sum Z and A = sum exp((l - m) / tau) (l - m).
+#pragma unroll
+            for (int i = 0; i < kMaxE / 32; ++i) {
+                if (lane + 32 * i < p.E && v[i] > -CUDART_INF_F) {
+                    const float q = expf((v[i] - tv[0]) * kEntropyInvTau);
+                    sum_all += q;
+                    sum_a += q * (v[i] - tv[0]);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sum_all += __shfl_xor_sync(0xffffffffu, sum_all, off);
+                sum_a += __shfl_xor_sync(0xffffffffu, sum_a, off);
+            }
         }
         if (lane == 0) {
             float wv[K];
             gate_weights<K>(tv, p.wmode, tv[0], sum_all, wv);
+            // Slots in use: all K, or K - 1 under the entropy rule.
+            const int ku = p.wmode == 3 ? entropy_slots<K>(sum_all, sum_a) : K;
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                p.idx[static_cast<size_t>(t) * K + j] = ti[j];
-                p.w[static_cast<size_t>(t) * K + j] = wv[j];
-                ds.sel[warp][j] = ti[j];
+                p.idx[static_cast<size_t>(t) * K + j] = j < ku ? ti[j] : -1;
+                p.w[static_cast<size_t>(t) * K + j] = j < ku ? wv[j] : 0.0f;
+                ds.sel[warp][j] = j < ku ? ti[j] : -1;
             }
         }
     }

@@ -143,17 +143,26 @@ def test_static_scratch_limit_matches_its_documented_formula(lib):
 def test_variant_arguments_are_checked_on_the_host(lib):
     V = binding.MoEVariant
     ws = 1 << 40
-    for bad in (V(3, 0, 0.0), V(-1, 0, 0.0), V(0, 2, 0.0), V(0, 0, -1.0), V(0, 0, float("nan")),
+    for bad in (V(4, 0, 0.0), V(-1, 0, 0.0), V(0, 2, 0.0), V(0, 0, -1.0), V(0, 0, float("nan")),
                 V(0, 0, float("inf"))):
         st = lib.moe_forward_variant(16, 512, 8, 1024, 2, FAKE, FAKE, None, FAKE, FAKE, FAKE, 0,
                                      None, None, None, ctypes.addressof(bad), FAKE, FAKE, ws, None)
         assert st == 1, (bad.weights, bad.activation, bad.capacity_factor)
-    assert lib.moe_route_variant(16, 512, 8, 2, FAKE, FAKE, None, 3, FAKE, FAKE, None, FAKE, ws,
+    assert lib.moe_route_variant(16, 512, 8, 2, FAKE, FAKE, None, 4, FAKE, FAKE, None, FAKE, ws,
                                  None) == 1
+    # the entropy rule needs k >= 2 and takes no capacity
+    assert lib.moe_route_variant(16, 512, 8, 1, FAKE, FAKE, None, 3, FAKE, FAKE, None, FAKE, ws,
+                                 None) == 1
+    for bad, want in ((V(3, 0, 0.0), 1), (V(3, 0, 1.2), 2)):
+        k = 1 if want == 1 else 2
+        st = lib.moe_forward_variant(16, 512, 8, 1024, k, FAKE, FAKE, None, FAKE, FAKE, FAKE, 0,
+                                     None, None, None, ctypes.addressof(bad), FAKE, FAKE, ws, None)
+        assert st == want
     assert lib.moe_route_variant(16, 512, 8, 9, FAKE, FAKE, None, 1, FAKE, FAKE, None, FAKE, ws,
                                  None) == 1
     h = open(os.path.join(ROOT, "include", "moe.h")).read()
     for name, v in (("MOE_WEIGHTS_SOFTMAX_TOPK", 0), ("MOE_WEIGHTS_SOFTMAX_ALL", 1),
-                    ("MOE_WEIGHTS_SIGMOID", 2), ("MOE_ACT_SILU", 0), ("MOE_ACT_SIGMOID", 1)):
+                    ("MOE_WEIGHTS_SIGMOID", 2), ("MOE_WEIGHTS_ENTROPY", 3), ("MOE_ACT_SILU", 0),
+                    ("MOE_ACT_SIGMOID", 1)):
         assert f"#define {name} {v}" in h
     assert ctypes.sizeof(V) == 16

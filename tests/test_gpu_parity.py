@@ -464,6 +464,115 @@ def test_forward_variant_matches_oracle(wl, variant):
         assert counts.max() > res["cap"]
 
 
+# Entropy-controlled k ("Mixtral 8x7B模型架构解析" entropy_aware_routing): the
+# router's Wg is scaled so that the tempered softmax's entropy falls on both
+# sides of the 0.8 threshold.  Where floating point decides the slot count,
+# tokens whose fp64 entropy is within 1e-3 of the threshold may go either way
+# and are compared with the oracle forced to the GPU's choice; likewise for
+# near ties of the last used logit.
+def _entropy_inputs(wl, scale=0.25, big=False):
+    inp = synth.make_inputs(wl, device=DEV) if big else _inputs(wl)
+    inp["Wg"] = (inp["Wg"].float() * scale).to(torch.bfloat16)
+    inp["bias"] = torch.linspace(-0.02, 0.03, wl.E, dtype=torch.float32, device=DEV)
+    return inp
+
+
+def _entropy_route_check(wl, inp, idx, w):
+    """GPU routing under the entropy rule vs the oracle.  Returns (oracle
+    route, mask of tokens the test cannot decide by fp64)."""
+    bias = inp["bias"].double().cpu().numpy()
+    r = oracle.route(bits(inp["x"]), bits(inp["Wg"]), wl.k, bias=bias, w_mode=oracle.W_ENTROPY)
+    L = r["logits"]
+    P = np.exp((L - L.max(1, keepdims=True)) / oracle.ENTROPY_TAU)
+    P /= P.sum(1, keepdims=True)
+    H = -np.where(P > 0, P * np.log(np.where(P > 0, P, 1.0)), 0.0).sum(1)
+    ku_o = (r["idx"] >= 0).sum(1)
+    Ls = -np.sort(-L, 1)
+    gap = np.array([Ls[t, ku_o[t] - 1] - Ls[t, ku_o[t]] for t in range(wl.T)])
+    unsure = (np.abs(H - oracle.ENTROPY_THRESHOLD) < 1e-3) | (gap < 1e-3)
+    far = ~unsure
+    ku_g = (idx >= 0).sum(1)
+    assert (idx[:, :wl.k - 1] >= 0).all() and ((idx >= 0).sum(1) >= wl.k - 1).all()
+    assert (w[idx < 0] == 0).all()
+    assert np.array_equal(ku_g[far], ku_o[far]), "slot counts differ"
+    for t in np.nonzero(far)[0]:
+        assert set(idx[t][idx[t] >= 0]) == set(r["idx"][t][r["idx"][t] >= 0]), t
+    wg = np.where(idx >= 0, w, 0.0)
+    wgs = np.take_along_axis(wg, np.argsort(np.where(idx >= 0, idx, 10**6), 1), 1)
+    wos = np.take_along_axis(r["w"], np.argsort(np.where(r["idx"] >= 0, r["idx"], 10**6), 1), 1)
+    assert np.max(np.abs(wgs[far] - wos[far])) < 2e-4
+    assert 0.1 < (ku_o == wl.k).mean() < 0.9, "both slot counts occur"
+    return r, unsure
+
+
+@pytest.mark.parametrize("wl", [Workload("ent_T300_E16_k3", 300, 256, 16, 128, 3),
+                                Workload("ent_tc_T1153_d4608_E256_k4", 1153, 4608, 256, 128, 4)],
+                         ids=lambda w: w.name)
+def test_route_entropy_controlled_k_matches_oracle(wl):
+    big = wl.T * wl.E * wl.d > 2 ** 30
+    inp = _entropy_inputs(wl, scale=0.25 if wl.E <= 16 else 0.6, big=big)
+    idx = torch.empty(wl.T, wl.k, dtype=torch.int32, device=DEV)
+    w = torch.empty(wl.T, wl.k, dtype=torch.float32, device=DEV)
+    counts = torch.empty(wl.E, dtype=torch.int32, device=DEV)
+    ws = workspace(wl)
+    moe.moe_route_variant(wl.T, wl.d, wl.E, wl.k, inp["x"], inp["Wg"], inp["bias"],
+                          moe.WEIGHTS_ENTROPY, idx, w, counts, ws)
+    assert moe.moe_get_device_error(ws)[0] == 0
+    idx, w, counts = idx.cpu().numpy(), w.cpu().numpy(), counts.cpu().numpy()
+    _entropy_route_check(wl, inp, idx, w)
+    assert np.array_equal(counts, np.bincount(idx[idx >= 0], minlength=wl.E))
+
+
+ENTROPY_FORWARD_CASES = [
+    Workload("ent_narrow_T300_d256_E8_k3", 300, 256, 8, 384, 3),
+    Workload("ent_narrow_T300_d256_E8_k2_shared", 300, 256, 8, 384, 2, d_ff_shared=256),
+    Workload("ent_wide_T200_d1152_E8_k3", 200, 1152, 8, 384, 3),
+    Workload("ent_wide_pair_T1100_d1152_E8_k2", 1100, 1152, 8, 512, 2),
+]
+
+
+@pytest.mark.parametrize("wl", ENTROPY_FORWARD_CASES, ids=lambda w: w.name)
+def test_forward_entropy_controlled_k_matches_oracle(wl):
+    from gpu_util import gpu_forward_variant
+    inp = _entropy_inputs(wl)
+    variant = (moe.WEIGHTS_ENTROPY, 0, 0.0)
+    idx = torch.empty(wl.T, wl.k, dtype=torch.int32, device=DEV)
+    w = torch.empty(wl.T, wl.k, dtype=torch.float32, device=DEV)
+    ws = workspace(wl)
+    moe.moe_route_variant(wl.T, wl.d, wl.E, wl.k, inp["x"], inp["Wg"], inp["bias"],
+                          moe.WEIGHTS_ENTROPY, idx, w, None, ws)
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    r, unsure = _entropy_route_check(wl, inp, idx, w)
+    out = gpu_forward_variant(wl, inp, variant).cpu().numpy().astype(np.float64)
+    tok = np.arange(wl.T) if wl.T <= 300 else sample_tokens(wl.T, 96, idx, unsure)
+    shared = None
+    if wl.d_ff_shared:
+        shared = (bits(inp["Ws1"]), bits(inp["Ws3"]), bits(inp["Ws2"]))
+    ref = oracle.forward(bits(inp["x"]), bits(inp["Wg"]), bits(inp["W1"]), bits(inp["W3"]),
+                         bits(inp["W2"]), wl.k, bias=inp["bias"].double().cpu().numpy(),
+                         tokens=tok, shared=shared, forced=idx[tok], w_mode=oracle.W_ENTROPY)
+    assert_close(out[tok], ref, wl.name)
+
+
+def test_entropy_controlled_k_argument_checks():
+    wl = Workload("ent_args", 16, 256, 8, 128, 1)
+    inp = _inputs(wl)
+    ws = workspace(wl)
+    out = torch.empty(16, 256, device=DEV)
+    with pytest.raises(moe.MoEError) as e:   # k = 1 leaves no slot to drop
+        moe.moe_forward_variant(16, 256, 8, 128, 1, inp["x"], inp["Wg"], None, inp["W1"],
+                                inp["W3"], inp["W2"], 0, None, None, None,
+                                (moe.WEIGHTS_ENTROPY, 0, 0.0), out, ws)
+    assert e.value.status == 1
+    wl2 = Workload("ent_args2", 16, 256, 8, 128, 2)
+    ws2 = workspace(wl2)
+    with pytest.raises(moe.MoEError) as e:   # not combined with a capacity
+        moe.moe_forward_variant(16, 256, 8, 128, 2, inp["x"], inp["Wg"], None, inp["W1"],
+                                inp["W3"], inp["W2"], 0, None, None, None,
+                                (moe.WEIGHTS_ENTROPY, 0, 1.0), out, ws2)
+    assert e.value.status == 2
+
+
 def test_forward_variant_none_is_the_method():
     wl = Workload("var_none", 200, 256, 8, 256, 2)
     inp = _inputs(wl)
