@@ -197,6 +197,11 @@ class ExpertParallelLayer:
     per GPU on one node).  Holds this rank's expert block W1/W3/W2[E/R, ...]
     and the replicated router (and shared expert).
 
+    The receive and output buffers are mapped into the peers with CUDA IPC,
+    which needs memory from cudaMalloc: torch's caching allocator in its
+    default mode (with expandable segments the handle export fails and the
+    constructor raises MoEError).
+
     With an NCCL group the collectives are stream-ordered: nothing waits on
     the host and a step can be captured in a CUDA graph.  With any other
     backend (gloo) the same steps are ordered on the host instead: the
