@@ -462,6 +462,15 @@ MOE_API moe_status moe_ipc_open_handle(const void *handle, void **base);
 /* Unmaps a base returned by moe_ipc_open_handle. */
 MOE_API moe_status moe_ipc_close(void *base);
 
+/* Failure-detection self-test: one thread waits, through the bounded wait
+ * every pipeline of the library uses, for a barrier phase that nothing
+ * completes.  After the wait's time bound (2 s) it sets
+ * MOE_DEVERR_TIMEOUT_MMA in the error word of ws (cleared first; ws at least
+ * 256 bytes) and the kernel returns; moe_get_device_error(ws) then reports
+ * MOE_ERR_TIMEOUT and the context stays usable.  The pages have no
+ * counterpart. */
+MOE_API moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Static description of a status code; never NULL. */
 MOE_API const char *moe_status_string(moe_status status);
 

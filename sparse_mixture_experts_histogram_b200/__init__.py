@@ -40,6 +40,7 @@ from .binding import (  # noqa: F401
     moe_permute,
     moe_route,
     moe_route_variant,
+    moe_selftest_wait_timeout,
     moe_status_string,
     moe_workspace_size,
     moe_workspace_size_ex,

@@ -34,7 +34,7 @@ ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "mo
                  "moe_forward_fp8", "moe_forward_fp8_traced", "moe_ep_recv_rows",
                  "moe_ep_workspace_size", "moe_ep_ffn_splits", "moe_ep_dispatch",
                  "moe_ep_expert_ffn", "moe_ep_combine", "moe_ipc_get_handle",
-                 "moe_ipc_open_handle", "moe_ipc_close")
+                 "moe_ipc_open_handle", "moe_ipc_close", "moe_selftest_wait_timeout")
 TRACE_EVENTS = 6
 #: What each of moe_forward_traced's events marks (event i = start of stage i).
 TRACE_STAGES = ("route", "scatter", "expert_ffn", "shared_ffn", "combine")
@@ -104,6 +104,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
             "moe_ipc_get_handle": (_I, [_P, _P, _P]),
             "moe_ipc_open_handle": (_I, [_P, _P]),
             "moe_ipc_close": (_I, [_P]),
+            "moe_selftest_wait_timeout": (_I, [_P, _SZ, _P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -356,3 +357,10 @@ def moe_ipc_open_handle(handle: bytes) -> int:
 
 def moe_ipc_close(base: int) -> None:
     _check(load_library().moe_ipc_close(base), "moe_ipc_close")
+
+
+def moe_selftest_wait_timeout(ws, stream=None):
+    """Runs a bounded wait that nothing completes (about 2 s); read the
+    result with moe_get_device_error(ws)."""
+    _check(load_library().moe_selftest_wait_timeout(_ptr(ws), _ws_bytes(ws), _stream(stream)),
+           "moe_selftest_wait_timeout")

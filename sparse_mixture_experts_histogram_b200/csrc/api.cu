@@ -943,6 +943,15 @@ moe_status moe_forward(int T, int d, int E, int d_ff, int k, const moe_bf16 *x,
                           nullptr, out, ws, ws_bytes, stream);
 }
 
+moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!ok_ptr(ws) || ws_bytes < kHeaderBytes) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    moe_status st = from_cuda(cudaMemsetAsync(ws, 0, kHeaderBytes, s));
+    if (st != MOE_OK) return st;
+    return from_cuda(launch_wait_timeout(static_cast<uint32_t *>(ws), s));
+}
+
 moe_status moe_get_device_error(const void *ws, uint32_t *code, moe_stream_t stream)
 {
     if (ws == nullptr) return MOE_ERR_INVALID_ARG;

@@ -157,6 +157,9 @@ struct EpCombineLaunch {
 cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s);
 cudaError_t launch_ep_combine(const EpCombineLaunch &a, cudaStream_t s);
 
+// Failure-detection self-test (selftest.cu): a bounded wait that runs out.
+cudaError_t launch_wait_timeout(uint32_t *err, cudaStream_t s);
+
 cudaError_t launch_route(const RouteLaunch &a, cudaStream_t s);
 cudaError_t launch_ranks(const RanksLaunch &a, cudaStream_t s);
 cudaError_t launch_scatter(const ScatterLaunch &a, cudaStream_t s);

@@ -166,3 +166,8 @@ def test_variant_arguments_are_checked_on_the_host(lib):
                     ("MOE_ACT_SIGMOID", 1)):
         assert f"#define {name} {v}" in h
     assert ctypes.sizeof(V) == 16
+
+
+def test_selftest_checks_its_workspace(lib):
+    assert lib.moe_selftest_wait_timeout(None, 1 << 20, None) == 1
+    assert lib.moe_selftest_wait_timeout(FAKE, 16, None) == 1   # smaller than the header

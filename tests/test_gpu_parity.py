@@ -208,6 +208,23 @@ def test_expert_ffn_matches_oracle(name, d, d_ff, sizes):
         assert_close(y[a:b], ref, f"{name} expert {e}")
 
 
+def test_bounded_wait_runs_out_and_the_context_stays_usable():
+    """Failure detection without a fault: a wait (the pipelines' bounded
+    wait) on a barrier phase that nothing completes gives up after its 2 s
+    bound, reports MOE_ERR_TIMEOUT through the error word, and the next
+    layer call on the same context still matches the oracle."""
+    import time
+    ws = torch.empty(4096, dtype=torch.uint8, device=DEV)
+    t0 = time.time()
+    moe.moe_selftest_wait_timeout(ws)
+    st, code = moe.moe_get_device_error(ws)
+    dt = time.time() - t0
+    assert st == 6 and code & 0x2, (st, code)      # MOE_ERR_TIMEOUT, TIMEOUT_MMA
+    assert 1.5 < dt < 60
+    wl = Workload("after_timeout", 64, 256, 8, 256, 2)
+    check_forward(wl, _inputs(wl))
+
+
 def test_expert_ffn_rejects_inconsistent_offsets():
     wl = Workload("bad_offsets", 64, 128, 4, 128, 1)
     inp = _inputs(wl)
