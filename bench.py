@@ -793,7 +793,8 @@ def ep_arm(args):
     ffn = []
     for r in range(R):
         flops = acc.ffn_flops(rows[r], wl.d, wl.d_ff, 1)
-        byts = 2 * 3 * hit[r] * wl.d * wl.d_ff + 2 * rows[r] * wl.d + 4 * p.ksplit * rows[r] * wl.d
+        yb = 2 if p.y_bf16 else 4 * p.ksplit  # output bytes per element of a row
+        byts = 2 * 3 * hit[r] * wl.d * wl.d_ff + 2 * rows[r] * wl.d + yb * rows[r] * wl.d
         t = med["expert_ffn"][r] * 1e-6
         ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
         if byts and flops / byts > ridge:
@@ -812,6 +813,7 @@ def ep_arm(args):
         "config": {"workload": f"{args.workload}_ep{R}_emulated", "ep_ranks": R,
                    "tokens_per_rank": T, "layer": describe(wls, args.workload)["layers"][0],
                    "recv_rows_per_rank": p.recv_rows, "down_ksplit": p.ksplit,
+                   "output_rows": "bf16" if p.y_bf16 else "fp32",
                    "l2": "weights larger than L2 stream from HBM every step"
                    if 2 * 3 * wl.E * wl.d * wl.d_ff > L2_BYTES else "may be L2-resident"},
         "ep": {"per_rank_us": med, "rank_kernels_us_max": max(rank_us),

@@ -365,7 +365,8 @@ MOE_API moe_status moe_get_device_error(const void *ws, uint32_t *code, moe_stre
  * Rank q owns experts [q*E/R, (q+1)*E/R) and holds only their weights
  * (W1, W3, W2 of moe_ep_expert_ffn are that block, [E/R, ...]).  Every rank
  * keeps a receive buffer recv_x [recv_rows, d] bf16 and an output buffer
- * recv_y [ksplit, recv_rows, d] fp32 that every other rank can address (its
+ * recv_y (fp32 [ksplit, recv_rows, d], or bf16 [recv_rows, d] where
+ * moe_ep_output_bf16 allows) that every other rank can address (its
  * own allocation, mapped into the peers with moe_ipc_get_handle /
  * moe_ipc_open_handle), with recv_rows = moe_ep_recv_rows(T_max, E, k, R).
  * One layer step, on every rank, all on one stream:
@@ -423,28 +424,35 @@ MOE_API moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank,
                                    int recv_rows, int32_t *pos_of_slot, int32_t *recv_offsets,
                                    void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* 1 when moe_ep_expert_ffn can write bf16 output rows for these sizes (the
+ * expert kernel then writes complete rows, no K split), else 0.  bf16 rows
+ * halve what the combine reads back over NVLink; each row is rounded once,
+ * as the hidden activations are. */
+MOE_API int moe_ep_output_bf16(int rows_hint, int d, int E_local, int d_ff);
+
 /* Step 5: moe_expert_ffn over this rank's E/R experts on its receive buffer
  * (recv_rows = moe_ep_recv_rows(T_max, E, k, R) rows, segments from
  * recv_offsets).  rows_hint: rows the rank expects to receive (T*k with
  * balanced experts; it picks the kernel's tiling, not the result); ksplit must be
- * moe_ep_ffn_splits(rows_hint, d, E/R, d_ff).  recv_y [ksplit, recv_rows, d]
- * fp32 out (rows beyond the segments are not written).  Keeps the error
- * word of the step's dispatch. */
+ * moe_ep_ffn_splits(rows_hint, d, E/R, d_ff).  y_bf16: 0, or 1 where
+ * moe_ep_output_bf16 allows it.  recv_y out: [ksplit, recv_rows, d] fp32, or
+ * [recv_rows, d] bf16 with y_bf16 (rows beyond the segments are not
+ * written).  Keeps the error word of the step's dispatch. */
 MOE_API moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R,
-                                     int rows_hint, int ksplit, const moe_bf16 *recv_x,
-                                     const int32_t *recv_offsets, const moe_bf16 *W1,
-                                     const moe_bf16 *W3, const moe_bf16 *W2, float *recv_y,
-                                     void *ws, size_t ws_bytes, moe_stream_t stream);
+                                     int rows_hint, int ksplit, int y_bf16,
+                                     const moe_bf16 *recv_x, const int32_t *recv_offsets,
+                                     const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2,
+                                     void *recv_y, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Step 7: out[t] = sum_{j<k} w[t,j] * (sum_q recv_y_o[q, pos_of_slot[t,j]])
  * (+ shared_y[t]), o = owner of idx[t,j], slots in order j = 0..k-1, the K
  * split partials q in order.  recv_y: host array of R device addresses of
- * the ranks' output buffers.  A slot with pos_of_slot -1 adds nothing.
- * out [T,d] fp32 (overwritten). */
+ * the ranks' output buffers, fp32, or bf16 rows with y_bf16 = 1 (ksplit 1).
+ * A slot with pos_of_slot -1 adds nothing.  out [T,d] fp32 (overwritten). */
 MOE_API moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int ksplit,
-                                  const int32_t *idx, const int32_t *pos_of_slot, const float *w,
-                                  const float *const *recv_y, const float *shared_y, float *out,
-                                  moe_stream_t stream);
+                                  int y_bf16, const int32_t *idx, const int32_t *pos_of_slot,
+                                  const float *w, const void *const *recv_y,
+                                  const float *shared_y, float *out, moe_stream_t stream);
 
 /* Size of an inter-process memory handle (cudaIpcMemHandle_t). */
 #define MOE_IPC_HANDLE_BYTES 64

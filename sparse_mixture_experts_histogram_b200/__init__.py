@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     moe_ep_dispatch,
     moe_ep_expert_ffn,
     moe_ep_ffn_splits,
+    moe_ep_output_bf16,
     moe_ep_recv_rows,
     moe_ep_workspace_size,
     moe_expert_ffn,

@@ -32,7 +32,8 @@ ABI_FUNCTIONS = ("moe_workspace_size", "moe_workspace_size_ex", "moe_route", "mo
                  "moe_expert_ffn_static", "moe_expert_ffn_static_bytes",
                  "moe_expert_ffn_static_error", "moe_forward_variant", "moe_route_variant",
                  "moe_forward_fp8", "moe_forward_fp8_traced", "moe_ep_recv_rows",
-                 "moe_ep_workspace_size", "moe_ep_ffn_splits", "moe_ep_dispatch",
+                 "moe_ep_workspace_size", "moe_ep_ffn_splits", "moe_ep_output_bf16",
+                 "moe_ep_dispatch",
                  "moe_ep_expert_ffn", "moe_ep_combine", "moe_ipc_get_handle",
                  "moe_ipc_open_handle", "moe_ipc_close", "moe_selftest_wait_timeout")
 TRACE_EVENTS = 6
@@ -99,8 +100,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
             "moe_ep_workspace_size": (_SZ, [_I] * 6),
             "moe_ep_ffn_splits": (_I, [_I] * 4),
             "moe_ep_dispatch": (_I, [_I] * 6 + [_P] * 4 + [_I] + [_P] * 3 + [_SZ, _P]),
-            "moe_ep_expert_ffn": (_I, [_I] * 8 + [_P] * 7 + [_SZ, _P]),
-            "moe_ep_combine": (_I, [_I] * 7 + [_P] * 6 + [_P]),
+            "moe_ep_output_bf16": (_I, [_I] * 4),
+            "moe_ep_expert_ffn": (_I, [_I] * 9 + [_P] * 7 + [_SZ, _P]),
+            "moe_ep_combine": (_I, [_I] * 8 + [_P] * 6 + [_P]),
             "moe_ipc_get_handle": (_I, [_P, _P, _P]),
             "moe_ipc_open_handle": (_I, [_P, _P]),
             "moe_ipc_close": (_I, [_P]),
@@ -317,23 +319,27 @@ def moe_ep_dispatch(T, d, E, k, R, rank, x, idx, counts_all, recv_x, recv_rows, 
                                           _ws_bytes(ws), _stream(stream)), "moe_ep_dispatch")
 
 
-def moe_ep_expert_ffn(T_max, d, E, d_ff, k, R, rows_hint, ksplit, recv_x, recv_offsets, W1, W3,
-                      W2, recv_y, ws, stream=None):
+def moe_ep_output_bf16(rows_hint, d, E_local, d_ff) -> int:
+    return int(load_library().moe_ep_output_bf16(rows_hint, d, E_local, d_ff))
+
+
+def moe_ep_expert_ffn(T_max, d, E, d_ff, k, R, rows_hint, ksplit, y_bf16, recv_x, recv_offsets,
+                      W1, W3, W2, recv_y, ws, stream=None):
     _check(load_library().moe_ep_expert_ffn(T_max, d, E, d_ff, k, R, rows_hint, ksplit,
-                                            _ptr(recv_x), _ptr(recv_offsets), _ptr(W1), _ptr(W3),
-                                            _ptr(W2), _ptr(recv_y), _ptr(ws), _ws_bytes(ws),
-                                            _stream(stream)), "moe_ep_expert_ffn")
+                                            int(y_bf16), _ptr(recv_x), _ptr(recv_offsets),
+                                            _ptr(W1), _ptr(W3), _ptr(W2), _ptr(recv_y), _ptr(ws),
+                                            _ws_bytes(ws), _stream(stream)), "moe_ep_expert_ffn")
 
 
-def moe_ep_combine(T, d, E, k, R, recv_rows, ksplit, idx, pos_of_slot, w, recv_y, shared_y, out,
-                   stream=None):
+def moe_ep_combine(T, d, E, k, R, recv_rows, ksplit, y_bf16, idx, pos_of_slot, w, recv_y,
+                   shared_y, out, stream=None):
     """``recv_y``: the R ranks' output buffers, in rank order."""
     if len(recv_y) != R:
         raise ValueError(f"need {R} output buffers")
-    _check(load_library().moe_ep_combine(T, d, E, k, R, recv_rows, ksplit, _ptr(idx),
-                                         _ptr(pos_of_slot), _ptr(w), _ptr_array(recv_y),
-                                         _ptr(shared_y), _ptr(out), _stream(stream)),
-           "moe_ep_combine")
+    _check(load_library().moe_ep_combine(T, d, E, k, R, recv_rows, ksplit, int(y_bf16),
+                                         _ptr(idx), _ptr(pos_of_slot), _ptr(w),
+                                         _ptr_array(recv_y), _ptr(shared_y), _ptr(out),
+                                         _stream(stream)), "moe_ep_combine")
 
 
 def moe_ipc_get_handle(dev_ptr) -> tuple[bytes, int]:

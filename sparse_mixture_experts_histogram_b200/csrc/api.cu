@@ -988,6 +988,14 @@ int moe_ep_ffn_splits(int rows_hint, int d, int E_local, int d_ff)
     return down_ksplit(rows_hint, E_local, d, d_ff);
 }
 
+int moe_ep_output_bf16(int rows_hint, int d, int E_local, int d_ff)
+{
+    // The CTA-pair kernel writes complete rows (it never splits K), so they
+    // can be bf16; the split-K kernel writes fp32 partials.
+    const int ks = moe_ep_ffn_splits(rows_hint, d, E_local, d_ff);
+    return ks == 1 && ffn_pair_eligible(rows_hint, E_local, 1) ? 1 : 0;
+}
+
 moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank, const moe_bf16 *x,
                            const int32_t *idx, const int32_t *counts_all,
                            moe_bf16 *const *recv_x, int recv_rows, int32_t *pos_of_slot,
@@ -1033,9 +1041,10 @@ moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank, const mo
 }
 
 moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R, int rows_hint,
-                             int ksplit, const moe_bf16 *recv_x, const int32_t *recv_offsets,
-                             const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2,
-                             float *recv_y, void *ws, size_t ws_bytes, moe_stream_t stream)
+                             int ksplit, int y_bf16, const moe_bf16 *recv_x,
+                             const int32_t *recv_offsets, const moe_bf16 *W1, const moe_bf16 *W3,
+                             const moe_bf16 *W2, void *recv_y, void *ws, size_t ws_bytes,
+                             moe_stream_t stream)
 {
     moe_status st = ep_check(T_max, d, E, d_ff, k, R);
     if (st != MOE_OK) return st;
@@ -1043,6 +1052,8 @@ moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R, in
     const int recv_rows = moe_ep_recv_rows(T_max, E, k, R);
     if (recv_rows < 1 || rows_hint < 1) return MOE_ERR_INVALID_ARG;
     if (ksplit != moe_ep_ffn_splits(rows_hint, d, E_local, d_ff)) return MOE_ERR_INVALID_ARG;
+    if (y_bf16 != 0 && (y_bf16 != 1 || !moe_ep_output_bf16(rows_hint, d, E_local, d_ff)))
+        return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(recv_x) || !ok_ptr(recv_offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
         !ok_ptr(recv_y) || !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
@@ -1068,7 +1079,8 @@ moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R, in
     f.W2 = W2;
     f.x = recv_x;
     f.H = reinterpret_cast<moe_bf16 *>(wsb + L.H);
-    f.Y = recv_y;
+    f.Y = static_cast<float *>(recv_y);
+    f.y_bf16 = y_bf16 != 0;
     f.h_ready = reinterpret_cast<uint32_t *>(wsb + L.ffnctr + kAlign);
     f.sched = reinterpret_cast<uint32_t *>(wsb + L.ffnctr);
     f.err = reinterpret_cast<uint32_t *>(wsb);
@@ -1078,12 +1090,13 @@ moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, int R, in
 }
 
 moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int ksplit,
-                          const int32_t *idx, const int32_t *pos_of_slot, const float *w,
-                          const float *const *recv_y, const float *shared_y, float *out,
-                          moe_stream_t stream)
+                          int y_bf16, const int32_t *idx, const int32_t *pos_of_slot,
+                          const float *w, const void *const *recv_y, const float *shared_y,
+                          float *out, moe_stream_t stream)
 {
     if (T < 1 || d < 1 || E < 1 || k < 1 || R < 1 || recv_rows < 1 || ksplit < 1)
         return MOE_ERR_INVALID_ARG;
+    if (y_bf16 != 0 && (y_bf16 != 1 || ksplit != 1)) return MOE_ERR_INVALID_ARG;
     if (R > kMaxRanksHost || k > 8 || T > (1 << 24) || d % 128 || d > 16384 || E > 256 ||
         ksplit > 8)
         return MOE_ERR_UNSUPPORTED;
@@ -1105,6 +1118,7 @@ moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int 
     c.pos_of_slot = pos_of_slot;
     c.w = w;
     c.recv_y = recv_y;
+    c.y_bf16 = y_bf16 != 0;
     c.shared_y = shared_y;
     c.out = out;
     return from_cuda(launch_ep_combine(c, reinterpret_cast<cudaStream_t>(stream)));

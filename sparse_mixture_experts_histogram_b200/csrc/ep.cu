@@ -13,8 +13,9 @@
 //    block's first row + the pair's rank in token order.  The scatter of the
 //    single-GPU layer and the all-to-all of rows are one pass over x.
 //  * ep_combine_kernel: each slot's expert output row is loaded from its
-//    owner's output buffer (peer memory) and the k rows are summed,
-//    gate-weighted, in slot order.
+//    owner's output buffer (peer memory; bf16 rows where the owner's expert
+//    kernel wrote complete sums, which halves what crosses NVLink on the way
+//    back) and the k rows are summed, gate-weighted, in slot order.
 //
 // Receive layout on owner q: its experts in index order; inside an expert,
 // the rows sent by rank 0, then rank 1, ...; inside one sender, token order.
@@ -253,7 +254,8 @@ struct EpCombineParams {
     int recv_rows;
     const int32_t *idx, *pos_of_slot;
     const float *w;
-    const float4 *y[kMaxRanks];  // every rank's output buffer [ksplit, recv_rows, d] fp32
+    const void *y[kMaxRanks];    // every rank's output buffer [ksplit, recv_rows, d], fp32
+                                 // or bf16 (kernel template; ksplit 1)
     const float4 *shared_y;      // [T, d] or nullptr
     float4 *out;
     int chunks;              // chunks of 32*kEpOutVec float4 per row
@@ -262,11 +264,25 @@ struct EpCombineParams {
 constexpr int kEpOutVec = 2;
 constexpr int kEpBatch = 4;  // (slot, partial) rows whose loads are in flight together
 
+// Four consecutive elements (group i of 4) of an fp32 or a bf16 array.
+template <bool BF>
+__device__ __forceinline__ float4 load_y4(const void *base, size_t i)
+{
+    if constexpr (BF) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(base) + i);
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+    } else {
+        return __ldg(reinterpret_cast<const float4 *>(base) + i);
+    }
+}
+
 // One warp per (token, chunk): y_j = sum of the K-split partials of slot j's
 // row (in order), out = sum_j w_j * y_j in slot order (+ shared_y).  The
 // (slot, partial) pairs are visited slot-major in batches of kEpBatch whose
 // loads are all issued before any is used; the order of every addition is
 // fixed.
+template <bool BF>
 __global__ void __launch_bounds__(32 * kEpWarps) ep_combine_kernel(const __grid_constant__ EpCombineParams p)
 {
     const int lane = threadIdx.x & 31;
@@ -320,12 +336,12 @@ __global__ void __launch_bounds__(32 * kEpWarps) ep_combine_kernel(const __grid_
             const int pos = __shfl_sync(0xffffffffu, my_pos, jj[i] & 31);
             const int q = __shfl_sync(0xffffffffu, my_q, jj[i] & 31);
             const bool ok = pi < npairs && pos >= 0;
-            const float4 *row = pick_rank(p.y, q) + ss[i] * p.part_stride +
-                                static_cast<size_t>(ok ? pos : 0) * nv;
+            const void *yq = pick_rank(p.y, q);
+            const size_t row = ss[i] * p.part_stride + static_cast<size_t>(ok ? pos : 0) * nv;
 #pragma unroll
             for (int u = 0; u < kEpOutVec; ++u) {
                 const int v = (c * kEpOutVec + u) * 32 + lane;
-                val[i][u] = (ok && v < nv) ? __ldg(row + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                val[i][u] = (ok && v < nv) ? load_y4<BF>(yq, row + v) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
 #pragma unroll
@@ -441,20 +457,22 @@ cudaError_t launch_ep_combine(const EpCombineLaunch &a, cudaStream_t s)
     p.k = a.k;
     p.El = a.E / a.R;
     p.ksplit = a.ksplit < 1 ? 1 : a.ksplit;
+    if (a.y_bf16 && p.ksplit != 1) return cudaErrorInvalidValue;
     p.recv_rows = a.recv_rows;
     p.part_stride = static_cast<size_t>(a.recv_rows) * (a.d / 4);
     p.idx = a.idx;
     p.pos_of_slot = a.pos_of_slot;
     p.w = a.w;
     for (int r = 0; r < kMaxRanks; ++r)
-        p.y[r] = reinterpret_cast<const float4 *>(r < a.R ? a.recv_y[r] : a.recv_y[0]);
+        p.y[r] = r < a.R ? a.recv_y[r] : a.recv_y[0];
     p.shared_y = reinterpret_cast<const float4 *>(a.shared_y);
     p.out = reinterpret_cast<float4 *>(a.out);
     const int nv = a.d / 4;
     p.chunks = (nv + 32 * kEpOutVec - 1) / (32 * kEpOutVec);
     const long long warps = static_cast<long long>(a.T) * p.chunks;
     const int blocks = static_cast<int>((warps + kEpWarps - 1) / kEpWarps);
-    ep_combine_kernel<<<blocks, 32 * kEpWarps, 0, s>>>(p);
+    if (a.y_bf16) ep_combine_kernel<true><<<blocks, 32 * kEpWarps, 0, s>>>(p);
+    else ep_combine_kernel<false><<<blocks, 32 * kEpWarps, 0, s>>>(p);
     return cudaGetLastError();
 }
 

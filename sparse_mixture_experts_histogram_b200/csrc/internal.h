@@ -149,7 +149,8 @@ struct EpCombineLaunch {
     int ksplit;                  // partial outputs per receive row
     const int32_t *idx, *pos_of_slot;
     const float *w;
-    const float *const *recv_y;  // [R] host array of device addresses
+    const void *const *recv_y;   // [R] host array of device addresses
+    bool y_bf16;                 // the output buffers hold bf16 rows (ksplit 1), not fp32
     const float *shared_y;       // [T, d] or nullptr
     float *out;
 };

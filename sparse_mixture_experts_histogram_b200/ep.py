@@ -40,7 +40,7 @@ def expert_block(E: int, R: int, rank: int) -> tuple[int, int]:
 class _Rank:
     """Buffers of one rank for tokens of at most T_max rows."""
     recv_x: torch.Tensor      # [recv_rows, d] bf16 (peers store into it)
-    recv_y: torch.Tensor      # [ksplit, recv_rows, d] fp32 (peers read from it)
+    recv_y: torch.Tensor      # [ksplit, recv_rows, d] fp32, or bf16 with ksplit 1 (peers read it)
     ws: torch.Tensor          # moe_ep_workspace_size bytes
     route_ws: torch.Tensor    # moe_workspace_size bytes (router)
     idx: torch.Tensor         # [T_max, k] int32
@@ -70,6 +70,8 @@ class _Plan:
         # pairs, spread over R owners.
         self.rows_hint = max(1, T_max * k)
         self.ksplit = B.moe_ep_ffn_splits(self.rows_hint, d, self.El, d_ff)
+        # Complete rows (no K split) come back as bf16: half the bytes.
+        self.y_bf16 = B.moe_ep_output_bf16(self.rows_hint, d, self.El, d_ff) == 1
 
     def alloc(self, device) -> _Rank:
         kw = dict(device=device)
@@ -80,7 +82,8 @@ class _Plan:
             shared_ws = torch.empty(need, dtype=torch.uint8, **kw)
         return _Rank(
             recv_x=torch.empty(self.recv_rows, self.d, dtype=torch.bfloat16, **kw),
-            recv_y=torch.empty(self.ksplit, self.recv_rows, self.d, dtype=torch.float32, **kw),
+            recv_y=torch.empty(self.ksplit, self.recv_rows, self.d,
+                               dtype=torch.bfloat16 if self.y_bf16 else torch.float32, **kw),
             ws=torch.empty(self.ws_bytes, dtype=torch.uint8, **kw),
             route_ws=torch.empty(B.moe_workspace_size(self.T_max, self.d, self.E, 128, self.k),
                                  dtype=torch.uint8, **kw),
@@ -124,12 +127,12 @@ def _dispatch(p: _Plan, b: _Rank, rank, x, counts_all, recv_x_all):
 
 
 def _ffn(p: _Plan, b: _Rank, W1, W3, W2):
-    B.moe_ep_expert_ffn(p.T_max, p.d, p.E, p.d_ff, p.k, p.R, p.rows_hint, p.ksplit, b.recv_x,
-                        b.recv_offsets, W1, W3, W2, b.recv_y, b.ws)
+    B.moe_ep_expert_ffn(p.T_max, p.d, p.E, p.d_ff, p.k, p.R, p.rows_hint, p.ksplit, p.y_bf16,
+                        b.recv_x, b.recv_offsets, W1, W3, W2, b.recv_y, b.ws)
 
 
 def _combine(p: _Plan, b: _Rank, T, recv_y_all, shared_y, out):
-    B.moe_ep_combine(T, p.d, p.E, p.k, p.R, p.recv_rows, p.ksplit, b.idx, b.pos, b.w,
+    B.moe_ep_combine(T, p.d, p.E, p.k, p.R, p.recv_rows, p.ksplit, p.y_bf16, b.idx, b.pos, b.w,
                      recv_y_all, shared_y, out)
 
 

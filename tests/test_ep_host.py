@@ -63,16 +63,22 @@ def test_dispatch_checks_its_arguments_on_the_host(lib):
 def test_expert_ffn_and_combine_check_their_arguments(lib):
     import ctypes
     ks = moe.moe_ep_ffn_splits(4 * 2, 512, 4, 1024)
-    args = lambda ksplit, R=2: (4, 512, 8, 1024, 2, R, 8, ksplit) + (FAKE,) * 7 + (1 << 40, None)
+    args = lambda ksplit, R=2, bf=0: ((4, 512, 8, 1024, 2, R, 8, ksplit, bf) + (FAKE,) * 7 +
+                                      (1 << 40, None))
     assert lib.moe_ep_expert_ffn(*args(ks + 1)) == 1    # ksplit not the library's
     assert lib.moe_ep_expert_ffn(*args(ks, R=3)) == 1   # E % R
+    assert moe.moe_ep_output_bf16(8, 512, 4, 1024) == 0  # decode-sized: split K, fp32 partials
+    assert lib.moe_ep_expert_ffn(*args(ks, bf=1)) == 1  # bf16 rows not available here
+    assert moe.moe_ep_output_bf16(4096, 4096, 1, 14336) == 1
     ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)
-    comb = lambda R=2, ksplit=1, E=8: lib.moe_ep_combine(4, 512, E, 2, R, 64, ksplit, FAKE, FAKE,
-                                                         FAKE, ptrs, None, FAKE, None)
+    comb = lambda R=2, ksplit=1, E=8, bf=0: lib.moe_ep_combine(4, 512, E, 2, R, 64, ksplit, bf,
+                                                               FAKE, FAKE, FAKE, ptrs, None, FAKE,
+                                                               None)
     assert comb(R=9) == 2
     assert comb(E=6, R=4) == 1
     assert comb(ksplit=0) == 1
     assert comb(ksplit=9) == 2
+    assert comb(ksplit=2, bf=1) == 1                    # bf16 rows hold complete sums only
 
 
 def test_expert_blocks_tile_the_experts():

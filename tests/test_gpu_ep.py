@@ -116,10 +116,10 @@ def test_ep_decode_splits_the_down_projection():
 
 def test_ep_prefill_tiles():
     """Prefill-sized segments (about 1000 rows per expert): the owners run
-    the CTA-pair expert kernel."""
+    the CTA-pair expert kernel and hand back bf16 rows."""
     R, Ts, d, E, d_ff, k = 2, [1024, 1000], 2048, 4, 1024, 2
     layer, inp, xs, outs = _run("ep_prefill", R, Ts, d, E, d_ff, k)
-    assert layer.plan.ksplit == 1
+    assert layer.plan.ksplit == 1 and layer.plan.y_bf16   # complete rows come back as bf16
     idx = _check_layout(layer, xs)
     _check_outputs(layer, inp, xs, outs, idx, tokens_per_rank=48)
 
