@@ -414,6 +414,8 @@ MOE_API int moe_ep_ffn_splits(int rows_hint, int d, int E_local, int d_ff);
  *   expert idx[t,j]; recv_offsets [E/R+1] int32 out: segment starts of this
  *   rank's experts in its own recv_x (valid once every rank's counts are in
  *   counts_all, which they are after step 2).
+ * T may be 0 (a rank with no tokens in this step: x, idx and pos_of_slot
+ * are then not read; it sends nothing but still gets its receive segments).
  * If counts_all's own row differs from the counts of idx, or some owner
  * would receive more than recv_rows rows, MOE_DEVERR_EP_COUNTS is set in the
  * workspace's error word, nothing is sent and pos_of_slot is all -1.  Resets
@@ -448,7 +450,8 @@ MOE_API moe_status moe_ep_expert_ffn(int T_max, int d, int E, int d_ff, int k, i
  * (+ shared_y[t]), o = owner of idx[t,j], slots in order j = 0..k-1, the K
  * split partials q in order.  recv_y: host array of R device addresses of
  * the ranks' output buffers, fp32, or bf16 rows with y_bf16 = 1 (ksplit 1).
- * A slot with pos_of_slot -1 adds nothing.  out [T,d] fp32 (overwritten). */
+ * A slot with pos_of_slot -1 adds nothing.  out [T,d] fp32 (overwritten).
+ * T = 0 does nothing. */
 MOE_API moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int ksplit,
                                   int y_bf16, const int32_t *idx, const int32_t *pos_of_slot,
                                   const float *w, const void *const *recv_y,

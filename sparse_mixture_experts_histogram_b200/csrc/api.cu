@@ -1001,15 +1001,19 @@ moe_status moe_ep_dispatch(int T, int d, int E, int k, int R, int rank, const mo
                            moe_bf16 *const *recv_x, int recv_rows, int32_t *pos_of_slot,
                            int32_t *recv_offsets, void *ws, size_t ws_bytes, moe_stream_t stream)
 {
-    moe_status st = ep_check(T, d, E, 128, k, R);
+    // A rank may have no tokens in a step: it sends nothing but still owns
+    // experts, so its plan (its receive segments) is computed all the same.
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    const int Tl = T > 0 ? T : 1;  // sizes of the checks and of the workspace layout
+    moe_status st = ep_check(Tl, d, E, 128, k, R);
     if (st != MOE_OK) return st;
     if (rank < 0 || rank >= R || recv_rows < 1 || recv_x == nullptr) return MOE_ERR_INVALID_ARG;
-    if (!ok_ptr(x) || !ok_ptr(idx) || !ok_ptr(counts_all) || !ok_ptr(pos_of_slot) ||
+    if ((T > 0 && (!ok_ptr(x) || !ok_ptr(idx) || !ok_ptr(pos_of_slot))) || !ok_ptr(counts_all) ||
         !ok_ptr(recv_offsets) || !ok_ptr(ws))
         return MOE_ERR_INVALID_ARG;
     for (int r = 0; r < R; ++r)
         if (!ok_ptr(recv_x[r])) return MOE_ERR_INVALID_ARG;
-    const EpLayout L = ep_layout(T, T, E, 128, k, R);
+    const EpLayout L = ep_layout(Tl, Tl, E, 128, k, R);
     if (ws_bytes < L.disp_end) return MOE_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
@@ -1094,6 +1098,7 @@ moe_status moe_ep_combine(int T, int d, int E, int k, int R, int recv_rows, int 
                           const float *w, const void *const *recv_y, const float *shared_y,
                           float *out, moe_stream_t stream)
 {
+    if (T == 0 && d >= 1 && E >= 1 && k >= 1 && R >= 1) return MOE_OK;  // no tokens, no rows
     if (T < 1 || d < 1 || E < 1 || k < 1 || R < 1 || recv_rows < 1 || ksplit < 1)
         return MOE_ERR_INVALID_ARG;
     if (y_bf16 != 0 && (y_bf16 != 1 || ksplit != 1)) return MOE_ERR_INVALID_ARG;

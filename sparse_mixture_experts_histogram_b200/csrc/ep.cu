@@ -411,7 +411,9 @@ cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s)
     pp.dout.offsets = a.offsets;
     pp.dout.counts = nullptr;
     pp.dout.done = a.done;
-    pp.dout.ntiles = (a.T + kTileTokens - 1) / kTileTokens;
+    // T = 0: one CTA with no tokens still computes the plan (zero counts of
+    // its own, the receive segments it owns).
+    pp.dout.ntiles = a.T > 0 ? (a.T + kTileTokens - 1) / kTileTokens : 1;
     pp.dout.cap = -1;
     pp.base = a.base;
     pp.recv_offsets = a.recv_offsets;
@@ -419,7 +421,7 @@ cudaError_t launch_ep_dispatch(const EpDispatchLaunch &a, cudaStream_t s)
     pp.err = a.err;
     ep_ranks_plan_kernel<<<pp.dout.ntiles, kTileTokens, 0, s>>>(pp);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || a.T == 0) return e;
 
     EpDispatchParams p{};
     p.T = a.T;

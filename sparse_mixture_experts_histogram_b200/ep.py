@@ -102,12 +102,15 @@ def _route(p: _Plan, b: _Rank, x, Wg, router_bias, counts_out):
     T = x.shape[0]
     if T > p.T_max:
         raise ValueError(f"{T} tokens > T_max={p.T_max}")
+    if T == 0:
+        counts_out.zero_()  # a rank with no tokens this step still takes part
+        return
     B.moe_route(T, p.d, p.E, p.k, x, Wg, router_bias, b.idx, b.w, counts_out, b.route_ws)
 
 
 def _shared(p: _Plan, b: _Rank, x, shared):
     """The always-on expert on this rank's own tokens (weights replicated)."""
-    if shared is None:
+    if shared is None or x.shape[0] == 0:
         return None
     T = x.shape[0]
     # [0, T] as the one segment's bounds, set by a device fill (no host copy,

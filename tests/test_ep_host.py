@@ -56,6 +56,12 @@ def test_dispatch_checks_its_arguments_on_the_host(lib):
     assert _dispatch(lib, rank=-1) == 1
     assert _dispatch(lib, recv=0) == 1       # no receive table
     assert _dispatch(lib, rows=0) == 1
+    assert _dispatch(lib, T=-1) == 1
+    # no tokens on this rank: combine has nothing to do (no GPU work)
+    import ctypes
+    ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert lib.moe_ep_combine(0, 512, 8, 2, 2, 64, 1, 0, None, None, None, ptrs, None, None,
+                              None) == 0
     assert _dispatch(lib, d=500) == 2        # d % 128
     assert _dispatch(lib, ws_bytes=16) == 3  # workspace too small
 
